@@ -1,0 +1,450 @@
+"""Throughput of the MoE token shuffle (plan + dispatch + combine) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config dsv3] [--impl ours|reference]
+
+One step = one pass of the whole path over one batch: moe_plan (histogram, scan, stable
+slots, per-rank dedup lists), moe_dispatch (token-major -> expert-major rows) and
+moe_combine (weighted gather-reduce back to token order), all on inputs resident in HBM.
+The metric is effective HBM GB/s over the algorithmic bytes of dispatch + combine
+(each x row read once, each receive row written once, each y row read once, each out
+row written once, plus slots and weights), also given as % of the HBM roofline and as
+tokens/s.  With N > 1 (torchrun) every GPU runs an independent replica of the same
+workload (the path has no exchange step), timed on the device; the job value is the sum
+of all ranks' bytes over the slowest rank's time.
+
+--impl reference times the CPU oracle (single thread, the machine's host core) on a bounded
+token sample of the same workload and prints the same metric.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import CONFIGS, Config, make_payload_x, make_payload_y, make_routing  # noqa: E402
+
+METRIC = "dispatch+combine effective HBM GB/s and % of B200 roofline; tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------- bytes
+def dispatch_bytes(cfg: Config, N: int | None = None) -> int:
+    """x rows read once, N*k receive rows written once, N*k slots read."""
+    N = cfg.N if N is None else N
+    return N * cfg.row_bytes + N * cfg.k * cfg.row_bytes + 4 * N * cfg.k
+
+
+def combine_bytes(cfg: Config, N: int | None = None) -> int:
+    """N*k bf16 rows of y read, N bf16 out rows written, slots and weights read."""
+    N = cfg.N if N is None else N
+    return 2 * N * cfg.k * cfg.H + 2 * N * cfg.H + 8 * N * cfg.k
+
+
+def plan_bytes(cfg: Config, N: int | None = None) -> int:
+    """ids read; slot, src_tok, src_j written; dedup lists (at most N*min(k,R)) written."""
+    N = cfg.N if N is None else N
+    return 4 * N * cfg.k * 4 + 8 * N * min(cfg.k, cfg.R)
+
+
+def workload_name(cfg: Config) -> str:
+    return (f"{cfg.name}: N={cfg.N} H={cfg.H} E={cfg.E} k={cfg.k} R={cfg.R} "
+            f"{cfg.payload} routing={cfg.routing} weights={cfg.weights} experts={cfg.y}")
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_traffic(kernel: str, units: int):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for rel in rec["sources"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec["sources_sha256"]:
+        return None
+    return rec["bytes_per_unit"] * units
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 100):
+        self.gpu = gpu_index
+        self.period = period_ms
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{self.gpu}.csv")
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", str(self.period)],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, v in enumerate(flags)
+                          if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------ ours
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_ours(args):
+    import moe_expert_shuffling_b200 as ms
+    from moe_expert_shuffling_b200 import build as lib_build
+
+    lib_build.build()
+    world, rank, local = dist_setup(args)
+    cfg = CONFIGS[args.config]
+    seed = args.seed + rank
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
+
+    idx_h, w_h = make_routing(cfg, seed)
+    with torch.cuda.stream(stream):
+        x, xs = make_payload_x(cfg, seed, dev)
+        y = make_payload_y(cfg, seed, dev)
+        idx = torch.from_numpy(idx_h).to(dev)
+        w = torch.from_numpy(w_h).to(dev)
+        recv = torch.empty((cfg.N * cfg.k, cfg.H), dtype=x.dtype, device=dev)
+        rs = (torch.empty((cfg.N * cfg.k, cfg.H // 128), dtype=torch.float32, device=dev)
+              if cfg.payload == "fp8" else None)
+        out = torch.empty((cfg.N, cfg.H), dtype=torch.bfloat16, device=dev)
+    stream.synchronize()
+    identity = y is None
+    plan = ms.moe_plan_create(cfg.N, cfg.k, cfg.E, cfg.R)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ms.moe_plan(idx, w, cfg.E, cfg.R, plan=plan, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if rs is not None:
+            ms.moe_dispatch(x, plan, recv=recv, x_scale=xs, recv_scale=rs, stream=stream)
+        else:
+            ms.moe_dispatch(x, plan, recv=recv, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        ms.moe_combine(recv if identity else y, plan, out=out, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    stream.synchronize()
+    if plan.check(stream) != 0:
+        raise SystemExit("device reported invalid routing or a timeout")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    elapsed_ms = evs[0][0].elapsed_time(evs[-1][3])
+    t_plan = [e[0].elapsed_time(e[1]) for e in evs]
+    t_disp = [e[1].elapsed_time(e[2]) for e in evs]
+    t_comb = [e[2].elapsed_time(e[3]) for e in evs]
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    ms_per_step = elapsed_ms / args.steps
+
+    db, cb = dispatch_bytes(cfg), combine_bytes(cfg)
+    job_bytes = (db + cb) * args.steps * world
+    value = job_bytes / (elapsed_ms * 1e-3) / 1e9
+    tokens_per_s = cfg.N * args.steps * world / (elapsed_ms * 1e-3)
+    peak, peak_kind = measured_hbm_peak()
+    disp_us = 1e3 * statistics.mean(t_disp)
+    comb_us = 1e3 * statistics.mean(t_comb)
+    plan_us = 1e3 * statistics.mean(t_plan)
+    if disp_us >= comb_us:
+        dom, dom_bytes, dom_us = "dispatch_bulk_kernel", db, disp_us
+    else:
+        dom, dom_bytes, dom_us = "combine_kernel", cb, comb_us
+    achieved = dom_bytes / (dom_us * 1e-6) / 1e9
+    launches_per_step = 5 + (1 if cfg.payload == "fp8" and (4 * (cfg.H // 128)) % 16 else 0)
+
+    # end to end: pinned host inputs -> device, step, result -> pinned host
+    e2e = None
+    if args.e2e_steps > 0:
+        idx_p = torch.from_numpy(idx_h).pin_memory()
+        w_p = torch.from_numpy(w_h).pin_memory()
+        x_p = x.cpu().pin_memory()
+        xs_p = xs.cpu().pin_memory() if xs is not None else None
+        y_p = y.cpu().pin_memory() if y is not None else None
+        out_p = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (idx_p, w_p, x_p, xs_p, y_p) if t is not None)
+        d2h = out_p.numel() * out_p.element_size()
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                idx.copy_(idx_p, non_blocking=True)
+                w.copy_(w_p, non_blocking=True)
+                x.copy_(x_p, non_blocking=True)
+                if xs_p is not None:
+                    xs.copy_(xs_p, non_blocking=True)
+                if y_p is not None:
+                    y.copy_(y_p, non_blocking=True)
+            step()
+            with torch.cuda.stream(stream):
+                out_p.copy_(out, non_blocking=True)
+
+        e2e_step()
+        stream.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        b.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b), world)
+        e2e = {"value": round((db + cb) * args.e2e_steps * world / (e_ms * 1e-3) / 1e9, 3),
+               "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(e_ms / args.e2e_steps, 3), "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        cpu = cpu_baseline(cfg, idx_h, w_h, x, xs, y, recv, args.cpu_seconds)
+
+    plan.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.payload == "bf16" else "fp8e4m3", "accum_dtype": "f32",
+        "data": "synthetic (seeded routing and N(0,1) payload; no traces or weights exist)",
+        "config": {"workload": workload_name(cfg), "model": f"{cfg.name}-shaped MoE layer shuffle",
+                   "global_batch": cfg.N * world, "seq_len": cfg.N, "parallelism": f"replicas{world}",
+                   "ep_ranks_logical": cfg.R,
+                   "l2": "no flush: every input (x, y) and output is larger than the 126 MB L2"},
+        "tokens_per_s": round(tokens_per_s, 1),
+        "pct_roofline": {"of_nominal_8000": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+                         f"of_{peak_kind}_{peak:g}": round(100 * value / world / peak, 2)},
+        "kernels_us": {"plan": round(plan_us, 2), "dispatch": round(disp_us, 2),
+                       "combine": round(comb_us, 2)},
+        "kernels_gbs": {"dispatch": round(db / (disp_us * 1e-6) / 1e9, 1),
+                        "combine": round(cb / (comb_us * 1e-6) / 1e9, 1),
+                        "plan": round(plan_bytes(cfg) / (plan_us * 1e-6) / 1e9, 1)},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "traffic": kernel_traffic(dom, cfg.N)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------ CPU oracle
+def oracle_sample_step(cfg: Config, idx_h, w_h, x_bytes, xs_bytes, y_bits, n):
+    """One oracle plan + dispatch + combine over the first n tokens of the workload."""
+    import oracle
+    p = oracle.plan(idx_h[:n], cfg.E, cfg.R)
+    if xs_bytes is not None:
+        recv, _ = oracle.dispatch(x_bytes[:n], p.slot, xs_bytes[:n])
+    else:
+        recv = oracle.dispatch(x_bytes[:n], p.slot)
+    y = recv.view(np.uint16).reshape(n * cfg.k, cfg.H) if y_bits is None else y_bits[:n * cfg.k]
+    oracle.combine(y, p.slot, w_h[:n])
+
+
+def host_payload(cfg: Config, x, xs, y, n_tokens):
+    def bits16(t):
+        return t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    if cfg.payload == "fp8":
+        xb = x[:n_tokens].cpu().numpy()
+        xsb = xs[:n_tokens].cpu().numpy().view(np.uint8)
+    else:
+        xb = bits16(x[:n_tokens]).view(np.uint8).reshape(n_tokens, -1)
+        xsb = None
+    yb = bits16(y[:n_tokens * cfg.k]) if y is not None else None
+    return xb, xsb, yb
+
+
+def cpu_baseline(cfg, idx_h, w_h, x, xs, y, recv, seconds):
+    """Time the oracle as it stands on a token sample sized for about `seconds` of work."""
+    n_max = min(cfg.N, 4096)
+    xb, xsb, yb = host_payload(cfg, x, xs, y, n_max)
+    n = min(64, n_max)
+    t0 = time.perf_counter()
+    oracle_sample_step(cfg, idx_h, w_h, xb, xsb, yb, n)
+    dt = time.perf_counter() - t0
+    n = int(max(16, min(n_max, n * (seconds / 3) / max(dt, 1e-6))))
+    reps, total_t = 0, 0.0
+    while total_t < seconds * 0.66 and reps < 50:
+        t0 = time.perf_counter()
+        oracle_sample_step(cfg, idx_h, w_h, xb, xsb, yb, n)
+        total_t += time.perf_counter() - t0
+        reps += 1
+    gbs = (dispatch_bytes(cfg, n) + combine_bytes(cfg, n)) * reps / total_t / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {n} of {cfg.N} tokens (same routing and payload), {reps} "
+                      f"plan+dispatch+combine passes, {total_t:.1f} s, single-threaded C"}
+
+
+def run_reference(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    cfg = CONFIGS[args.config]
+    idx_h, w_h = make_routing(cfg, args.seed)
+    n_max = min(cfg.N, 4096)
+    cfg_s = cfg.with_tokens(n_max)
+    x, xs = make_payload_x(cfg_s, args.seed, "cpu")
+    y = make_payload_y(cfg_s, args.seed, "cpu")
+    xb, xsb, yb = host_payload(cfg_s, x, xs, y, n_max)
+    # size the per-step sample so that warmup + steps take about args.ref_seconds
+    n = min(64, n_max)
+    t0 = time.perf_counter()
+    oracle_sample_step(cfg, idx_h, w_h, xb, xsb, yb, n)
+    dt = time.perf_counter() - t0
+    per_step = args.ref_seconds / max(1, args.steps + args.warmup)
+    n = int(max(16, min(n_max, n * per_step / max(dt, 1e-6))))
+    for _ in range(args.warmup):
+        oracle_sample_step(cfg, idx_h, w_h, xb, xsb, yb, n)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(cfg, idx_h, w_h, xb, xsb, yb, n)
+    el = time.perf_counter() - t0
+    nbytes = dispatch_bytes(cfg, n) + combine_bytes(cfg, n)
+    value = nbytes * args.steps / el / 1e9
+    sample = (f"first {n} of {cfg.N} tokens per step (same routing; payload drawn on the host), "
+              f"single-threaded C oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * el / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.payload == "bf16" else "fp8e4m3", "accum_dtype": "f32",
+        "data": "synthetic", "config": {"workload": workload_name(cfg)},
+        "tokens_per_s": round(n * args.steps / el, 1),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="dsv3", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=90.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,187 @@
+/*
+ * moe_shuffle.h -- C ABI of the B200 MoE token-shuffle library (libmoeshuffle.so).
+ *
+ * The library moves token rows between a token-major layout and an expert-major,
+ * rank-segmented layout on one GPU, with the layout change done inside the data
+ * movement (FUSCO, arXiv 2512.22036, abstract: the expert-major layout of MoE conflicts
+ * with the device-major layout communication expects, so the shuffle is fused into the
+ * move).  Expert-parallel ranks are logical: rank r owns the contiguous receive rows of
+ * experts r*E/R .. (r+1)*E/R - 1 in one buffer in this GPU's memory.
+ *
+ * Conventions for every call:
+ *   - Pointers named "device" are CUDA device pointers on the current device.  Payload
+ *     arrays (x, recv, y, out) must be 16-byte aligned, routing arrays 4-byte aligned.
+ *     Arrays are dense and row-major.  A plan is used on the device it was created on.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Calls only enqueue work on it; none of them synchronises the host or copies
+ *     device data to the host, except moe_plan_check.
+ *   - Arguments are checked on the host before anything is enqueued; a bad argument
+ *     returns MOE_EINVAL and enqueues nothing.  A CUDA failure returns MOE_ECUDA.
+ *     moe_last_error() then describes the failure (per host thread).
+ *   - Routing ids are checked on the device: an id outside [0,E) or an id repeated
+ *     within one token sets a bit in the plan's error word (read with moe_plan_check);
+ *     the affected entries get slot -1 and are skipped by dispatch and combine, so bad
+ *     routing never makes a kernel touch memory outside the caller's buffers.
+ *
+ * Limits: 1 <= k <= 32, k <= E <= 1024, E % R == 0, 0 <= N, N*k < 2^31.
+ */
+#ifndef MOE_SHUFFLE_H
+#define MOE_SHUFFLE_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_EINVAL = 1,  /* bad argument; nothing was enqueued */
+    MOE_ECUDA = 2,   /* a CUDA runtime call or kernel launch failed */
+    MOE_ENOMEM = 3   /* device allocation failed */
+} moe_status;
+
+typedef enum {
+    MOE_BF16 = 0,    /* 2-byte rows; H % 8 == 0 */
+    MOE_FP8E4M3 = 1  /* 1-byte rows plus one fp32 scale per 128 columns; H % 128 == 0 */
+} moe_dtype;
+
+/* Bits of the plan's device error word. */
+#define MOE_ERR_ID_RANGE 1u   /* a routing id outside [0, E) */
+#define MOE_ERR_ID_DUP 2u     /* a token listed the same expert twice */
+#define MOE_ERR_BOUNDS 4u     /* an internal index fell outside its array (entry skipped) */
+#define MOE_ERR_TIMEOUT 8u    /* a device wait gave up after its iteration limit */
+
+/* Opaque plan: device arrays owned by the library, reusable across calls. */
+typedef struct moe_plan_s *moe_plan_t;
+
+/* Device pointers into a plan (valid until moe_plan_destroy; contents valid once the
+ * stream of the last moe_plan call has reached that point). */
+typedef struct {
+    int32_t N, k, E, R;            /* shape of the last moe_plan call */
+    int32_t experts_per_rank;      /* E / R */
+    int32_t capacity_tokens;       /* largest N this plan accepts */
+    int32_t *cnt;                  /* [E]    entries routed to each expert */
+    int32_t *expert_off;           /* [E+1]  first receive row of each expert segment */
+    int32_t *rcnt;                 /* [R]    tokens that touch rank r (dedup moves) */
+    int32_t *rank_off;             /* [R+1]  first receive row of each rank */
+    int32_t *rtok_off;             /* [R+1]  start of each rank's dedup list */
+    int32_t *slot;                 /* [N*k]  receive row of entry (t, j), or -1 if invalid */
+    int32_t *src_tok;              /* [N*k]  token of each receive row */
+    int32_t *src_j;                /* [N*k]  top-k column of each receive row */
+    int32_t *rtok;                 /* [sum rcnt] tokens of rank r, ascending */
+    uint32_t *fanout;              /* [sum rcnt] bit j: column j of that token is on rank r */
+    uint32_t *err;                 /* [1]    MOE_ERR_* bits of the last moe_plan call */
+    const float *topk_w;           /* the weights given to the last moe_plan call */
+} moe_plan_view;
+
+/*
+ * moe_plan_create -- allocate a plan for up to `max_tokens` tokens of shape (k, E, R).
+ * Allocates device memory once (cudaMalloc); later moe_plan calls reuse it.
+ * On success *out receives the plan.  max_tokens >= 0.
+ */
+MOE_API moe_status moe_plan_create(int32_t max_tokens, int32_t k, int32_t E, int32_t R,
+                           moe_plan_t *out);
+
+/*
+ * moe_plan -- build the logical-segment plan of one routing (FUSCO abstract: the
+ * "lightweight planning" that turns the captured layout into placements and drops
+ * redundant transfers; DySHARP blog, section 5: a destination maps a token's logical
+ * index to its own local address, which is what slot[] is).
+ *
+ *   topk_idx  device int32 [N, k]  expert ids of each token (caller-owned, read here)
+ *   topk_w    device fp32  [N, k]  routing weights; only the pointer is kept, and
+ *                                  moe_combine reads it, so it must stay valid and
+ *                                  unchanged until the last combine using this plan
+ *   N, k, E, R                     tokens, experts per token, experts, ranks
+ *   stream                         cudaStream_t as void*
+ *   plan      in/out: if *plan is NULL a plan sized for N tokens is created (device
+ *             allocation); otherwise *plan is reused and must have been created with
+ *             the same (k, E, R) and capacity >= N, else MOE_EINVAL.
+ *
+ * Computes, for expert e on rank e / (E/R):
+ *   cnt[e], expert_off = exclusive scan of cnt, rank_off[r] = expert_off[r*E/R];
+ *   slot[t,j] = expert_off[e] + #{t' < t : e in topk_idx[t',:]} (stable, ascending t);
+ *   src_tok/src_j = inverse of slot;
+ *   rcnt[r] = #{t : some expert of t is on r}, rtok_off = exclusive scan of rcnt,
+ *   rtok/fanout = the tokens of rank r in ascending order with the mask of their
+ *   columns on r -- one move per (token, rank) pair.
+ * Deterministic (no result depends on thread timing).  Enqueues three kernels.
+ */
+MOE_API moe_status moe_plan(const int32_t *topk_idx, const float *topk_w, int32_t N, int32_t k,
+                    int32_t E, int32_t R, void *stream, moe_plan_t *plan);
+
+/*
+ * moe_dispatch -- recv[slot[t,j], :] = x[t, :] for every entry (FUSCO abstract and the
+ * FUSCO summary, Group 3: rows are placed straight into the expert-major layout with no
+ * intermediate buffer or later rearrangement).  Each token row is read from memory once
+ * and written to all of its k receive rows.
+ *
+ *   x           device [N, H] of `dtype` (bf16, or fp8 e4m3 bytes)
+ *   dtype       MOE_BF16 or MOE_FP8E4M3
+ *   x_scale     device fp32 [N, H/128] for fp8 (moved with its row), NULL for bf16
+ *   H           elements per row
+ *   plan        a plan built by moe_plan (its N and k are used)
+ *   recv        device [N*k, H] of `dtype`, caller-allocated, fully overwritten
+ *   recv_scale  device fp32 [N*k, H/128] for fp8, NULL for bf16
+ * Rows are copied bit for bit; nothing is converted.
+ */
+MOE_API moe_status moe_dispatch(const void *x, moe_dtype dtype, const float *x_scale, int32_t H,
+                        moe_plan_t plan, void *recv, float *recv_scale, void *stream);
+
+/*
+ * moe_combine -- out[t, :] = bf16_rne( fp32 fma chain over j = 0..k-1 of
+ * topk_w[t,j] * y[slot[t,j], :] ), starting from +0 (DySHARP blog, sections 1-2: the
+ * experts' results for a token are brought back and summed).  The chain order is the
+ * top-k column order, so the result does not depend on the launch configuration.
+ *
+ *   y     device bf16 [N*k, H]  expert outputs in the receive layout
+ *   H     elements per row (H % 8 == 0)
+ *   plan  the plan whose slots laid out y; its weights pointer is read
+ *   out   device bf16 [N, H], caller-allocated, fully overwritten
+ */
+MOE_API moe_status moe_combine(const void *y, int32_t H, moe_plan_t plan, void *out, void *stream);
+
+/* moe_plan_query -- fill *view with the plan's shape and device pointers. */
+MOE_API moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *view);
+
+/*
+ * moe_plan_check -- wait for `stream`, then copy the plan's error word to *flags
+ * (MOE_ERR_* bits; 0 = the routing was valid and every wait finished).
+ */
+MOE_API moe_status moe_plan_check(moe_plan_t plan, void *stream, uint32_t *flags);
+
+/* moe_plan_destroy -- free the plan (synchronises the device). NULL is a no-op. */
+MOE_API moe_status moe_plan_destroy(moe_plan_t plan);
+
+/* Message of the last failing call on this host thread ("" if none). */
+MOE_API const char *moe_last_error(void);
+
+/* Library version string. */
+MOE_API const char *moe_version(void);
+
+/* Launch parameters that moe_tune can override (process-wide; 0 restores the default).
+ * They change speed only, never results.  Not safe to call while another host thread
+ * is launching. */
+typedef enum {
+    MOE_TUNE_DISPATCH_STAGES = 0,        /* shared-memory row stages per dispatch warp (2..8) */
+    MOE_TUNE_DISPATCH_LAG = 1,           /* store groups a warp keeps in flight (1..stages-1) */
+    MOE_TUNE_DISPATCH_CTAS_PER_SM = 2,   /* cap on resident dispatch CTAs per SM */
+    MOE_TUNE_DISPATCH_WARPS_PER_CTA = 3, /* dispatch warps per CTA (1..4) */
+    MOE_TUNE_COMBINE_VEC_PER_LANE = 4,   /* 16-byte vectors per lane per combine unit (1, 2, 4) */
+    MOE_TUNE_COMBINE_CTAS_PER_SM = 5     /* cap on resident combine CTAs per SM */
+} moe_knob;
+
+MOE_API moe_status moe_tune(moe_knob knob, int32_t value);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_SHUFFLE_H */

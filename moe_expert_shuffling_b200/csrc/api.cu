@@ -1,0 +1,372 @@
+// C ABI of libmoeshuffle: argument checks, plan ownership and kernel launches.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "common.cuh"
+#include "internal.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+moe_status fail(moe_status st, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+moe_status ok()
+{
+    g_last_error.clear();
+    return MOE_OK;
+}
+
+moe_status cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(MOE_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status check_shape(int64_t N, int32_t k, int32_t E, int32_t R)
+{
+    if (N < 0)
+        return fail(MOE_EINVAL, "N must be >= 0 (got %lld)", static_cast<long long>(N));
+    if (k < 1 || k > moe::kMaxTopk)
+        return fail(MOE_EINVAL, "k must be in [1, %d] (got %d)", moe::kMaxTopk, k);
+    if (E < k || E > moe::kMaxExperts)
+        return fail(MOE_EINVAL, "E must be in [k, %d] (got E=%d, k=%d)", moe::kMaxExperts, E, k);
+    if (R < 1 || E % R != 0)
+        return fail(MOE_EINVAL, "R must divide E (got E=%d, R=%d)", E, R);
+    if (N * k >= (int64_t(1) << 31))
+        return fail(MOE_EINVAL, "N*k must be < 2^31 (got %lld)", static_cast<long long>(N * k));
+    return MOE_OK;
+}
+
+moe_status current_device(int *dev)
+{
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    return MOE_OK;
+}
+
+moe_status check_plan_device(const moe_plan_s *p)
+{
+    int dev = 0;
+    moe_status st = current_device(&dev);
+    if (st != MOE_OK)
+        return st;
+    if (dev != p->device)
+        return fail(MOE_EINVAL, "plan lives on device %d but device %d is current", p->device,
+                    dev);
+    return MOE_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+namespace moe {
+
+Tuning &tuning()
+{
+    static Tuning t;
+    return t;
+}
+
+int sm_count(int device)
+{
+    static int cache[64] = {0};
+    if (device < 0 || device >= 64)
+        return 148;
+    if (cache[device] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+            n <= 0)
+            n = 148;
+        cache[device] = n;
+    }
+    return cache[device];
+}
+
+}  // namespace moe
+
+extern "C" {
+
+const char *moe_last_error(void) { return g_last_error.c_str(); }
+
+const char *moe_version(void) { return "moeshuffle 0.1.0 (sm_100a)"; }
+
+moe_status moe_tune(moe_knob knob, int32_t value)
+{
+    if (value < 0)
+        return fail(MOE_EINVAL, "tuning values must be >= 0");
+    moe::Tuning &t = moe::tuning();
+    switch (knob) {
+    case MOE_TUNE_DISPATCH_STAGES: t.dispatch_stages = value; break;
+    case MOE_TUNE_DISPATCH_LAG: t.dispatch_lag = value; break;
+    case MOE_TUNE_DISPATCH_CTAS_PER_SM: t.dispatch_ctas_per_sm = value; break;
+    case MOE_TUNE_DISPATCH_WARPS_PER_CTA: t.dispatch_warps_per_cta = value; break;
+    case MOE_TUNE_COMBINE_VEC_PER_LANE: t.combine_vec_per_lane = value; break;
+    case MOE_TUNE_COMBINE_CTAS_PER_SM: t.combine_ctas_per_sm = value; break;
+    default: return fail(MOE_EINVAL, "unknown tuning knob %d", static_cast<int>(knob));
+    }
+    return ok();
+}
+
+moe_status moe_plan_create(int32_t max_tokens, int32_t k, int32_t E, int32_t R, moe_plan_t *out)
+{
+    if (!out)
+        return fail(MOE_EINVAL, "out must not be NULL");
+    *out = nullptr;
+    moe_status st = check_shape(max_tokens, k, E, R);
+    if (st != MOE_OK)
+        return st;
+    int dev = 0;
+    if ((st = current_device(&dev)) != MOE_OK)
+        return st;
+
+    moe_plan_s *p = new (std::nothrow) moe_plan_s();
+    if (!p)
+        return fail(MOE_ENOMEM, "host allocation failed");
+    p->cap = max_tokens;
+    p->k = k;
+    p->E = E;
+    p->R = R;
+    p->epr = E / R;
+    p->device = dev;
+    p->nt_cap = static_cast<int32_t>(moe::ceil_div(max_tokens, moe::kPlanTile));
+    p->rtok_cap = static_cast<int64_t>(max_tokens) * (k < R ? k : R);
+    const int64_t rows = static_cast<int64_t>(max_tokens) * k;
+    const int64_t nt = p->nt_cap > 0 ? p->nt_cap : 1;
+
+    // One allocation, every array 256-byte aligned.
+    struct Part {
+        void **dst;
+        size_t bytes;
+    } parts[] = {
+        {reinterpret_cast<void **>(&p->cnt), sizeof(int32_t) * E},
+        {reinterpret_cast<void **>(&p->expert_off), sizeof(int32_t) * (E + 1)},
+        {reinterpret_cast<void **>(&p->rcnt), sizeof(int32_t) * R},
+        {reinterpret_cast<void **>(&p->rank_off), sizeof(int32_t) * (R + 1)},
+        {reinterpret_cast<void **>(&p->rtok_off), sizeof(int32_t) * (R + 1)},
+        {reinterpret_cast<void **>(&p->slot), sizeof(int32_t) * (rows > 0 ? rows : 1)},
+        {reinterpret_cast<void **>(&p->src_tok), sizeof(int32_t) * (rows > 0 ? rows : 1)},
+        {reinterpret_cast<void **>(&p->src_j), sizeof(int32_t) * (rows > 0 ? rows : 1)},
+        {reinterpret_cast<void **>(&p->rtok), sizeof(int32_t) * (p->rtok_cap > 0 ? p->rtok_cap : 1)},
+        {reinterpret_cast<void **>(&p->fanout), sizeof(uint32_t) * (p->rtok_cap > 0 ? p->rtok_cap : 1)},
+        {reinterpret_cast<void **>(&p->err), sizeof(uint32_t)},
+        {reinterpret_cast<void **>(&p->tile_cnt), sizeof(int32_t) * E * nt},
+        {reinterpret_cast<void **>(&p->tile_rcnt), sizeof(int32_t) * R * nt},
+        {reinterpret_cast<void **>(&p->tile_err), sizeof(uint32_t) * nt},
+    };
+    size_t total = 0;
+    for (const Part &part : parts)
+        total += align256(part.bytes);
+    void *mem = nullptr;
+    cudaError_t e = cudaMalloc(&mem, total);
+    if (e != cudaSuccess) {
+        delete p;
+        (void)cudaGetLastError();
+        return fail(e == cudaErrorMemoryAllocation ? MOE_ENOMEM : MOE_ECUDA,
+                    "cudaMalloc(%zu): %s", total, cudaGetErrorString(e));
+    }
+    e = cudaMemset(mem, 0, total);
+    if (e != cudaSuccess) {
+        cudaFree(mem);
+        delete p;
+        return cuda_fail(e, "cudaMemset");
+    }
+    size_t off = 0;
+    for (const Part &part : parts) {
+        *part.dst = static_cast<char *>(mem) + off;
+        off += align256(part.bytes);
+    }
+    p->mem = mem;
+    p->mem_bytes = total;
+    *out = p;
+    return ok();
+}
+
+moe_status moe_plan(const int32_t *topk_idx, const float *topk_w, int32_t N, int32_t k, int32_t E,
+                    int32_t R, void *stream, moe_plan_t *plan)
+{
+    if (!plan)
+        return fail(MOE_EINVAL, "plan must not be NULL");
+    moe_status st = check_shape(N, k, E, R);
+    if (st != MOE_OK)
+        return st;
+    if (N > 0 && (!topk_idx || !topk_w))
+        return fail(MOE_EINVAL, "topk_idx and topk_w must not be NULL when N > 0");
+    if (!aligned(topk_idx, 4) || !aligned(topk_w, 4))
+        return fail(MOE_EINVAL, "topk_idx and topk_w must be 4-byte aligned");
+    if (*plan) {
+        moe_plan_s *p = *plan;
+        if (p->k != k || p->E != E || p->R != R)
+            return fail(MOE_EINVAL,
+                        "plan was created for (k=%d, E=%d, R=%d), called with (k=%d, E=%d, R=%d)",
+                        p->k, p->E, p->R, k, E, R);
+        if (N > p->cap)
+            return fail(MOE_EINVAL,
+                        "plan capacity is %d tokens, called with N=%d (create a larger plan "
+                        "with moe_plan_create)",
+                        p->cap, N);
+        if ((st = check_plan_device(p)) != MOE_OK)
+            return st;
+    } else {
+        if ((st = moe_plan_create(N, k, E, R, plan)) != MOE_OK)
+            return st;
+    }
+    moe_plan_s *p = *plan;
+    p->N = N;
+    p->topk_w = topk_w;
+    cudaError_t e = moe::launch_plan(p, topk_idx, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "plan kernels");
+    return ok();
+}
+
+moe_status moe_dispatch(const void *x, moe_dtype dtype, const float *x_scale, int32_t H,
+                        moe_plan_t plan, void *recv, float *recv_scale, void *stream)
+{
+    if (!plan)
+        return fail(MOE_EINVAL, "plan must not be NULL");
+    moe_plan_s *p = plan;
+    if (H <= 0 || H > (1 << 24))
+        return fail(MOE_EINVAL, "H must be in [1, 2^24] (got %d)", H);
+    uint32_t elem = 0, srow = 0;
+    if (dtype == MOE_BF16) {
+        if (H % 8 != 0)
+            return fail(MOE_EINVAL, "bf16 rows need H %% 8 == 0 (got H=%d)", H);
+        if (x_scale || recv_scale)
+            return fail(MOE_EINVAL, "bf16 dispatch takes no scales");
+        elem = 2;
+    } else if (dtype == MOE_FP8E4M3) {
+        if (H % 128 != 0)
+            return fail(MOE_EINVAL, "fp8 rows need H %% 128 == 0 (got H=%d)", H);
+        if (p->N > 0 && (!x_scale || !recv_scale))
+            return fail(MOE_EINVAL, "fp8 dispatch needs x_scale and recv_scale");
+        elem = 1;
+        srow = static_cast<uint32_t>(4 * (H / 128));
+        const size_t sa = (srow % 16 == 0) ? 16 : 4;
+        if (!aligned(x_scale, sa) || !aligned(recv_scale, sa))
+            return fail(MOE_EINVAL, "scale arrays must be %zu-byte aligned", sa);
+    } else {
+        return fail(MOE_EINVAL, "unknown dtype %d", static_cast<int>(dtype));
+    }
+    if (p->N > 0 && (!x || !recv))
+        return fail(MOE_EINVAL, "x and recv must not be NULL");
+    if (!aligned(x, 16) || !aligned(recv, 16))
+        return fail(MOE_EINVAL, "x and recv must be 16-byte aligned");
+    moe_status st = check_plan_device(p);
+    if (st != MOE_OK)
+        return st;
+    moe::DispatchArgs a;
+    a.x = static_cast<const uint8_t *>(x);
+    a.xs = reinterpret_cast<const uint8_t *>(x_scale);
+    a.recv = static_cast<uint8_t *>(recv);
+    a.rs = reinterpret_cast<uint8_t *>(recv_scale);
+    a.slot = p->slot;
+    a.err = p->err;
+    a.N = p->N;
+    a.k = p->k;
+    a.n_rows = p->N * p->k;
+    a.row_bytes = static_cast<uint32_t>(H) * elem;
+    a.srow_bytes = srow;
+    cudaError_t e = moe::launch_dispatch(a, p->device, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "dispatch kernel");
+    return ok();
+}
+
+moe_status moe_combine(const void *y, int32_t H, moe_plan_t plan, void *out, void *stream)
+{
+    if (!plan)
+        return fail(MOE_EINVAL, "plan must not be NULL");
+    moe_plan_s *p = plan;
+    if (H <= 0 || H > (1 << 24) || H % 8 != 0)
+        return fail(MOE_EINVAL, "H must be a multiple of 8 in [8, 2^24] (got %d)", H);
+    if (p->N > 0 && (!y || !out || !p->topk_w))
+        return fail(MOE_EINVAL, "y, out and the plan's weights must not be NULL");
+    if (!aligned(y, 16) || !aligned(out, 16))
+        return fail(MOE_EINVAL, "y and out must be 16-byte aligned");
+    moe_status st = check_plan_device(p);
+    if (st != MOE_OK)
+        return st;
+    moe::CombineArgs a;
+    a.y = static_cast<const uint16_t *>(y);
+    a.slot = p->slot;
+    a.w = p->topk_w;
+    a.out = static_cast<uint16_t *>(out);
+    a.N = p->N;
+    a.k = p->k;
+    a.n_rows = p->N * p->k;
+    a.H = H;
+    cudaError_t e = moe::launch_combine(a, p->device, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "combine kernel");
+    return ok();
+}
+
+moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *v)
+{
+    if (!plan || !v)
+        return fail(MOE_EINVAL, "plan and view must not be NULL");
+    const moe_plan_s *p = plan;
+    v->N = p->N;
+    v->k = p->k;
+    v->E = p->E;
+    v->R = p->R;
+    v->experts_per_rank = p->epr;
+    v->capacity_tokens = p->cap;
+    v->cnt = p->cnt;
+    v->expert_off = p->expert_off;
+    v->rcnt = p->rcnt;
+    v->rank_off = p->rank_off;
+    v->rtok_off = p->rtok_off;
+    v->slot = p->slot;
+    v->src_tok = p->src_tok;
+    v->src_j = p->src_j;
+    v->rtok = p->rtok;
+    v->fanout = p->fanout;
+    v->err = p->err;
+    v->topk_w = p->topk_w;
+    return ok();
+}
+
+moe_status moe_plan_check(moe_plan_t plan, void *stream, uint32_t *flags)
+{
+    if (!plan || !flags)
+        return fail(MOE_EINVAL, "plan and flags must not be NULL");
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaStreamSynchronize");
+    e = cudaMemcpy(flags, plan->err, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaMemcpy(err)");
+    return ok();
+}
+
+moe_status moe_plan_destroy(moe_plan_t plan)
+{
+    if (!plan)
+        return ok();
+    cudaError_t e = cudaSuccess;
+    if (plan->mem)
+        e = cudaFree(plan->mem);
+    delete plan;
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaFree");
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,253 @@
+// Dispatch: recv[slot[t, j]] = x[t] for every routed entry, with the expert-major layout
+// produced by the copy itself (FUSCO, arXiv 2512.22036, abstract; FUSCO summary, Group 3:
+// data is placed at its destination with no staging buffer and no later rearrangement).
+//
+// Engine: a persistent grid of warps, each running its own pipeline over work units
+// (token, row chunk).  Lane 0 stages a chunk of x[t] into shared memory with one bulk
+// async copy (cp.async.bulk, completion on an mbarrier); once it has landed, lane j
+// issues the bulk store of that chunk to receive row slot[t, j].  So every token row
+// is read from HBM once and written k times -- the "read once, fan out locally" form of
+// FUSCO's dedup (one move per token, which is at most one per destination rank).  A
+// stage is refilled only after the stores reading it have drained (wait_group.read).
+// fp8 rows carry their fp32 scale block along when its size is a multiple of 16 bytes;
+// otherwise a small second kernel moves the scales.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr uint32_t kMaxChunkBytes = 32768;
+constexpr int kMaxStages = 8;
+
+struct DispatchParams {
+    const uint8_t *x;
+    const uint8_t *xs;
+    uint8_t *recv;
+    uint8_t *rs;
+    const int32_t *slot;
+    uint32_t *err;
+    uint32_t units;         // N * nchunks (< 2^31)
+    int32_t k, n_rows;
+    uint32_t nchunks;
+    int32_t stages, lag;
+    uint32_t row_bytes, srow_bytes, chunk_bytes, stage_bytes, scale_off, bar_bytes;
+    bool bulk_scales;
+};
+
+__global__ void __launch_bounds__(128) dispatch_bulk_kernel(const DispatchParams p)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, wpc = blockDim.x >> 5;
+    const int S = p.stages;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem) + wid * S;
+    uint8_t *stage0 = smem + p.bar_bytes + static_cast<size_t>(wid) * S * p.stage_bytes;
+
+    const uint32_t gw = blockIdx.x * wpc + wid;
+    const uint32_t nw = gridDim.x * wpc;
+    const int n_my = gw < p.units ? static_cast<int>((p.units - gw + nw - 1) / nw) : 0;
+
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s)
+            mbar_init(&bars[s], 1);
+        mbar_init_fence();
+    }
+    __syncwarp();
+
+    // Issue the load of this warp's i-th unit into stage i % S (lane 0 only).
+    auto issue_load = [&](int i) {
+        const uint32_t u = gw + static_cast<uint32_t>(i) * nw;
+        const uint32_t t = u / p.nchunks;
+        const uint32_t c = u - t * p.nchunks;
+        const uint32_t off = c * p.chunk_bytes;
+        const uint32_t len = min(p.chunk_bytes, p.row_bytes - off);
+        const int s = static_cast<int>(i % S);
+        uint8_t *st = stage0 + static_cast<size_t>(s) * p.stage_bytes;
+        const bool sc = p.bulk_scales && c == 0;
+        mbar_arrive_expect_tx(&bars[s], len + (sc ? p.srow_bytes : 0u));
+        bulk_load(st, p.x + static_cast<int64_t>(t) * p.row_bytes + off, len, &bars[s]);
+        if (sc)
+            bulk_load(st + p.scale_off, p.xs + static_cast<int64_t>(t) * p.srow_bytes,
+                      p.srow_bytes, &bars[s]);
+    };
+
+    int next_load = S < n_my ? S : n_my;  // units [0, next_load) have been issued
+    if (lane == 0)
+        for (int i = 0; i < next_load; ++i)
+            issue_load(i);
+
+    int32_t cur = -1;
+    if (n_my > 0 && lane < p.k)
+        cur = __ldg(p.slot + (gw / p.nchunks) * p.k + lane);
+
+    bool ok = true;
+    int i = 0;
+    for (; i < n_my; ++i) {
+        const int s = i % S;
+        const uint32_t parity = static_cast<uint32_t>((i / S) & 1);
+        const uint32_t u = gw + static_cast<uint32_t>(i) * nw;
+        const uint32_t t = u / p.nchunks;
+        const uint32_t c = u - t * p.nchunks;
+        const uint32_t off = c * p.chunk_bytes;
+        const uint32_t len = min(p.chunk_bytes, p.row_bytes - off);
+
+        // Slots of the next unit, fetched while this unit's row is in flight.
+        int32_t nxt = -1;
+        if (i + 1 < n_my && lane < p.k)
+            nxt = __ldg(p.slot + ((u + nw) / p.nchunks) * p.k + lane);
+
+        const bool landed = mbar_wait_bounded(&bars[s], parity);
+        if (!__all_sync(0xffffffffu, landed)) {
+            ok = false;
+            break;
+        }
+        const uint8_t *st = stage0 + static_cast<size_t>(s) * p.stage_bytes;
+        if (lane < p.k && static_cast<uint32_t>(cur) < static_cast<uint32_t>(p.n_rows)) {
+            bulk_store(p.recv + static_cast<int64_t>(cur) * p.row_bytes + off, st, len);
+            if (p.bulk_scales && c == 0)
+                bulk_store(p.rs + static_cast<int64_t>(cur) * p.srow_bytes, st + p.scale_off,
+                           p.srow_bytes);
+        }
+        bulk_commit();
+
+        // Refill the stage of unit i - lag once its stores have read shared memory.
+        const int r = i - p.lag;
+        if (r >= 0 && r + S < n_my) {
+            bulk_wait_read_dyn(p.lag);
+            __syncwarp();
+            if (lane == 0)
+                issue_load(r + S);
+            next_load = r + S + 1;
+        }
+        cur = nxt;
+    }
+    bulk_wait_all();
+    if (!ok) {
+        if (lane == 0)
+            atomicOr(p.err, MOE_ERR_TIMEOUT);
+        // Let loads still in flight land before this warp's shared memory is released.
+        for (int m = i; m < next_load; ++m)
+            (void)mbar_wait_bounded(&bars[m % S], static_cast<uint32_t>((m / S) & 1));
+    }
+}
+
+// Scale rows whose size is not a multiple of 16 bytes: one thread per fp32 scale.
+__global__ void dispatch_scales_kernel(const float *__restrict__ xs, float *__restrict__ rs,
+                                       const int32_t *__restrict__ slot, int64_t entries,
+                                       int32_t k, int32_t ncols, int32_t n_rows)
+{
+    const int64_t total = entries * ncols;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t ent = i / ncols;
+        const int32_t c = static_cast<int32_t>(i - ent * ncols);
+        const int32_t s = slot[ent];
+        if (static_cast<uint32_t>(s) < static_cast<uint32_t>(n_rows))
+            rs[static_cast<int64_t>(s) * ncols + c] = xs[(ent / k) * ncols + c];
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const DispatchArgs &a, int device, cudaStream_t stream)
+{
+    if (a.N == 0)
+        return cudaSuccess;
+    const Tuning &tu = tuning();
+    int stages = tu.dispatch_stages > 0 ? tu.dispatch_stages : 4;
+    stages = std::min(std::max(stages, 2), kMaxStages);
+    int lag = tu.dispatch_lag > 0 ? tu.dispatch_lag : 2;
+    lag = std::min(std::max(lag, 1), std::min(stages - 1, 7));
+    int wpc = tu.dispatch_warps_per_cta > 0 ? tu.dispatch_warps_per_cta : 1;
+    wpc = std::min(std::max(wpc, 1), 4);
+
+    const uint32_t nchunks =
+        static_cast<uint32_t>(ceil_div(a.row_bytes, kMaxChunkBytes));
+    const uint32_t chunk =
+        static_cast<uint32_t>(round_up(ceil_div(a.row_bytes, nchunks), 16));
+    const bool bulk_scales = a.srow_bytes > 0 && a.srow_bytes % 16 == 0;
+    const uint32_t scale_off = static_cast<uint32_t>(round_up(chunk, 128));
+    const uint32_t stage_bytes =
+        static_cast<uint32_t>(round_up(scale_off + (bulk_scales ? a.srow_bytes : 0u), 128));
+
+    int max_optin = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                           device);
+    if (e != cudaSuccess)
+        return e;
+    auto smem_for = [&](int st) {
+        return static_cast<size_t>(round_up(static_cast<int64_t>(wpc) * st * 8, 128)) +
+               static_cast<size_t>(wpc) * st * stage_bytes;
+    };
+    while (stages > 2 && smem_for(stages) > static_cast<size_t>(max_optin))
+        --stages;
+    while (wpc > 1 && smem_for(stages) > static_cast<size_t>(max_optin))
+        --wpc;
+    if (smem_for(stages) > static_cast<size_t>(max_optin))
+        return cudaErrorInvalidValue;
+    lag = std::min(lag, stages - 1);
+    const size_t smem = smem_for(stages);
+
+    e = cudaFuncSetAttribute(dispatch_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess)
+        return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_bulk_kernel, wpc * 32,
+                                                      smem);
+    if (e != cudaSuccess)
+        return e;
+    if (per_sm < 1)
+        return cudaErrorInvalidConfiguration;
+    if (tu.dispatch_ctas_per_sm > 0)
+        per_sm = std::min(per_sm, tu.dispatch_ctas_per_sm);
+
+    DispatchParams p;
+    p.x = a.x;
+    p.xs = a.xs;
+    p.recv = a.recv;
+    p.rs = a.rs;
+    p.slot = a.slot;
+    p.err = a.err;
+    const int64_t units = static_cast<int64_t>(a.N) * nchunks;
+    if (units >= (int64_t(1) << 31))
+        return cudaErrorInvalidValue;
+    p.units = static_cast<uint32_t>(units);
+    p.k = a.k;
+    p.n_rows = a.n_rows;
+    p.nchunks = nchunks;
+    p.stages = stages;
+    p.lag = lag;
+    p.row_bytes = a.row_bytes;
+    p.srow_bytes = a.srow_bytes;
+    p.chunk_bytes = chunk;
+    p.stage_bytes = stage_bytes;
+    p.scale_off = scale_off;
+    p.bar_bytes = static_cast<uint32_t>(round_up(static_cast<int64_t>(wpc) * stages * 8, 128));
+    p.bulk_scales = bulk_scales;
+
+    const int64_t warps_needed = p.units;
+    const int64_t grid = std::max<int64_t>(
+        1, std::min<int64_t>(ceil_div(warps_needed, wpc), static_cast<int64_t>(sm_count(device)) * per_sm));
+    dispatch_bulk_kernel<<<static_cast<unsigned>(grid), wpc * 32, smem, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+
+    if (a.srow_bytes > 0 && !bulk_scales) {
+        const int32_t ncols = static_cast<int32_t>(a.srow_bytes / 4);
+        const int64_t entries = static_cast<int64_t>(a.N) * a.k;
+        const int64_t total = entries * ncols;
+        const int64_t blocks = std::min<int64_t>(ceil_div(total, 256), sm_count(device) * 8);
+        dispatch_scales_kernel<<<static_cast<unsigned>(std::max<int64_t>(blocks, 1)), 256, 0,
+                                 stream>>>(reinterpret_cast<const float *>(a.xs),
+                                           reinterpret_cast<float *>(a.rs), a.slot, entries, a.k,
+                                           ncols, a.n_rows);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace moe

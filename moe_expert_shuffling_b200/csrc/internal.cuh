@@ -1,0 +1,75 @@
+// Host-side internals shared by the C ABI (api.cu) and the kernel launchers.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "moe_shuffle.h"
+
+// Plan object behind moe_plan_t.  All arrays live in one device allocation.
+struct moe_plan_s {
+    int32_t cap = 0;        // largest N accepted
+    int32_t N = 0, k = 0, E = 0, R = 0, epr = 0;
+    int32_t nt_cap = 0;     // tiles for `cap` tokens
+    int64_t rtok_cap = 0;   // entries of rtok/fanout: cap * min(k, R)
+    int device = 0;
+    void *mem = nullptr;
+    size_t mem_bytes = 0;
+    // outputs
+    int32_t *cnt = nullptr, *expert_off = nullptr, *rcnt = nullptr, *rank_off = nullptr,
+            *rtok_off = nullptr, *slot = nullptr, *src_tok = nullptr, *src_j = nullptr,
+            *rtok = nullptr;
+    uint32_t *fanout = nullptr, *err = nullptr;
+    // scratch: per-tile counts [E][nt] and [R][nt] (then their column prefixes), tile flags
+    int32_t *tile_cnt = nullptr, *tile_rcnt = nullptr;
+    uint32_t *tile_err = nullptr;
+    const float *topk_w = nullptr;
+};
+
+namespace moe {
+
+// Tokens per plan tile (one CTA of the count and rank kernels).
+constexpr int kPlanWarps = 8;
+constexpr int kPlanTokensPerWarp = 16;
+constexpr int kPlanTile = kPlanWarps * kPlanTokensPerWarp;
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopk = 32;
+
+// Tunable launch parameters (0 = built-in default).  Set through moe_tune.
+struct Tuning {
+    int dispatch_stages = 0;
+    int dispatch_lag = 0;
+    int dispatch_ctas_per_sm = 0;
+    int dispatch_warps_per_cta = 0;
+    int combine_vec_per_lane = 0;
+    int combine_ctas_per_sm = 0;
+};
+Tuning &tuning();
+
+int sm_count(int device);
+
+cudaError_t launch_plan(moe_plan_s *p, const int32_t *topk_idx, cudaStream_t stream);
+
+struct DispatchArgs {
+    const uint8_t *x;      // [N, row_bytes]
+    const uint8_t *xs;     // [N, srow_bytes] or null
+    uint8_t *recv;         // [n_rows, row_bytes]
+    uint8_t *rs;           // [n_rows, srow_bytes] or null
+    const int32_t *slot;   // [N*k]
+    uint32_t *err;
+    int32_t N, k, n_rows;
+    uint32_t row_bytes, srow_bytes;
+};
+cudaError_t launch_dispatch(const DispatchArgs &a, int device, cudaStream_t stream);
+
+struct CombineArgs {
+    const uint16_t *y;     // bf16 [n_rows, H]
+    const int32_t *slot;   // [N*k]
+    const float *w;        // [N*k]
+    uint16_t *out;         // bf16 [N, H]
+    int32_t N, k, n_rows, H;
+};
+cudaError_t launch_combine(const CombineArgs &a, int device, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,119 @@
+"""The C ABI library loads, exports every function include/*.h declares, and rejects bad
+arguments on the host before touching the GPU (these calls make no CUDA call)."""
+
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from moe_expert_shuffling_b200 import build
+    path = build.build()
+    lib = ctypes.CDLL(path)
+    lib.moe_last_error.restype = ctypes.c_char_p
+    lib.moe_version.restype = ctypes.c_char_p
+    return lib
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names |= set(re.findall(r"^MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", text, flags=re.M))
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("moe_plan", "moe_dispatch", "moe_combine", "moe_plan_create",
+                     "moe_plan_query", "moe_plan_check", "moe_plan_destroy", "moe_last_error"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from moe_expert_shuffling_b200 import build
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    declared = declared_functions()
+    missing = declared - exported
+    assert not missing, missing
+    # nothing else of ours leaks out of the library
+    ours = {s for s in exported if s.startswith("moe_")}
+    assert ours == declared, ours ^ declared
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_version(lib):
+    assert b"sm_100a" in lib.moe_version()
+
+
+def _plan(lib, N, k, E, R):
+    h = ctypes.c_void_p(0)
+    st = lib.moe_plan(ctypes.c_void_p(0), ctypes.c_void_p(0), N, k, E, R, ctypes.c_void_p(0),
+                      ctypes.byref(h))
+    return st, lib.moe_last_error().decode()
+
+
+@pytest.mark.parametrize("N,k,E,R,msg", [
+    (4, 2, 8, 3, "R must divide E"),
+    (4, 33, 64, 4, "k must be in"),
+    (4, 0, 8, 4, "k must be in"),
+    (-1, 2, 8, 4, "N must be >= 0"),
+    (4, 4, 2048, 4, "E must be in"),
+    (4, 9, 8, 4, "E must be in"),
+    (1 << 28, 8, 64, 4, "N*k must be < 2^31"),
+    (4, 2, 8, 4, "must not be NULL"),       # valid shape, but no routing arrays
+])
+def test_plan_rejects_bad_arguments_on_host(lib, N, k, E, R, msg):
+    st, err = _plan(lib, N, k, E, R)
+    assert st == 1, err          # MOE_EINVAL
+    assert msg in err
+
+
+def test_null_plan_rejected(lib):
+    assert lib.moe_dispatch(None, 0, None, 64, None, None, None, None) == 1
+    assert b"plan" in lib.moe_last_error()
+    assert lib.moe_combine(None, 64, None, None, None) == 1
+    assert lib.moe_plan(None, None, 0, 1, 1, 1, None, None) == 1
+    assert lib.moe_plan_query(None, None) == 1
+    assert lib.moe_plan_check(None, None, None) == 1
+    assert lib.moe_plan_create(4, 2, 8, 4, None) == 1
+
+
+def test_destroy_null_is_noop(lib):
+    assert lib.moe_plan_destroy(None) == 0
+
+
+def test_tune_rejects_unknown_knob(lib):
+    assert lib.moe_tune(99, 1) == 1
+    assert lib.moe_tune(0, -1) == 1
+    assert lib.moe_tune(0, 0) == 0   # default restored
+
+
+def test_python_binding_imports_and_knows_knobs():
+    import moe_expert_shuffling_b200 as ms
+    assert ms.version().startswith("moeshuffle")
+    assert set(ms.KNOBS) >= {"dispatch_stages", "combine_vec_per_lane"}
+    with pytest.raises(TypeError):
+        ms.moe_plan("not a tensor", None, 8, 4)
+
+
+def test_product_has_no_oracle_dependency():
+    """The CUDA library and its binding never import, link or call the oracle."""
+    pkg = os.path.join(ROOT, "moe_expert_shuffling_b200")
+    for path in glob.glob(os.path.join(pkg, "**", "*"), recursive=True):
+        if os.path.isfile(path) and path.endswith((".py", ".cu", ".cuh", ".h")):
+            text = open(path).read()
+            assert "oracle" not in text.lower(), path
+    out = subprocess.run(["ldd", os.path.join(pkg, "libmoeshuffle.so")], capture_output=True,
+                         text=True).stdout
+    assert "oracle" not in out

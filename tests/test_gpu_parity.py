@@ -1,0 +1,223 @@
+"""Parity of the CUDA path with the CPU oracle on the same seeded inputs.
+
+Plan and dispatch must match bit for bit; combine must be within 1 bf16 ulp, max abs 1e-2
+and max rel 8e-3 (and, since both sides run the same fp32 fma chain, is expected to
+match bit for bit as well).  Full-size cases run in the launch configuration the
+benchmark times (the library defaults)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.shuffle_cases import (
+    assert_combine_close, assert_plan_equal, bits16, bits_to_f32, gpu_plan, make_inputs,
+    plan_to_host,
+)
+from workloads import CONFIGS
+
+pytestmark = pytest.mark.gpu
+
+ALL = ["tiny", "mixtral", "dsv3", "skew", "long"]
+
+
+def run_all(cfg, seed, y_identity=False):
+    """GPU plan/dispatch/combine and oracle plan/dispatch/combine; returns both sides."""
+    import moe_expert_shuffling_b200 as ms
+    idx, w, x, xs, y = make_inputs(cfg, seed, y=not y_identity)
+    p, ti, tw = gpu_plan(idx, w, cfg.E, cfg.R)
+    if cfg.payload == "fp8":
+        recv, rs = ms.moe_dispatch(x, p, x_scale=xs)
+    else:
+        recv, rs = ms.moe_dispatch(x, p), None
+    yy = recv if y_identity else y
+    out = ms.moe_combine(yy, p)
+    torch.cuda.synchronize()
+    assert p.check() == 0
+
+    ref = oracle.plan(idx, cfg.E, cfg.R)
+    gp = plan_to_host(p)
+    x_h = x.cpu()
+    if cfg.payload == "fp8":
+        ref_recv, ref_rs = oracle.dispatch(x_h.numpy(), ref.slot, xs.cpu().numpy())
+        got_recv = recv.cpu().numpy()
+        got_rs = rs.cpu().numpy().view(np.uint8)
+    else:
+        ref_recv = oracle.dispatch(bits16(x_h).view(np.uint8).reshape(cfg.N, -1), ref.slot)
+        ref_rs = got_rs = None
+        got_recv = bits16(recv).view(np.uint8).reshape(cfg.N * cfg.k, -1)
+    y_h = ref_recv.view(np.uint16).reshape(cfg.N * cfg.k, cfg.H) if y_identity else bits16(y)
+    ref_out = oracle.combine(y_h, ref.slot, w)
+    return dict(gp=gp, ref=ref, got_recv=got_recv, ref_recv=ref_recv, got_rs=got_rs,
+                ref_rs=ref_rs, got_out=bits16(out), ref_out=ref_out, x=x_h)
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_full_size_parity(name):
+    cfg = CONFIGS[name]
+    r = run_all(cfg, 0, y_identity=(cfg.y == "identity"))
+    assert_plan_equal(r["gp"], r["ref"])
+    assert np.array_equal(r["got_recv"], r["ref_recv"])
+    if r["ref_rs"] is not None:
+        assert np.array_equal(r["got_rs"], r["ref_rs"])
+    assert_combine_close(r["got_out"], r["ref_out"])
+    assert np.array_equal(r["got_out"], r["ref_out"])
+
+
+@pytest.mark.parametrize("name,seed", [("tiny", 1), ("tiny", 2), ("dsv3", 1), ("skew", 2)])
+def test_more_seeds(name, seed):
+    cfg = CONFIGS[name]
+    if name in ("dsv3", "skew"):
+        cfg = cfg.with_tokens(3000)   # several tiles plus a ragged tail
+    r = run_all(cfg, seed)
+    assert_plan_equal(r["gp"], r["ref"])
+    assert np.array_equal(r["got_recv"], r["ref_recv"])
+    assert np.array_equal(r["got_out"], r["ref_out"])
+
+
+@pytest.mark.parametrize("name", ["mixtral", "dsv3"])
+def test_identity_experts_return_x(name):
+    """combine(dispatch(x)) == x with y = recv and weights summing to 1."""
+    cfg = CONFIGS[name]
+    r = run_all(cfg, 0, y_identity=True)
+    assert np.array_equal(bits_to_f32(r["got_out"]), bits_to_f32(bits16(r["x"])))
+
+
+@pytest.mark.parametrize("cfg", [
+    CONFIGS["tiny"].with_tokens(1),
+    CONFIGS["tiny"].with_tokens(127),
+    CONFIGS["tiny"].with_tokens(129),
+    CONFIGS["dsv3"].with_tokens(1000).replace(H=256),
+    CONFIGS["tiny"].replace(k=1, N=777),                                   # top-1
+    CONFIGS["dsv3"].replace(N=300, H=64, E=64, k=32, R=8),                 # maximum k
+    CONFIGS["dsv3"].replace(N=400, H=64, E=1024, k=8, R=1024),             # maximum E, E == R
+    CONFIGS["dsv3"].replace(N=400, H=64, E=1024, k=8, R=1),                # one rank
+    CONFIGS["tiny"].replace(N=200, H=8),                                   # smallest bf16 row
+    CONFIGS["tiny"].replace(N=70, H=20000),                                # row split in chunks
+    CONFIGS["long"].replace(N=300, H=128),                                 # 4-byte scale rows
+    CONFIGS["long"].replace(N=300, H=640),                                 # 20-byte scale rows
+    CONFIGS["long"].replace(N=50, H=65536),                                # chunked fp8 row
+    CONFIGS["long"].replace(N=1000, H=512, k=4, E=16, R=16),
+], ids=lambda c: f"{c.name}-N{c.N}-H{c.H}-E{c.E}-k{c.k}-R{c.R}-{c.payload}")
+def test_edge_shapes(cfg):
+    r = run_all(cfg, 0)
+    assert_plan_equal(r["gp"], r["ref"])
+    assert np.array_equal(r["got_recv"], r["ref_recv"])
+    if r["ref_rs"] is not None:
+        assert np.array_equal(r["got_rs"], r["ref_rs"])
+    assert_combine_close(r["got_out"], r["ref_out"])
+    assert np.array_equal(r["got_out"], r["ref_out"])
+
+
+def test_empty_input():
+    import moe_expert_shuffling_b200 as ms
+    ti = torch.zeros((0, 8), dtype=torch.int32, device="cuda")
+    tw = torch.zeros((0, 8), dtype=torch.float32, device="cuda")
+    p = ms.moe_plan(ti, tw, 256, 32)
+    recv = ms.moe_dispatch(torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda"), p)
+    out = ms.moe_combine(recv, p)
+    assert recv.shape == (0, 64) and out.shape == (0, 64)
+    assert p.check() == 0
+    a = p.arrays()
+    assert int(a["expert_off"].abs().sum()) == 0 and int(a["rtok_off"].abs().sum()) == 0
+
+
+def test_plan_reuse_and_capacity():
+    import moe_expert_shuffling_b200 as ms
+    cfg = CONFIGS["dsv3"].with_tokens(2000)
+    p = ms.moe_plan_create(2000, cfg.k, cfg.E, cfg.R)
+    for seed, N in ((0, 2000), (1, 1500), (2, 129)):
+        c = cfg.with_tokens(N)
+        idx, w, x, _, y = make_inputs(c, seed)
+        p, ti, tw = gpu_plan(idx, w, c.E, c.R, plan=p)
+        recv = ms.moe_dispatch(x, p)
+        out = ms.moe_combine(y, p)
+        ref = oracle.plan(idx, c.E, c.R)
+        assert_plan_equal(plan_to_host(p), ref)
+        ref_recv = oracle.dispatch(bits16(x).view(np.uint8).reshape(N, -1), ref.slot)
+        assert np.array_equal(bits16(recv).view(np.uint8).reshape(N * c.k, -1), ref_recv)
+        assert np.array_equal(bits16(out), oracle.combine(bits16(y), ref.slot, w))
+    idx, w, *_ = make_inputs(cfg.with_tokens(2001), 0, y=False)
+    with pytest.raises(ms.MoeError, match="capacity"):
+        gpu_plan(idx, w, cfg.E, cfg.R, plan=p)
+    with pytest.raises(ms.MoeError, match="created for"):
+        gpu_plan(idx[:10, :4].copy(), w[:10, :4].copy(), cfg.E, cfg.R, plan=p)
+
+
+def test_invalid_routing_is_flagged_and_contained():
+    """Out-of-range and repeated ids set error bits, get slot -1 and are skipped."""
+    import moe_expert_shuffling_b200 as ms
+    cfg = CONFIGS["tiny"].with_tokens(300)
+    idx, w, x, _, y = make_inputs(cfg, 0)
+    bad = idx.copy()
+    bad[3, 0] = cfg.E            # out of range
+    bad[10, 1] = -5              # negative
+    bad[20, 1] = bad[20, 0]      # repeated in one token
+    bad[299, 0] = 2 ** 31 - 1
+    p, ti, tw = gpu_plan(bad, w, cfg.E, cfg.R)
+    recv = torch.zeros((cfg.N * cfg.k, cfg.H), dtype=torch.bfloat16, device="cuda")
+    ms.moe_dispatch(x, p, recv=recv)
+    out = ms.moe_combine(y, p)
+    flags = p.check()
+    assert flags & ms.ERR_ID_RANGE and flags & ms.ERR_ID_DUP
+    assert not flags & (ms.ERR_BOUNDS | ms.ERR_TIMEOUT)
+    g = plan_to_host(p)
+    valid = np.ones_like(bad, dtype=bool)
+    valid[3, 0] = valid[10, 1] = valid[20, 1] = valid[299, 0] = False
+    assert np.all(g["slot"][~valid] == -1)
+    # the valid entries form the plan of the routing with the bad entries removed
+    n_valid = int(valid.sum())
+    assert int(g["cnt"].sum()) == n_valid
+    s = g["slot"][valid]
+    assert np.array_equal(np.sort(s), np.arange(n_valid))
+    xb = bits16(x)
+    rb = bits16(recv)
+    tok = np.nonzero(valid)[0]
+    assert np.array_equal(rb[s], xb[tok])
+    # combine of a token with a skipped entry sums only its valid entries
+    yb = bits16(y)
+    t = 3
+    acc = np.float32(0)
+    for j in range(cfg.k):
+        if valid[t, j]:
+            acc = np.float32(acc + np.float32(w[t, j]) * bits_to_f32(yb[g["slot"][t, j]]))
+    got = bits_to_f32(bits16(out)[t])
+    assert np.allclose(got, acc, rtol=8e-3, atol=1e-2)
+
+
+@pytest.mark.parametrize("knobs", [
+    {"dispatch_stages": 2, "dispatch_lag": 1},
+    {"dispatch_stages": 8, "dispatch_lag": 4, "dispatch_warps_per_cta": 2},
+    {"dispatch_ctas_per_sm": 1, "combine_ctas_per_sm": 1},
+    {"combine_vec_per_lane": 1},
+    {"combine_vec_per_lane": 4},
+])
+def test_launch_configuration_does_not_change_results(knobs):
+    import moe_expert_shuffling_b200 as ms
+    cfg = CONFIGS["dsv3"].with_tokens(1500)
+    try:
+        for k, v in knobs.items():
+            ms.moe_tune(k, v)
+        r = run_all(cfg, 2)
+    finally:
+        for k in knobs:
+            ms.moe_tune(k, 0)
+    assert_plan_equal(r["gp"], r["ref"])
+    assert np.array_equal(r["got_recv"], r["ref_recv"])
+    assert np.array_equal(r["got_out"], r["ref_out"])
+
+
+def test_side_stream():
+    import moe_expert_shuffling_b200 as ms
+    cfg = CONFIGS["dsv3"].with_tokens(700)
+    idx, w, x, _, y = make_inputs(cfg, 1)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        ti = torch.from_numpy(idx).cuda()
+        tw = torch.from_numpy(w).cuda()
+        p = ms.moe_plan(ti, tw, cfg.E, cfg.R)
+        recv = ms.moe_dispatch(x, p)
+        out = ms.moe_combine(y, p)
+    s.synchronize()
+    ref = oracle.plan(idx, cfg.E, cfg.R)
+    assert np.array_equal(bits16(out), oracle.combine(bits16(y), ref.slot, w))
