@@ -91,6 +91,12 @@ __device__ __forceinline__ void bulk_store(void *dst, const void *src_smem, uint
                  : "memory");
 }
 
+// Order earlier shared-memory accesses before later async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_commit()
 {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");

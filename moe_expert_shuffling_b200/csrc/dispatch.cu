@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(128) dispatch_bulk_kernel(const DispatchParams
             ok = false;
             break;
         }
+        fence_proxy_async_smem();
         const uint8_t *st = stage0 + static_cast<size_t>(s) * p.stage_bytes;
         if (lane < p.k && static_cast<uint32_t>(cur) < static_cast<uint32_t>(p.n_rows)) {
             bulk_store(p.recv + static_cast<int64_t>(cur) * p.row_bytes + off, st, len);
