@@ -184,6 +184,8 @@ def run_ours(args):
     lib_build.build()
     world, rank, local = dist_setup(args)
     cfg = CONFIGS[args.config]
+    if args.tokens > 0:
+        cfg = cfg.with_tokens(args.tokens)
     seed = args.seed + rank
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(device=dev)
@@ -387,6 +389,8 @@ def run_reference(args):
     if int(os.environ.get("RANK", "0")) != 0:
         return
     cfg = CONFIGS[args.config]
+    if args.tokens > 0:
+        cfg = cfg.with_tokens(args.tokens)
     idx_h, w_h = make_routing(cfg, args.seed)
     n_max = min(cfg.N, 4096)
     cfg_s = cfg.with_tokens(n_max)
@@ -432,6 +436,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="dsv3", choices=sorted(CONFIGS))
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count (small cases for profiling)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=5)
