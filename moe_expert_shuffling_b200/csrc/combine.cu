@@ -153,9 +153,9 @@ cudaError_t launch_combine(const CombineArgs &a, int device, cudaStream_t stream
     if (a.N == 0)
         return cudaSuccess;
     const Tuning &tu = tuning();
-    int vpl = tu.combine_vec_per_lane > 0 ? tu.combine_vec_per_lane : 2;
+    int vpl = tu.combine_vec_per_lane > 0 ? tu.combine_vec_per_lane : 1;
     if (vpl != 1 && vpl != 2 && vpl != 4)
-        vpl = 2;
+        vpl = 1;
     CombineParams p;
     p.y = a.y;
     p.slot = a.slot;

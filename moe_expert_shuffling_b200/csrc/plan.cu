@@ -9,10 +9,11 @@
 //               counts of (token, rank) moves -> scratch [E][tiles], [R][tiles]
 //   plan_scan   one CTA per expert row and per rank row: exclusive scan over tiles,
 //               row totals -> cnt[E], rcnt[R]; CTA 0 also gathers the tile flags
-//   plan_rank   one CTA per tile: segment starts (scan of cnt/rcnt), then each warp
+//   plan_rank   one CTA per tile: segment starts (scan of cnt/rcnt), entry classes and
+//               per-warp counts in parallel over the tile's entries, then each warp
 //               walks its 16 tokens in order, one token per step with lane j holding
-//               column j.  Ids of one valid token are distinct, so the lanes of a step
-//               touch distinct counters and the walk needs no atomics.
+//               column j.  The valid ids of one token are distinct, so the lanes of a
+//               step touch distinct counters and the walk needs no atomics.
 #include "common.cuh"
 #include "internal.cuh"
 
@@ -21,35 +22,58 @@ namespace {
 
 constexpr int kPlanThreads = kPlanWarps * 32;
 constexpr int kScanThreads = 256;
-constexpr uint32_t kFull = 0xffffffffu;
+constexpr uint32_t kFull = 0xffffffffu;  // all lanes of a warp
 
-// Classification of column `lane` of one token (lanes >= k hold no entry).
-struct Entry {
-    bool valid;       // id in [0, E) and not repeated by an earlier column
-    bool leader;      // valid and the first valid column of its rank
-    int32_t r;        // rank of the expert (valid entries only)
-    uint32_t same_rank;  // lanes of the token's valid columns on rank r
-    uint32_t flags;   // MOE_ERR_* raised by this column
-};
-
-__device__ __forceinline__ Entry classify(int32_t e, int lane, int k, int E, int epr)
+// Entry classification, shared by the count and rank kernels so both see the same
+// entries.  An entry (t, j) is valid when its id is in [0, E) and no earlier column of
+// token t holds the same id; a valid entry leads its rank when no earlier valid column
+// of t is on the same rank.  Two passes over a tile of ids in shared memory:
+//   pass 1: vid[i] = id if valid else -1 (and error flags)
+//   pass 2: lead[i] = for a leader, the mask of t's valid columns on its rank, else 0
+// Each entry scans only its own token's k <= 32 columns, in parallel over all threads.
+__device__ __forceinline__ uint32_t classify_pass1(const int32_t *ids, int32_t *vid, int n_ent,
+                                                   int k, int E)
 {
-    Entry c;
-    const bool present = lane < k;
-    const bool in_range = present && static_cast<uint32_t>(e) < static_cast<uint32_t>(E);
-    c.flags = (present && !in_range) ? MOE_ERR_ID_RANGE : 0u;
-    // Invalid lanes get a key no valid id can take (valid keys are small non-negative).
-    const int32_t key = in_range ? e : static_cast<int32_t>(0x80000000u | lane);
-    const uint32_t same_id = __match_any_sync(kFull, key);
-    const bool dup = in_range && (same_id & lanemask_lt()) != 0u;
-    if (dup)
-        c.flags |= MOE_ERR_ID_DUP;
-    c.valid = in_range && !dup;
-    c.r = c.valid ? e / epr : -1;
-    const int32_t rkey = c.valid ? c.r : static_cast<int32_t>(0x80000000u | lane);
-    c.same_rank = __match_any_sync(kFull, rkey);
-    c.leader = c.valid && (c.same_rank & lanemask_lt()) == 0u;
-    return c;
+    uint32_t flags = 0;
+    for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
+        const int j = i % k;
+        const int32_t *row = ids + (i - j);
+        const int32_t e = row[j];
+        bool valid = static_cast<uint32_t>(e) < static_cast<uint32_t>(E);
+        if (!valid) {
+            flags |= MOE_ERR_ID_RANGE;
+        } else {
+            for (int q = 0; q < j; ++q)
+                if (row[q] == e) {
+                    valid = false;
+                    flags |= MOE_ERR_ID_DUP;
+                    break;
+                }
+        }
+        vid[i] = valid ? e : -1;
+    }
+    return flags;
+}
+
+// Pass 2 for entry i (vid must be complete).  Returns the leader mask (0 if not a leader).
+__device__ __forceinline__ uint32_t classify_leader(const int32_t *vid, int i, int k, int epr)
+{
+    const int j = i % k;
+    const int32_t *row = vid + (i - j);
+    const int32_t e = row[j];
+    if (e < 0)
+        return 0u;
+    const int32_t r = e / epr;
+    uint32_t mask = 0;
+    for (int q = 0; q < k; ++q) {
+        const int32_t eq = row[q];
+        if (eq >= 0 && eq / epr == r) {
+            if (q < j)
+                return 0u;  // an earlier valid column leads this rank
+            mask |= 1u << q;
+        }
+    }
+    return mask;
 }
 
 // Exclusive block scan of one value per thread; *total gets the block sum.
@@ -111,38 +135,35 @@ __global__ void __launch_bounds__(kPlanThreads)
     int32_t *hist = smem;            // [E]
     int32_t *rhist = hist + E;       // [R]
     int32_t *ids = rhist + R;        // [kPlanTile * k]
+    int32_t *vid = ids + kPlanTile * k;  // [kPlanTile * k]
     __shared__ uint32_t s_err;
 
     const int tile = blockIdx.x;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t t0 = static_cast<int64_t>(tile) * kPlanTile;
     const int64_t left = N - t0;
     const int ntok = static_cast<int>(left < kPlanTile ? left : kPlanTile);
+    const int n_ent = ntok * k;
 
     for (int i = threadIdx.x; i < E + R; i += blockDim.x)
         smem[i] = 0;
     const int32_t *src = topk_idx + t0 * k;
-    for (int i = threadIdx.x; i < ntok * k; i += blockDim.x)
+    for (int i = threadIdx.x; i < n_ent; i += blockDim.x)
         ids[i] = __ldg(src + i);
     if (threadIdx.x == 0)
         s_err = 0;
     __syncthreads();
-
-    uint32_t flags = 0;
-    for (int i = 0; i < kPlanTokensPerWarp; ++i) {
-        const int tl = warp * kPlanTokensPerWarp + i;
-        if (tl >= ntok)
-            break;  // warp-uniform
-        const int32_t e = lane < k ? ids[tl * k + lane] : -1;
-        const Entry c = classify(e, lane, k, E, epr);
-        flags |= c.flags;
-        if (c.valid)
-            atomicAdd(&hist[e], 1);
-        if (c.leader)
-            atomicAdd(&rhist[c.r], 1);
-    }
+    const uint32_t flags = classify_pass1(ids, vid, n_ent, k, E);
     if (flags)
         atomicOr(&s_err, flags);
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
+        const int32_t e = vid[i];
+        if (e < 0)
+            continue;
+        atomicAdd(&hist[e], 1);
+        if (classify_leader(vid, i, k, epr))
+            atomicAdd(&rhist[e / epr], 1);
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
         tile_cnt[static_cast<int64_t>(e) * nt + tile] = hist[e];
@@ -210,6 +231,8 @@ __global__ void __launch_bounds__(kPlanThreads)
     int32_t *wcnt = roff + R + 1;               // [warps][E]
     int32_t *wrcnt = wcnt + kPlanWarps * E;     // [warps][R]
     int32_t *ids = wrcnt + kPlanWarps * R;      // [kPlanTile * k]
+    int32_t *vid = ids + kPlanTile * k;         // [kPlanTile * k]
+    uint32_t *lead = reinterpret_cast<uint32_t *>(vid + kPlanTile * k);  // [kPlanTile * k]
     __shared__ int32_t warp_sums[kPlanThreads / 32];
 
     const int tile = blockIdx.x;
@@ -217,6 +240,7 @@ __global__ void __launch_bounds__(kPlanThreads)
     const int64_t t0 = static_cast<int64_t>(tile) * kPlanTile;
     const int64_t left = N - t0;
     const int ntok = static_cast<int>(left <= 0 ? 0 : (left < kPlanTile ? left : kPlanTile));
+    const int n_ent = ntok * k;
 
     // Segment starts: exclusive scans of the expert and rank totals.
     scan_into(cnt, E, eoff, warp_sums);
@@ -224,7 +248,7 @@ __global__ void __launch_bounds__(kPlanThreads)
     for (int i = threadIdx.x; i < kPlanWarps * (E + R); i += blockDim.x)
         wcnt[i] = 0;  // wcnt and wrcnt are contiguous
     const int32_t *src = topk_idx + t0 * k;
-    for (int i = threadIdx.x; i < ntok * k; i += blockDim.x)
+    for (int i = threadIdx.x; i < n_ent; i += blockDim.x)
         ids[i] = __ldg(src + i);
     __syncthreads();
     if (tile == 0) {
@@ -238,21 +262,20 @@ __global__ void __launch_bounds__(kPlanThreads)
     if (ntok == 0)
         return;  // block-uniform; no barrier follows for this block
 
-    // Per-warp counts of its own tokens.
-    int32_t *my_cnt = wcnt + warp * E;
-    int32_t *my_rcnt = wrcnt + warp * R;
-    const int tw0 = warp * kPlanTokensPerWarp;
-    for (int i = 0; i < kPlanTokensPerWarp; ++i) {
-        const int tl = tw0 + i;
-        if (tl >= ntok)
-            break;
-        const int32_t e = lane < k ? ids[tl * k + lane] : -1;
-        const Entry c = classify(e, lane, k, E, epr);
-        if (c.valid)
-            my_cnt[e] += 1;
-        if (c.leader)
-            my_rcnt[c.r] += 1;
-        __syncwarp();
+    classify_pass1(ids, vid, n_ent, k, E);  // flags were reported by the count kernel
+    __syncthreads();
+    // Leader masks and per-warp counts (warp w owns tokens [16w, 16w + 16) of the tile).
+    for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
+        const int32_t e = vid[i];
+        uint32_t m = 0;
+        if (e >= 0) {
+            const int w = (i / k) / kPlanTokensPerWarp;
+            atomicAdd(&wcnt[w * E + e], 1);
+            m = classify_leader(vid, i, k, epr);
+            if (m)
+                atomicAdd(&wrcnt[w * R + e / epr], 1);
+        }
+        lead[i] = m;
     }
     __syncthreads();
 
@@ -275,18 +298,23 @@ __global__ void __launch_bounds__(kPlanThreads)
     }
     __syncthreads();
 
-    // Ordered walk: one token per step, lane j = column j.
+    // Ordered walk: one token per step, lane j = column j.  The valid columns of a token
+    // hold distinct experts and its leaders distinct ranks, so the lanes of one step never
+    // touch the same counter.
+    int32_t *my_cnt = wcnt + warp * E;
+    int32_t *my_rcnt = wrcnt + warp * R;
+    const int tw0 = warp * kPlanTokensPerWarp;
     uint32_t flags = 0;
-    for (int i = 0; i < kPlanTokensPerWarp; ++i) {
-        const int tl = tw0 + i;
+    for (int q = 0; q < kPlanTokensPerWarp; ++q) {
+        const int tl = tw0 + q;
         if (tl >= ntok)
-            break;
+            break;  // warp-uniform
         const int64_t t = t0 + tl;
-        const int32_t e = lane < k ? ids[tl * k + lane] : -1;
-        const Entry c = classify(e, lane, k, E, epr);
         if (lane < k) {
+            const int i = tl * k + lane;
+            const int32_t e = vid[i];
             int32_t s = -1;
-            if (c.valid) {
+            if (e >= 0) {
                 s = my_cnt[e];
                 my_cnt[e] = s + 1;
                 if (static_cast<uint32_t>(s) < static_cast<uint32_t>(n_rows)) {
@@ -296,18 +324,20 @@ __global__ void __launch_bounds__(kPlanThreads)
                     flags |= MOE_ERR_BOUNDS;
                     s = -1;
                 }
+                const uint32_t m = lead[i];
+                if (m) {
+                    const int32_t r = e / epr;
+                    const int32_t pos = my_rcnt[r];
+                    my_rcnt[r] = pos + 1;
+                    if (pos >= 0 && pos < rtok_cap) {
+                        rtok[pos] = static_cast<int32_t>(t);
+                        fanout[pos] = m;
+                    } else {
+                        flags |= MOE_ERR_BOUNDS;
+                    }
+                }
             }
             slot[t * k + lane] = s;
-        }
-        if (c.leader) {
-            const int32_t pos = my_rcnt[c.r];
-            my_rcnt[c.r] = pos + 1;
-            if (pos >= 0 && pos < rtok_cap) {
-                rtok[pos] = static_cast<int32_t>(t);
-                fanout[pos] = c.same_rank;
-            } else {
-                flags |= MOE_ERR_BOUNDS;
-            }
         }
         __syncwarp();
     }
@@ -315,11 +345,11 @@ __global__ void __launch_bounds__(kPlanThreads)
         atomicOr(err, flags);
 }
 
-size_t count_smem(int E, int R, int k) { return sizeof(int32_t) * (E + R + kPlanTile * k); }
+size_t count_smem(int E, int R, int k) { return sizeof(int32_t) * (E + R + 2 * kPlanTile * k); }
 size_t rank_smem(int E, int R, int k)
 {
     return sizeof(int32_t) *
-           ((E + 1) + (R + 1) + static_cast<size_t>(kPlanWarps) * (E + R) + kPlanTile * k);
+           ((E + 1) + (R + 1) + static_cast<size_t>(kPlanWarps) * (E + R) + 3 * kPlanTile * k);
 }
 
 }  // namespace
