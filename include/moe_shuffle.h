@@ -174,8 +174,11 @@ typedef enum {
     MOE_TUNE_DISPATCH_LAG = 1,           /* store groups a warp keeps in flight (1..stages-1) */
     MOE_TUNE_DISPATCH_CTAS_PER_SM = 2,   /* cap on resident dispatch CTAs per SM */
     MOE_TUNE_DISPATCH_WARPS_PER_CTA = 3, /* dispatch warps per CTA (1..4) */
-    MOE_TUNE_COMBINE_VEC_PER_LANE = 4,   /* 16-byte vectors per lane per combine unit (1, 2, 4) */
-    MOE_TUNE_COMBINE_CTAS_PER_SM = 5     /* cap on resident combine CTAs per SM */
+    MOE_TUNE_COMBINE_VEC_PER_LANE = 4,   /* LSU combine: 16-byte vectors per lane (1, 2, 4) */
+    MOE_TUNE_COMBINE_CTAS_PER_SM = 5,    /* cap on resident combine CTAs per SM */
+    MOE_TUNE_COMBINE_STAGES = 6,         /* bulk combine: shared-memory stages (2..16) */
+    MOE_TUNE_COMBINE_ENGINE = 7,         /* 0 or 1: bulk-copy engine, 2: LSU engine */
+    MOE_TUNE_COMBINE_SMEM_KB = 8         /* bulk combine: shared-memory budget per CTA (KB) */
 } moe_knob;
 
 MOE_API moe_status moe_tune(moe_knob knob, int32_t value);

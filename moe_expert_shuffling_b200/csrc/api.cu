@@ -118,6 +118,9 @@ moe_status moe_tune(moe_knob knob, int32_t value)
     case MOE_TUNE_DISPATCH_WARPS_PER_CTA: t.dispatch_warps_per_cta = value; break;
     case MOE_TUNE_COMBINE_VEC_PER_LANE: t.combine_vec_per_lane = value; break;
     case MOE_TUNE_COMBINE_CTAS_PER_SM: t.combine_ctas_per_sm = value; break;
+    case MOE_TUNE_COMBINE_STAGES: t.combine_stages = value; break;
+    case MOE_TUNE_COMBINE_ENGINE: t.combine_mode = value; break;
+    case MOE_TUNE_COMBINE_SMEM_KB: t.combine_smem_kb = value; break;
     default: return fail(MOE_EINVAL, "unknown tuning knob %d", static_cast<int>(knob));
     }
     return ok();
@@ -307,6 +310,7 @@ moe_status moe_combine(const void *y, int32_t H, moe_plan_t plan, void *out, voi
     a.slot = p->slot;
     a.w = p->topk_w;
     a.out = static_cast<uint16_t *>(out);
+    a.err = p->err;
     a.N = p->N;
     a.k = p->k;
     a.n_rows = p->N * p->k;

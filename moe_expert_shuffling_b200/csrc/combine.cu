@@ -1,13 +1,18 @@
 // Combine: out[t] = bf16_rne( fp32 fma chain over j = 0..k-1 of w[t, j] * y[slot[t, j]] ),
 // starting from +0 -- the expert results of a token brought back and summed (DySHARP blog,
 // sections 1-2).  The chain runs in top-k column order, so every launch configuration
-// gives the same bits.
+// and both engines give the same bits.
 //
-// Engine: a persistent grid of warps over work units (token, column chunk of 32*VPL
-// 16-byte vectors).  A warp reads the token's k slots and weights once (lane j holds
-// column j), then each lane issues all of its KB x VPL row loads before the first fma,
-// so up to KB*VPL 16-byte loads per lane are in flight.  Loads bypass L1 (each byte of
-// y is read once); the output vector is written once with a streaming store.
+// Bulk engine (default): persistent CTAs, one producer warp and four consumer warps.
+// Work unit = (token, 2 KB column chunk of every row).  The producer issues one bulk
+// async copy per routed row chunk (lane j copies row slot[t, j]) into a ring of stages
+// in shared memory, each completing on a "full" mbarrier; consumers take a stage, each
+// thread reduces 8 columns over the k rows from shared memory and writes 16 bytes of
+// out, then release the stage on its "empty" mbarrier.  Bytes in flight are bounded by
+// shared memory (up to ~190 KB per SM) rather than by registers.
+//
+// LSU engine (for comparison): a persistent grid of warps over (token, 32*VPL vector)
+// units; each lane issues its KB x VPL 16-byte loads before the first fma.
 #include <algorithm>
 
 #include <cuda_bf16.h>
@@ -55,7 +60,7 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float *acc)
 }
 
 template <int KB, int VPL>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineParams p)
+__global__ void __launch_bounds__(kCombineThreads) combine_lsu_kernel(const CombineParams p)
 {
     const int lane = threadIdx.x & 31;
     const uint32_t gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -116,10 +121,162 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineP
     }
 }
 
+
+// ------------------------------------------------------------------ bulk engine
+constexpr uint32_t kChunk = 2048;                       // bytes of each row per unit
+constexpr int kConsumerWarps = kChunk / 16 / 32;        // one 16-byte vector per thread
+constexpr int kBulkThreads = 32 * (1 + kConsumerWarps);
+constexpr int kMaxBulkStages = 16;
+
+struct CombineBulkParams {
+    const uint8_t *y;
+    const int32_t *slot;
+    const float *w;
+    uint8_t *out;
+    uint32_t *err;
+    int32_t N, k, n_rows;
+    uint32_t row_bytes, nchunks, stages, stage_bytes, bar_bytes;
+};
+
+__global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const CombineBulkParams p)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int S = static_cast<int>(p.stages);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    uint64_t *empty = full + S;
+    uint8_t *ring = smem + p.bar_bytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int k = p.k;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    const uint32_t b = blockIdx.x, G = gridDim.x;
+    const int n_tok = b < static_cast<uint32_t>(p.N)
+                          ? static_cast<int>((static_cast<uint32_t>(p.N) - b + G - 1) / G)
+                          : 0;
+    const int n_units = n_tok * static_cast<int>(p.nchunks);
+
+    if (warp == 0) {
+        // ---------------- producer: lane j < k copies row slot[t, j]
+        int32_t s_cur = (n_tok > 0 && lane < k) ? __ldg(p.slot + static_cast<int64_t>(b) * k + lane) : -1;
+        int i = 0;
+        bool ok = true;
+        for (int m = 0; m < n_tok && ok; ++m) {
+            const uint32_t t = b + static_cast<uint32_t>(m) * G;
+            int32_t s_nxt = -1;
+            if (m + 1 < n_tok && lane < k)
+                s_nxt = __ldg(p.slot + static_cast<int64_t>(t + G) * k + lane);
+            const bool valid =
+                lane < k && static_cast<uint32_t>(s_cur) < static_cast<uint32_t>(p.n_rows);
+            const uint32_t nv = __popc(__ballot_sync(0xffffffffu, valid));
+            for (uint32_t c = 0; c < p.nchunks; ++c, ++i) {
+                const int st = i % S;
+                const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(&empty[st], ph ^ 1u))) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t off = c * kChunk;
+                const uint32_t len = min(kChunk, p.row_bytes - off);
+                if (lane == 0)
+                    mbar_arrive_expect_tx(&full[st], nv * len);
+                __syncwarp();
+                if (valid)
+                    bulk_load(ring + static_cast<size_t>(st) * p.stage_bytes + lane * kChunk,
+                              p.y + static_cast<int64_t>(s_cur) * p.row_bytes + off, len,
+                              &full[st]);
+            }
+            s_cur = s_nxt;
+        }
+        if (!ok) {
+            if (lane == 0)
+                atomicOr(p.err, MOE_ERR_TIMEOUT);
+            // let the copies of the last stages land before the CTA's memory is released
+            for (int q = (i > S ? i - S : 0); q < i; ++q)
+                (void)mbar_wait_bounded(&full[q % S], static_cast<uint32_t>((q / S) & 1));
+        }
+        return;
+    }
+
+    // ---------------- consumers: thread v owns bytes [16v, 16v + 16) of every chunk
+    const uint32_t v16 = static_cast<uint32_t>(threadIdx.x - 32) * 16u;
+    int32_t s_cur = -1, s_nxt = -1;
+    float w_cur = 0.f, w_nxt = 0.f;
+    if (n_tok > 0 && lane < k) {
+        s_cur = __ldg(p.slot + static_cast<int64_t>(b) * k + lane);
+        w_cur = __ldg(p.w + static_cast<int64_t>(b) * k + lane);
+    }
+    int i = 0;
+    for (int m = 0; m < n_tok; ++m) {
+        const uint32_t t = b + static_cast<uint32_t>(m) * G;
+        if (m + 1 < n_tok && lane < k) {
+            s_nxt = __ldg(p.slot + static_cast<int64_t>(t + G) * k + lane);
+            w_nxt = __ldg(p.w + static_cast<int64_t>(t + G) * k + lane);
+        }
+        bool ok = true;
+        for (uint32_t c = 0; c < p.nchunks; ++c, ++i) {
+            const int st = i % S;
+            const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[st], ph))) {
+                ok = false;
+                break;
+            }
+            const uint32_t off = c * kChunk;
+            const uint32_t len = min(kChunk, p.row_bytes - off);
+            const uint8_t *stage = ring + static_cast<size_t>(st) * p.stage_bytes + v16;
+            float acc[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                acc[e] = 0.f;
+            const bool mine = v16 < len;
+            for (int j0 = 0; j0 < k; j0 += 8) {
+                uint4 q[8];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int j = j0 + jj;
+                    const int32_t sj = __shfl_sync(0xffffffffu, s_cur, j & 31);
+                    const bool use = j < k && mine &&
+                                     static_cast<uint32_t>(sj) < static_cast<uint32_t>(p.n_rows);
+                    q[jj] = use ? lds_v4(stage + j * kChunk) : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int j = j0 + jj;
+                    const int32_t sj = __shfl_sync(0xffffffffu, s_cur, j & 31);
+                    const float wj = __shfl_sync(0xffffffffu, w_cur, j & 31);
+                    if (j < k && static_cast<uint32_t>(sj) < static_cast<uint32_t>(p.n_rows))
+                        fma_bf16x8(acc, wj, q[jj]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[st]);
+            if (mine)
+                st_stream_v4(p.out + static_cast<int64_t>(t) * p.row_bytes + off + v16,
+                             pack_bf16x8(acc));
+        }
+        if (!ok) {
+            if (lane == 0)
+                atomicOr(p.err, MOE_ERR_TIMEOUT);
+            return;
+        }
+        s_cur = s_nxt;
+        w_cur = w_nxt;
+    }
+    (void)n_units;
+}
+
 template <int KB, int VPL>
 cudaError_t launch_one(const CombineParams &p, int device, int ctas_per_sm, cudaStream_t stream)
 {
-    auto kern = combine_kernel<KB, VPL>;
+    auto kern = combine_lsu_kernel<KB, VPL>;
     int per_sm = 0;
     cudaError_t e =
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCombineThreads, 0);
@@ -148,11 +305,68 @@ cudaError_t launch_kb(const CombineParams &p, int vpl, int device, int ctas, cud
 
 }  // namespace
 
+cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t stream)
+{
+    const Tuning &tu = tuning();
+    CombineBulkParams p;
+    p.y = reinterpret_cast<const uint8_t *>(a.y);
+    p.slot = a.slot;
+    p.w = a.w;
+    p.out = reinterpret_cast<uint8_t *>(a.out);
+    p.err = a.err;
+    p.N = a.N;
+    p.k = a.k;
+    p.n_rows = a.n_rows;
+    p.row_bytes = static_cast<uint32_t>(a.H) * 2u;
+    p.nchunks = static_cast<uint32_t>(ceil_div(p.row_bytes, kChunk));
+    p.stage_bytes = static_cast<uint32_t>(a.k) * kChunk;
+
+    int max_optin = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                           device);
+    if (e != cudaSuccess)
+        return e;
+    const int budget = tu.combine_smem_kb > 0 ? std::min(tu.combine_smem_kb * 1024, max_optin)
+                                              : std::min(200 * 1024, max_optin);
+    int S = tu.combine_stages > 0 ? tu.combine_stages : kMaxBulkStages;
+    S = std::min(S, kMaxBulkStages);
+    auto smem_for = [&](int st) {
+        return static_cast<size_t>(round_up(2 * st * 8, 128)) +
+               static_cast<size_t>(st) * p.stage_bytes;
+    };
+    while (S > 2 && smem_for(S) > static_cast<size_t>(budget))
+        --S;
+    if (smem_for(S) > static_cast<size_t>(max_optin))
+        return cudaErrorInvalidValue;
+    p.stages = static_cast<uint32_t>(S);
+    p.bar_bytes = static_cast<uint32_t>(round_up(2 * S * 8, 128));
+    const size_t smem = smem_for(S);
+    e = cudaFuncSetAttribute(combine_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess)
+        return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_bulk_kernel, kBulkThreads,
+                                                      smem);
+    if (e != cudaSuccess)
+        return e;
+    if (per_sm < 1)
+        return cudaErrorInvalidConfiguration;
+    if (tu.combine_ctas_per_sm > 0)
+        per_sm = std::min(per_sm, tu.combine_ctas_per_sm);
+    const int64_t grid =
+        std::max<int64_t>(1, std::min<int64_t>(a.N, static_cast<int64_t>(sm_count(device)) * per_sm));
+    combine_bulk_kernel<<<static_cast<unsigned>(grid), kBulkThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const CombineArgs &a, int device, cudaStream_t stream)
 {
     if (a.N == 0)
         return cudaSuccess;
     const Tuning &tu = tuning();
+    if (tu.combine_mode != 2)
+        return launch_combine_bulk(a, device, stream);
     int vpl = tu.combine_vec_per_lane > 0 ? tu.combine_vec_per_lane : 1;
     if (vpl != 1 && vpl != 2 && vpl != 4)
         vpl = 1;

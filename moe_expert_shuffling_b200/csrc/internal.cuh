@@ -44,6 +44,9 @@ struct Tuning {
     int dispatch_warps_per_cta = 0;
     int combine_vec_per_lane = 0;
     int combine_ctas_per_sm = 0;
+    int combine_stages = 0;
+    int combine_mode = 0;      // 0/1: bulk engine, 2: LSU engine
+    int combine_smem_kb = 0;
 };
 Tuning &tuning();
 
@@ -68,6 +71,7 @@ struct CombineArgs {
     const int32_t *slot;   // [N*k]
     const float *w;        // [N*k]
     uint16_t *out;         // bf16 [N, H]
+    uint32_t *err;
     int32_t N, k, n_rows, H;
 };
 cudaError_t launch_combine(const CombineArgs &a, int device, cudaStream_t stream);

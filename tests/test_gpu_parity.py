@@ -99,8 +99,14 @@ def test_identity_experts_return_x(name):
     CONFIGS["long"].replace(N=50, H=65536),                                # chunked fp8 row
     CONFIGS["long"].replace(N=1000, H=512, k=4, E=16, R=16),
 ], ids=lambda c: f"{c.name}-N{c.N}-H{c.H}-E{c.E}-k{c.k}-R{c.R}-{c.payload}")
-def test_edge_shapes(cfg):
-    r = run_all(cfg, 0)
+@pytest.mark.parametrize("engine", [0, 2], ids=["bulk", "lsu"])
+def test_edge_shapes(cfg, engine):
+    import moe_expert_shuffling_b200 as ms
+    ms.moe_tune("combine_engine", engine)
+    try:
+        r = run_all(cfg, 0)
+    finally:
+        ms.moe_tune("combine_engine", 0)
     assert_plan_equal(r["gp"], r["ref"])
     assert np.array_equal(r["got_recv"], r["ref_recv"])
     if r["ref_rs"] is not None:
@@ -189,8 +195,11 @@ def test_invalid_routing_is_flagged_and_contained():
     {"dispatch_stages": 2, "dispatch_lag": 1},
     {"dispatch_stages": 8, "dispatch_lag": 4, "dispatch_warps_per_cta": 2},
     {"dispatch_ctas_per_sm": 1, "combine_ctas_per_sm": 1},
-    {"combine_vec_per_lane": 1},
-    {"combine_vec_per_lane": 4},
+    {"combine_engine": 2, "combine_vec_per_lane": 1},
+    {"combine_engine": 2, "combine_vec_per_lane": 2},
+    {"combine_engine": 2, "combine_vec_per_lane": 4},
+    {"combine_stages": 2},
+    {"combine_smem_kb": 64, "combine_ctas_per_sm": 2},
 ])
 def test_launch_configuration_does_not_change_results(knobs):
     import moe_expert_shuffling_b200 as ms
