@@ -127,6 +127,7 @@ constexpr uint32_t kChunk = 2048;                       // bytes of each row per
 constexpr int kConsumerWarps = kChunk / 16 / 32;        // one 16-byte vector per thread
 constexpr int kBulkThreads = 32 * (1 + kConsumerWarps);
 constexpr int kMaxBulkStages = 16;
+constexpr int kDefaultSmemBudget = 64 * 1024;
 
 struct CombineBulkParams {
     const uint8_t *y;
@@ -326,8 +327,9 @@ cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t s
                                            device);
     if (e != cudaSuccess)
         return e;
+    // Several CTAs per SM (more consumer warps) beat one CTA with a deeper ring.
     const int budget = tu.combine_smem_kb > 0 ? std::min(tu.combine_smem_kb * 1024, max_optin)
-                                              : std::min(200 * 1024, max_optin);
+                                              : std::min(kDefaultSmemBudget, max_optin);
     int S = tu.combine_stages > 0 ? tu.combine_stages : kMaxBulkStages;
     S = std::min(S, kMaxBulkStages);
     auto smem_for = [&](int st) {

@@ -4,16 +4,18 @@
 // transfers; DySHARP blog, section 5: the destination maps a token's logical index to a
 // local address -- slot[t, j] is that map.
 //
-// Three kernels, all deterministic (counts are order-free; ranks follow token order):
+// Three kernels, all deterministic (no result depends on thread timing):
 //   plan_count  one CTA per tile of 128 tokens: per-tile expert counts and per-tile
 //               counts of (token, rank) moves -> scratch [E][tiles], [R][tiles]
 //   plan_scan   one CTA per expert row and per rank row: exclusive scan over tiles,
 //               row totals -> cnt[E], rcnt[R]; CTA 0 also gathers the tile flags
-//   plan_rank   one CTA per tile: segment starts (scan of cnt/rcnt), entry classes and
-//               per-warp counts in parallel over the tile's entries, then each warp
-//               walks its 16 tokens in order, one token per step with lane j holding
-//               column j.  The valid ids of one token are distinct, so the lanes of a
-//               step touch distinct counters and the walk needs no atomics.
+//   plan_rank   one CTA per tile: segment starts, then every entry's stable rank inside
+//               its segment as a popcount over a per-expert bitmask of the tile's tokens
+//               (bit t set when token t selects the expert), so no step is sequential.
+//
+// Inside a tile a warp looks at several tokens at once: lane = (token, column) with the
+// columns of one token in a segment of W = next power of two >= k lanes, so a token's
+// k ids are compared with width-W shuffles.
 #include "common.cuh"
 #include "internal.cuh"
 
@@ -24,56 +26,73 @@ constexpr int kPlanThreads = kPlanWarps * 32;
 constexpr int kScanThreads = 256;
 constexpr uint32_t kFull = 0xffffffffu;  // all lanes of a warp
 
-// Entry classification, shared by the count and rank kernels so both see the same
-// entries.  An entry (t, j) is valid when its id is in [0, E) and no earlier column of
+// Classification of one entry, shared by the count and rank kernels so both see the
+// same entries.  Entry (t, j) is valid when its id is in [0, E) and no earlier column of
 // token t holds the same id; a valid entry leads its rank when no earlier valid column
-// of t is on the same rank.  Two passes over a tile of ids in shared memory:
-//   pass 1: vid[i] = id if valid else -1 (and error flags)
-//   pass 2: lead[i] = for a leader, the mask of t's valid columns on its rank, else 0
-// Each entry scans only its own token's k <= 32 columns, in parallel over all threads.
-__device__ __forceinline__ uint32_t classify_pass1(const int32_t *ids, int32_t *vid, int n_ent,
-                                                   int k, int E)
+// of t is on that rank, and then carries the mask of t's valid columns on the rank.
+struct Entry {
+    int32_t e;        // the id if valid, else -1
+    int32_t r;        // its rank if valid, else -1
+    uint32_t lead;    // mask of the token's valid columns on rank r if this entry leads
+    uint32_t flags;   // MOE_ERR_* raised by this entry
+};
+
+// Lane layout of a warp step: `wbits` = log2 of the segment width W >= k.
+struct LaneMap {
+    int wbits, per_step, steps;
+};
+
+__device__ __forceinline__ LaneMap lane_map(int k)
 {
-    uint32_t flags = 0;
-    for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
-        const int j = i % k;
-        const int32_t *row = ids + (i - j);
-        const int32_t e = row[j];
-        bool valid = static_cast<uint32_t>(e) < static_cast<uint32_t>(E);
-        if (!valid) {
-            flags |= MOE_ERR_ID_RANGE;
-        } else {
-            for (int q = 0; q < j; ++q)
-                if (row[q] == e) {
-                    valid = false;
-                    flags |= MOE_ERR_ID_DUP;
-                    break;
-                }
-        }
-        vid[i] = valid ? e : -1;
-    }
-    return flags;
+    LaneMap m;
+    m.wbits = 0;
+    while ((1 << m.wbits) < k)
+        ++m.wbits;
+    m.per_step = 32 >> m.wbits;  // tokens per warp step
+    m.steps = (kPlanTokensPerWarp + m.per_step - 1) / m.per_step;
+    return m;
 }
 
-// Pass 2 for entry i (vid must be complete).  Returns the leader mask (0 if not a leader).
-__device__ __forceinline__ uint32_t classify_leader(const int32_t *vid, int i, int k, int epr)
+// All 32 lanes must call.  `tl` is the token's index in the tile, `present` whether
+// this lane holds an entry (token in range and column < k).
+__device__ __forceinline__ Entry classify(const int32_t *ids, const int32_t *rank_of, int tl,
+                                          int j, bool present, int k, int E, int width)
 {
-    const int j = i % k;
-    const int32_t *row = vid + (i - j);
-    const int32_t e = row[j];
-    if (e < 0)
-        return 0u;
-    const int32_t r = e / epr;
-    uint32_t mask = 0;
+    Entry c;
+    const int32_t id = present ? ids[tl * k + j] : -1;
+    const bool in_range = present && static_cast<uint32_t>(id) < static_cast<uint32_t>(E);
+    bool valid = in_range;
     for (int q = 0; q < k; ++q) {
-        const int32_t eq = row[q];
-        if (eq >= 0 && eq / epr == r) {
+        const int32_t iq = __shfl_sync(kFull, id, q, width);
+        if (q < j && iq == id)
+            valid = false;
+    }
+    c.flags = (present && !in_range ? MOE_ERR_ID_RANGE : 0u) |
+              (in_range && !valid ? MOE_ERR_ID_DUP : 0u);
+    c.e = valid ? id : -1;
+    c.r = valid ? rank_of[id] : -1;
+    uint32_t mask = 0;
+    bool leader = valid;
+    for (int q = 0; q < k; ++q) {
+        const int32_t rq = __shfl_sync(kFull, c.r, q, width);
+        if (valid && rq == c.r) {
             if (q < j)
-                return 0u;  // an earlier valid column leads this rank
+                leader = false;
             mask |= 1u << q;
         }
     }
-    return mask;
+    c.lead = leader ? mask : 0u;
+    return c;
+}
+
+// Number of set bits of a 128-bit tile mask below bit `tl`.
+__device__ __forceinline__ int32_t bits_below(const uint32_t *m4, int tl)
+{
+    const int w = tl >> 5;
+    int32_t n = __popc(m4[w] & ((1u << (tl & 31)) - 1u));
+    for (int q = 0; q < w; ++q)
+        n += __popc(m4[q]);
+    return n;
 }
 
 // Exclusive block scan of one value per thread; *total gets the block sum.
@@ -134,36 +153,44 @@ __global__ void __launch_bounds__(kPlanThreads)
     extern __shared__ int32_t smem[];
     int32_t *hist = smem;            // [E]
     int32_t *rhist = hist + E;       // [R]
-    int32_t *ids = rhist + R;        // [kPlanTile * k]
-    int32_t *vid = ids + kPlanTile * k;  // [kPlanTile * k]
+    int32_t *rank_of = rhist + R;    // [E]
+    int32_t *ids = rank_of + E;      // [kPlanTile * k]
     __shared__ uint32_t s_err;
 
     const int tile = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t t0 = static_cast<int64_t>(tile) * kPlanTile;
     const int64_t left = N - t0;
     const int ntok = static_cast<int>(left < kPlanTile ? left : kPlanTile);
-    const int n_ent = ntok * k;
 
     for (int i = threadIdx.x; i < E + R; i += blockDim.x)
         smem[i] = 0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        rank_of[e] = e / epr;
     const int32_t *src = topk_idx + t0 * k;
-    for (int i = threadIdx.x; i < n_ent; i += blockDim.x)
+    for (int i = threadIdx.x; i < ntok * k; i += blockDim.x)
         ids[i] = __ldg(src + i);
     if (threadIdx.x == 0)
         s_err = 0;
     __syncthreads();
-    const uint32_t flags = classify_pass1(ids, vid, n_ent, k, E);
+
+    const LaneMap lm = lane_map(k);
+    const int j = lane & ((1 << lm.wbits) - 1);
+    const int sub = lane >> lm.wbits;
+    uint32_t flags = 0;
+    for (int st = 0; st < lm.steps; ++st) {
+        const int tw = st * lm.per_step + sub;           // token within the warp's 16
+        const int tl = warp * kPlanTokensPerWarp + tw;
+        const bool present = tw < kPlanTokensPerWarp && tl < ntok && j < k;
+        const Entry c = classify(ids, rank_of, tl, j, present, k, E, 1 << lm.wbits);
+        flags |= c.flags;
+        if (c.e >= 0)
+            atomicAdd(&hist[c.e], 1);
+        if (c.lead)
+            atomicAdd(&rhist[c.r], 1);
+    }
     if (flags)
         atomicOr(&s_err, flags);
-    __syncthreads();
-    for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
-        const int32_t e = vid[i];
-        if (e < 0)
-            continue;
-        atomicAdd(&hist[e], 1);
-        if (classify_leader(vid, i, k, epr))
-            atomicAdd(&rhist[e / epr], 1);
-    }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
         tile_cnt[static_cast<int64_t>(e) * nt + tile] = hist[e];
@@ -226,12 +253,13 @@ __global__ void __launch_bounds__(kPlanThreads)
                      uint32_t *__restrict__ err)
 {
     extern __shared__ int32_t smem[];
-    int32_t *eoff = smem;                       // [E+1]
-    int32_t *roff = eoff + E + 1;               // [R+1]
-    int32_t *wcnt = roff + R + 1;               // [warps][E]
-    int32_t *wrcnt = wcnt + kPlanWarps * E;     // [warps][R]
-    int32_t *ids = wrcnt + kPlanWarps * R;      // [kPlanTile * k]
-    int32_t *vid = ids + kPlanTile * k;         // [kPlanTile * k]
+    int32_t *ebase = smem;                        // [E+1] segment starts, then tile bases
+    int32_t *rbase = ebase + E + 1;               // [R+1]
+    int32_t *rank_of = rbase + R + 1;             // [E]
+    uint32_t *emask = reinterpret_cast<uint32_t *>(rank_of + E);  // [E][4] tokens per expert
+    uint32_t *rmask = emask + 4 * E;              // [R][4] tokens per rank
+    int32_t *ids = reinterpret_cast<int32_t *>(rmask + 4 * R);    // [kPlanTile * k]
+    int32_t *vid = ids + kPlanTile * k;           // [kPlanTile * k] valid id or -1
     uint32_t *lead = reinterpret_cast<uint32_t *>(vid + kPlanTile * k);  // [kPlanTile * k]
     __shared__ int32_t warp_sums[kPlanThreads / 32];
 
@@ -240,116 +268,98 @@ __global__ void __launch_bounds__(kPlanThreads)
     const int64_t t0 = static_cast<int64_t>(tile) * kPlanTile;
     const int64_t left = N - t0;
     const int ntok = static_cast<int>(left <= 0 ? 0 : (left < kPlanTile ? left : kPlanTile));
-    const int n_ent = ntok * k;
 
     // Segment starts: exclusive scans of the expert and rank totals.
-    scan_into(cnt, E, eoff, warp_sums);
-    scan_into(rcnt, R, roff, warp_sums);
-    for (int i = threadIdx.x; i < kPlanWarps * (E + R); i += blockDim.x)
-        wcnt[i] = 0;  // wcnt and wrcnt are contiguous
+    scan_into(cnt, E, ebase, warp_sums);
+    scan_into(rcnt, R, rbase, warp_sums);
+    for (int i = threadIdx.x; i < 4 * (E + R); i += blockDim.x)
+        emask[i] = 0u;  // emask and rmask are contiguous
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        rank_of[e] = e / epr;
     const int32_t *src = topk_idx + t0 * k;
-    for (int i = threadIdx.x; i < n_ent; i += blockDim.x)
+    for (int i = threadIdx.x; i < ntok * k; i += blockDim.x)
         ids[i] = __ldg(src + i);
     __syncthreads();
     if (tile == 0) {
         for (int i = threadIdx.x; i <= E; i += blockDim.x)
-            expert_off[i] = eoff[i];
+            expert_off[i] = ebase[i];
         for (int i = threadIdx.x; i <= R; i += blockDim.x) {
-            rtok_off[i] = roff[i];
-            rank_off[i] = eoff[i * epr];
+            rtok_off[i] = rbase[i];
+            rank_off[i] = ebase[i * epr];
         }
     }
     if (ntok == 0)
         return;  // block-uniform; no barrier follows for this block
-
-    classify_pass1(ids, vid, n_ent, k, E);  // flags were reported by the count kernel
     __syncthreads();
-    // Leader masks and per-warp counts (warp w owns tokens [16w, 16w + 16) of the tile).
-    for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
-        const int32_t e = vid[i];
-        uint32_t m = 0;
-        if (e >= 0) {
-            const int w = (i / k) / kPlanTokensPerWarp;
-            atomicAdd(&wcnt[w * E + e], 1);
-            m = classify_leader(vid, i, k, epr);
-            if (m)
-                atomicAdd(&wrcnt[w * R + e / epr], 1);
-        }
-        lead[i] = m;
-    }
-    __syncthreads();
+    // This tile's first receive row per expert and first dedup entry per rank.
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        ebase[e] += tile_cnt[static_cast<int64_t>(e) * nt + tile];
+    for (int r = threadIdx.x; r < R; r += blockDim.x)
+        rbase[r] += tile_rcnt[static_cast<int64_t>(r) * nt + tile];
 
-    // Start of each warp's run: segment start + earlier tiles + earlier warps of this tile.
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int32_t run = eoff[e] + tile_cnt[static_cast<int64_t>(e) * nt + tile];
-        for (int w = 0; w < kPlanWarps; ++w) {
-            const int32_t v = wcnt[w * E + e];
-            wcnt[w * E + e] = run;
-            run += v;
-        }
-    }
-    for (int r = threadIdx.x; r < R; r += blockDim.x) {
-        int32_t run = roff[r] + tile_rcnt[static_cast<int64_t>(r) * nt + tile];
-        for (int w = 0; w < kPlanWarps; ++w) {
-            const int32_t v = wrcnt[w * R + r];
-            wrcnt[w * R + r] = run;
-            run += v;
+    // Pass A: classify, and mark each token in its expert's and rank's tile mask.
+    const LaneMap lm = lane_map(k);
+    const int j = lane & ((1 << lm.wbits) - 1);
+    const int sub = lane >> lm.wbits;
+    for (int st = 0; st < lm.steps; ++st) {
+        const int tw = st * lm.per_step + sub;
+        const int tl = warp * kPlanTokensPerWarp + tw;
+        const bool present = tw < kPlanTokensPerWarp && tl < ntok && j < k;
+        const Entry c = classify(ids, rank_of, tl, j, present, k, E, 1 << lm.wbits);
+        if (present) {
+            vid[tl * k + j] = c.e;
+            lead[tl * k + j] = c.lead;
+            const uint32_t bit = 1u << (tl & 31);
+            if (c.e >= 0)
+                atomicOr(&emask[4 * c.e + (tl >> 5)], bit);
+            if (c.lead)
+                atomicOr(&rmask[4 * c.r + (tl >> 5)], bit);
         }
     }
     __syncthreads();
 
-    // Ordered walk: one token per step, lane j = column j.  The valid columns of a token
-    // hold distinct experts and its leaders distinct ranks, so the lanes of one step never
-    // touch the same counter.
-    int32_t *my_cnt = wcnt + warp * E;
-    int32_t *my_rcnt = wrcnt + warp * R;
-    const int tw0 = warp * kPlanTokensPerWarp;
+    // Pass B: stable rank = tile base + earlier tokens of the tile on the same expert.
     uint32_t flags = 0;
-    for (int q = 0; q < kPlanTokensPerWarp; ++q) {
-        const int tl = tw0 + q;
-        if (tl >= ntok)
-            break;  // warp-uniform
+    for (int st = 0; st < lm.steps; ++st) {
+        const int tw = st * lm.per_step + sub;
+        const int tl = warp * kPlanTokensPerWarp + tw;
+        if (!(tw < kPlanTokensPerWarp && tl < ntok && j < k))
+            continue;
         const int64_t t = t0 + tl;
-        if (lane < k) {
-            const int i = tl * k + lane;
-            const int32_t e = vid[i];
-            int32_t s = -1;
-            if (e >= 0) {
-                s = my_cnt[e];
-                my_cnt[e] = s + 1;
-                if (static_cast<uint32_t>(s) < static_cast<uint32_t>(n_rows)) {
-                    src_tok[s] = static_cast<int32_t>(t);
-                    src_j[s] = lane;
+        const int i = tl * k + j;
+        const int32_t e = vid[i];
+        int32_t s = -1;
+        if (e >= 0) {
+            s = ebase[e] + bits_below(&emask[4 * e], tl);
+            if (static_cast<uint32_t>(s) < static_cast<uint32_t>(n_rows)) {
+                src_tok[s] = static_cast<int32_t>(t);
+                src_j[s] = j;
+            } else {
+                flags |= MOE_ERR_BOUNDS;
+                s = -1;
+            }
+            const uint32_t m = lead[i];
+            if (m) {
+                const int32_t r = rank_of[e];
+                const int32_t pos = rbase[r] + bits_below(&rmask[4 * r], tl);
+                if (pos >= 0 && pos < rtok_cap) {
+                    rtok[pos] = static_cast<int32_t>(t);
+                    fanout[pos] = m;
                 } else {
                     flags |= MOE_ERR_BOUNDS;
-                    s = -1;
-                }
-                const uint32_t m = lead[i];
-                if (m) {
-                    const int32_t r = e / epr;
-                    const int32_t pos = my_rcnt[r];
-                    my_rcnt[r] = pos + 1;
-                    if (pos >= 0 && pos < rtok_cap) {
-                        rtok[pos] = static_cast<int32_t>(t);
-                        fanout[pos] = m;
-                    } else {
-                        flags |= MOE_ERR_BOUNDS;
-                    }
                 }
             }
-            slot[t * k + lane] = s;
         }
-        __syncwarp();
+        slot[t * k + j] = s;
     }
     if (flags)
         atomicOr(err, flags);
 }
 
-size_t count_smem(int E, int R, int k) { return sizeof(int32_t) * (E + R + 2 * kPlanTile * k); }
+size_t count_smem(int E, int R, int k) { return sizeof(int32_t) * (2 * E + R + kPlanTile * k); }
 size_t rank_smem(int E, int R, int k)
 {
-    return sizeof(int32_t) *
-           ((E + 1) + (R + 1) + static_cast<size_t>(kPlanWarps) * (E + R) + 3 * kPlanTile * k);
+    return sizeof(int32_t) * ((E + 1) + (R + 1) + E + 4 * (E + R) + 3 * kPlanTile * k);
 }
 
 }  // namespace
