@@ -178,7 +178,9 @@ typedef enum {
     MOE_TUNE_COMBINE_CTAS_PER_SM = 5,    /* cap on resident combine CTAs per SM */
     MOE_TUNE_COMBINE_STAGES = 6,         /* bulk combine: shared-memory stages (2..16) */
     MOE_TUNE_COMBINE_ENGINE = 7,         /* 0 or 1: bulk-copy engine, 2: LSU engine */
-    MOE_TUNE_COMBINE_SMEM_KB = 8         /* bulk combine: shared-memory budget per CTA (KB) */
+    MOE_TUNE_COMBINE_SMEM_KB = 8,        /* bulk combine: shared-memory budget per CTA (KB) */
+    MOE_TUNE_DISPATCH_UNITS_PER_WARP = 9, /* (token, chunk) units per dispatch warp */
+    MOE_TUNE_COMBINE_TOKENS_PER_CTA = 10 /* tokens per bulk-combine CTA */
 } moe_knob;
 
 MOE_API moe_status moe_tune(moe_knob knob, int32_t value);

@@ -121,6 +121,8 @@ moe_status moe_tune(moe_knob knob, int32_t value)
     case MOE_TUNE_COMBINE_STAGES: t.combine_stages = value; break;
     case MOE_TUNE_COMBINE_ENGINE: t.combine_mode = value; break;
     case MOE_TUNE_COMBINE_SMEM_KB: t.combine_smem_kb = value; break;
+    case MOE_TUNE_DISPATCH_UNITS_PER_WARP: t.dispatch_units_per_warp = value; break;
+    case MOE_TUNE_COMBINE_TOKENS_PER_CTA: t.combine_tokens_per_cta = value; break;
     default: return fail(MOE_EINVAL, "unknown tuning knob %d", static_cast<int>(knob));
     }
     return ok();

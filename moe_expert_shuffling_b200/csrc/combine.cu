@@ -131,6 +131,7 @@ constexpr int kMaxBulkStages = 16;
 // SM, spread over 4 CTAs, is fastest; deeper rings or more CTAs are slower.
 constexpr int kDefaultSmemBudget = 32 * 1024 + 128;
 constexpr int kDefaultCtasPerSm = 4;
+constexpr int kDefaultTokensPerCta = 16;
 
 struct CombineBulkParams {
     const uint8_t *y;
@@ -140,6 +141,7 @@ struct CombineBulkParams {
     uint32_t *err;
     int32_t N, k, n_rows;
     uint32_t row_bytes, nchunks, stages, stage_bytes, bar_bytes;
+    uint32_t per_cta;       // tokens of each CTA: [cta * per_cta, +per_cta)
 };
 
 __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const CombineBulkParams p)
@@ -161,11 +163,10 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
     }
     __syncthreads();
 
-    const uint32_t b = blockIdx.x, G = gridDim.x;
+    const uint32_t b = blockIdx.x * p.per_cta;  // this CTA's first token
     const int n_tok = b < static_cast<uint32_t>(p.N)
-                          ? static_cast<int>((static_cast<uint32_t>(p.N) - b + G - 1) / G)
+                          ? static_cast<int>(min(p.per_cta, static_cast<uint32_t>(p.N) - b))
                           : 0;
-    const int n_units = n_tok * static_cast<int>(p.nchunks);
 
     if (warp == 0) {
         // ---------------- producer: lane j < k copies row slot[t, j]
@@ -173,10 +174,10 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
         int i = 0;
         bool ok = true;
         for (int m = 0; m < n_tok && ok; ++m) {
-            const uint32_t t = b + static_cast<uint32_t>(m) * G;
+            const uint32_t t = b + static_cast<uint32_t>(m);
             int32_t s_nxt = -1;
             if (m + 1 < n_tok && lane < k)
-                s_nxt = __ldg(p.slot + static_cast<int64_t>(t + G) * k + lane);
+                s_nxt = __ldg(p.slot + static_cast<int64_t>(t + 1) * k + lane);
             const bool valid =
                 lane < k && static_cast<uint32_t>(s_cur) < static_cast<uint32_t>(p.n_rows);
             const uint32_t nv = __popc(__ballot_sync(0xffffffffu, valid));
@@ -219,10 +220,10 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
     }
     int i = 0;
     for (int m = 0; m < n_tok; ++m) {
-        const uint32_t t = b + static_cast<uint32_t>(m) * G;
+        const uint32_t t = b + static_cast<uint32_t>(m);
         if (m + 1 < n_tok && lane < k) {
-            s_nxt = __ldg(p.slot + static_cast<int64_t>(t + G) * k + lane);
-            w_nxt = __ldg(p.w + static_cast<int64_t>(t + G) * k + lane);
+            s_nxt = __ldg(p.slot + static_cast<int64_t>(t + 1) * k + lane);
+            w_nxt = __ldg(p.w + static_cast<int64_t>(t + 1) * k + lane);
         }
         bool ok = true;
         for (uint32_t c = 0; c < p.nchunks; ++c, ++i) {
@@ -274,7 +275,6 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
         s_cur = s_nxt;
         w_cur = w_nxt;
     }
-    (void)n_units;
 }
 
 template <int KB, int VPL>
@@ -359,8 +359,15 @@ cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t s
         return cudaErrorInvalidConfiguration;
     per_sm = std::min(per_sm, tu.combine_ctas_per_sm > 0 ? tu.combine_ctas_per_sm
                                                           : kDefaultCtasPerSm);
-    const int64_t grid =
-        std::max<int64_t>(1, std::min<int64_t>(a.N, static_cast<int64_t>(sm_count(device)) * per_sm));
+    // Contiguous runs of tokens per CTA; the grid covers all tokens so that CTAs that
+    // finish early are replaced by the block scheduler.
+    const int64_t resident = static_cast<int64_t>(sm_count(device)) * per_sm;
+    int64_t per_cta = tu.combine_tokens_per_cta > 0 ? tu.combine_tokens_per_cta
+                                                    : kDefaultTokensPerCta;
+    if (ceil_div(a.N, per_cta) < resident)
+        per_cta = std::max<int64_t>(1, ceil_div(a.N, resident));
+    p.per_cta = static_cast<uint32_t>(per_cta);
+    const int64_t grid = std::max<int64_t>(1, ceil_div(a.N, per_cta));
     combine_bulk_kernel<<<static_cast<unsigned>(grid), kBulkThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }

@@ -2,7 +2,7 @@
 // produced by the copy itself (FUSCO, arXiv 2512.22036, abstract; FUSCO summary, Group 3:
 // data is placed at its destination with no staging buffer and no later rearrangement).
 //
-// Engine: a persistent grid of warps, each running its own pipeline over work units
+// Engine: warps each running their own pipeline over a contiguous run of work units
 // (token, row chunk).  Lane 0 stages a chunk of x[t] into shared memory with one bulk
 // async copy (cp.async.bulk, completion on an mbarrier); once it has landed, lane j
 // issues the bulk store of that chunk to receive row slot[t, j].  So every token row
@@ -21,6 +21,7 @@ namespace {
 
 constexpr uint32_t kMaxChunkBytes = 32768;
 constexpr int kMaxStages = 8;
+constexpr int kDefaultUnitsPerWarp = 8;
 
 struct DispatchParams {
     const uint8_t *x;
@@ -30,6 +31,7 @@ struct DispatchParams {
     const int32_t *slot;
     uint32_t *err;
     uint32_t units;         // N * nchunks (< 2^31)
+    uint32_t per_warp;      // units of each warp: [warp * per_warp, +per_warp)
     int32_t k, n_rows;
     uint32_t nchunks;
     int32_t stages, lag;
@@ -46,8 +48,8 @@ __global__ void __launch_bounds__(128) dispatch_bulk_kernel(const DispatchParams
     uint8_t *stage0 = smem + p.bar_bytes + static_cast<size_t>(wid) * S * p.stage_bytes;
 
     const uint32_t gw = blockIdx.x * wpc + wid;
-    const uint32_t nw = gridDim.x * wpc;
-    const int n_my = gw < p.units ? static_cast<int>((p.units - gw + nw - 1) / nw) : 0;
+    const uint32_t u0 = gw * p.per_warp;  // this warp's first unit
+    const int n_my = u0 < p.units ? static_cast<int>(min(p.per_warp, p.units - u0)) : 0;
 
     if (lane == 0) {
         for (int s = 0; s < S; ++s)
@@ -58,7 +60,7 @@ __global__ void __launch_bounds__(128) dispatch_bulk_kernel(const DispatchParams
 
     // Issue the load of this warp's i-th unit into stage i % S (lane 0 only).
     auto issue_load = [&](int i) {
-        const uint32_t u = gw + static_cast<uint32_t>(i) * nw;
+        const uint32_t u = u0 + static_cast<uint32_t>(i);
         const uint32_t t = u / p.nchunks;
         const uint32_t c = u - t * p.nchunks;
         const uint32_t off = c * p.chunk_bytes;
@@ -80,14 +82,14 @@ __global__ void __launch_bounds__(128) dispatch_bulk_kernel(const DispatchParams
 
     int32_t cur = -1;
     if (n_my > 0 && lane < p.k)
-        cur = __ldg(p.slot + (gw / p.nchunks) * p.k + lane);
+        cur = __ldg(p.slot + (u0 / p.nchunks) * p.k + lane);
 
     bool ok = true;
     int i = 0;
     for (; i < n_my; ++i) {
         const int s = i % S;
         const uint32_t parity = static_cast<uint32_t>((i / S) & 1);
-        const uint32_t u = gw + static_cast<uint32_t>(i) * nw;
+        const uint32_t u = u0 + static_cast<uint32_t>(i);
         const uint32_t t = u / p.nchunks;
         const uint32_t c = u - t * p.nchunks;
         const uint32_t off = c * p.chunk_bytes;
@@ -96,7 +98,7 @@ __global__ void __launch_bounds__(128) dispatch_bulk_kernel(const DispatchParams
         // Slots of the next unit, fetched while this unit's row is in flight.
         int32_t nxt = -1;
         if (i + 1 < n_my && lane < p.k)
-            nxt = __ldg(p.slot + ((u + nw) / p.nchunks) * p.k + lane);
+            nxt = __ldg(p.slot + ((u + 1) / p.nchunks) * p.k + lane);
 
         const bool landed = mbar_wait_bounded(&bars[s], parity);
         if (!__all_sync(0xffffffffu, landed)) {
@@ -229,9 +231,15 @@ cudaError_t launch_dispatch(const DispatchArgs &a, int device, cudaStream_t stre
     p.bar_bytes = static_cast<uint32_t>(round_up(static_cast<int64_t>(wpc) * stages * 8, 128));
     p.bulk_scales = bulk_scales;
 
-    const int64_t warps_needed = p.units;
-    const int64_t grid = std::max<int64_t>(
-        1, std::min<int64_t>(ceil_div(warps_needed, wpc), static_cast<int64_t>(sm_count(device)) * per_sm));
+    // Each warp takes a contiguous run of units; the grid covers all of them, so CTAs
+    // that finish early are replaced by the block scheduler (balances the tail).
+    const int64_t resident_warps = static_cast<int64_t>(sm_count(device)) * per_sm * wpc;
+    int64_t per_warp = tu.dispatch_units_per_warp > 0 ? tu.dispatch_units_per_warp
+                                                      : kDefaultUnitsPerWarp;
+    if (per_warp < 0 || ceil_div(units, per_warp) < resident_warps)
+        per_warp = std::max<int64_t>(1, ceil_div(units, resident_warps));
+    p.per_warp = static_cast<uint32_t>(per_warp);
+    const int64_t grid = std::max<int64_t>(1, ceil_div(ceil_div(units, per_warp), wpc));
     dispatch_bulk_kernel<<<static_cast<unsigned>(grid), wpc * 32, smem, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess)

@@ -47,6 +47,8 @@ struct Tuning {
     int combine_stages = 0;
     int combine_mode = 0;      // 0/1: bulk engine, 2: LSU engine
     int combine_smem_kb = 0;
+    int dispatch_units_per_warp = 0;
+    int combine_tokens_per_cta = 0;
 };
 Tuning &tuning();
 
