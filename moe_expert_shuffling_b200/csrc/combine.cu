@@ -127,11 +127,12 @@ constexpr uint32_t kChunk = 2048;                       // bytes of each row per
 constexpr int kConsumerWarps = kChunk / 16 / 32;        // one 16-byte vector per thread
 constexpr int kBulkThreads = 32 * (1 + kConsumerWarps);
 constexpr int kMaxBulkStages = 16;
-// Measured on B200 (dsv3 and long shapes): about 128-144 KB of row chunks in flight per
-// SM, spread over 4 CTAs, is fastest; deeper rings or more CTAs are slower.
-constexpr int kDefaultSmemBudget = 32 * 1024 + 128;
-constexpr int kDefaultCtasPerSm = 4;
-constexpr int kDefaultTokensPerCta = 16;
+// Measured on B200 (dsv3 and long shapes): a ring of 32-36 KB per CTA, 3 CTAs per SM and
+// short runs of 4 tokens per CTA (the block scheduler evens out the tail) are fastest;
+// deeper rings, more CTAs per SM and persistent CTAs are slower.
+constexpr int kDefaultSmemBudget = 36 * 1024 + 128;
+constexpr int kDefaultCtasPerSm = 3;
+constexpr int kDefaultTokensPerCta = 4;
 
 struct CombineBulkParams {
     const uint8_t *y;

@@ -21,7 +21,10 @@ namespace {
 
 constexpr uint32_t kMaxChunkBytes = 32768;
 constexpr int kMaxStages = 8;
-constexpr int kDefaultUnitsPerWarp = 8;
+// Measured on B200 (dsv3 and long shapes): short runs of 2 units per warp on a grid that
+// covers all units beat persistent warps by ~12% (the block scheduler evens out the
+// tail); 4 stages with 2 store groups in flight per warp.
+constexpr int kDefaultUnitsPerWarp = 2;
 
 struct DispatchParams {
     const uint8_t *x;
