@@ -148,6 +148,31 @@ MOE_API moe_status moe_dispatch(const void *x, moe_dtype dtype, const float *x_s
  */
 MOE_API moe_status moe_combine(const void *y, int32_t H, moe_plan_t plan, void *out, void *stream);
 
+/*
+ * moe_plan_noalloc -- the plan of moe_plan, for callers that may not allocate device
+ * memory: a process whose allocator owns every byte of the GPU, or a latency-critical
+ * loop that cannot afford an allocation's device-wide synchronisation.  (The pages
+ * describe no counterpart; this is a property of this library's interface.)
+ *
+ * Writes the same arrays, with the same values, as moe_plan into arrays the caller
+ * owns: cnt[E], expert_off[E+1], rcnt[R], rank_off[R+1], rtok_off[R+1], slot[N*k],
+ * src_tok[N*k], src_j[N*k], rtok and fanout [N*min(k,R)], err[1] (all device, 4-byte
+ * aligned).  Calls no cudaMalloc or cudaFree.  Its per-tile scratch counts live in one
+ * fixed 1 MiB array in device memory that every GPU loading the library keeps until the
+ * process exits; a call needing more than (E + R + 1) * ceil(N / 128) <= 262144 scratch
+ * words returns MOE_EINVAL.  The first call on each device does a one-time set-up (it
+ * looks up that array's device address); make that first call before any stream capture
+ * begins.  All
+ * calls share the array, so calls whose kernels could overlap on the GPU race and must
+ * be ordered (one stream, or events).  topk_w is not taken: moe_combine needs a plan
+ * from moe_plan.
+ */
+MOE_API moe_status moe_plan_noalloc(const int32_t *topk_idx, int32_t N, int32_t k, int32_t E,
+                                    int32_t R, int32_t *cnt, int32_t *expert_off, int32_t *rcnt,
+                                    int32_t *rank_off, int32_t *rtok_off, int32_t *slot,
+                                    int32_t *src_tok, int32_t *src_j, int32_t *rtok,
+                                    uint32_t *fanout, uint32_t *err, void *stream);
+
 /* moe_plan_query -- fill *view with the plan's shape and device pointers. */
 MOE_API moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *view);
 

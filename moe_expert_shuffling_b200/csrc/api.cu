@@ -77,6 +77,17 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 namespace moe {
 
+moe_status record_error(moe_status st, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
 Tuning &tuning()
 {
     static Tuning t;

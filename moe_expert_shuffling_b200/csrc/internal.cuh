@@ -56,6 +56,22 @@ int sm_count(int device);
 
 cudaError_t launch_plan(moe_plan_s *p, const int32_t *topk_idx, cudaStream_t stream);
 
+// The planner's kernels on explicit arrays (for callers that own every buffer).  The
+// scratch arrays hold E*tiles, R*tiles and tiles words, tiles = ceil(N / kPlanTile).
+struct PlanArrays {
+    const int32_t *topk_idx;
+    int32_t N, k, E, R;
+    int64_t rtok_cap;
+    int32_t *cnt, *expert_off, *rcnt, *rank_off, *rtok_off, *slot, *src_tok, *src_j, *rtok;
+    uint32_t *fanout, *err;
+    int32_t *tile_cnt, *tile_rcnt;
+    uint32_t *tile_err;
+};
+cudaError_t launch_plan_arrays(const PlanArrays &a, cudaStream_t stream);
+
+// Record a failure for moe_last_error() and return `st`.
+moe_status record_error(moe_status st, const char *fmt, ...);
+
 struct DispatchArgs {
     const uint8_t *x;      // [N, row_bytes]
     const uint8_t *xs;     // [N, srow_bytes] or null

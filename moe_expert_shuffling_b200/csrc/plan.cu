@@ -397,4 +397,41 @@ cudaError_t launch_plan(moe_plan_s *p, const int32_t *topk_idx, cudaStream_t str
     return cudaGetLastError();
 }
 
+cudaError_t launch_plan_arrays(const PlanArrays &a, cudaStream_t stream)
+{
+    static bool attrs_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= 64)
+        dev = 0;
+    if (!attrs_set[dev]) {
+        const int max_rank = static_cast<int>(rank_smem(kMaxExperts, kMaxExperts, kMaxTopk));
+        const int max_count = static_cast<int>(count_smem(kMaxExperts, kMaxExperts, kMaxTopk));
+        e = cudaFuncSetAttribute(plan_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 max_rank);
+        if (e != cudaSuccess)
+            return e;
+        e = cudaFuncSetAttribute(plan_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 max_count);
+        if (e != cudaSuccess)
+            return e;
+        attrs_set[dev] = true;
+    }
+    const int32_t N = a.N, k = a.k, E = a.E, R = a.R, epr = E / R;
+    const int32_t nt = static_cast<int32_t>(ceil_div(N, kPlanTile));
+    if (nt > 0) {
+        plan_count_kernel<<<nt, kPlanThreads, count_smem(E, R, k), stream>>>(
+            a.topk_idx, N, k, E, epr, R, nt, a.tile_cnt, a.tile_rcnt, a.tile_err);
+    }
+    plan_scan_kernel<<<E + R, kScanThreads, 0, stream>>>(a.tile_cnt, a.tile_rcnt, E, R, nt, a.cnt,
+                                                          a.rcnt, a.tile_err, a.err);
+    plan_rank_kernel<<<nt > 0 ? nt : 1, kPlanThreads, rank_smem(E, R, k), stream>>>(
+        a.topk_idx, N, k, E, epr, R, nt, a.tile_cnt, a.tile_rcnt, a.cnt, a.rcnt, a.expert_off,
+        a.rank_off, a.rtok_off, a.slot, a.src_tok, a.src_j, a.rtok, a.fanout, N * k, a.rtok_cap,
+        a.err);
+    return cudaGetLastError();
+}
+
 }  // namespace moe
