@@ -255,7 +255,7 @@ def run_ours(args):
     if disp_us >= comb_us:
         dom, dom_bytes, dom_us = "dispatch_bulk_kernel", db, disp_us
     else:
-        dom, dom_bytes, dom_us = "combine_kernel", cb, comb_us
+        dom, dom_bytes, dom_us = "combine_bulk_kernel", cb, comb_us
     achieved = dom_bytes / (dom_us * 1e-6) / 1e9
     launches_per_step = 5 + (1 if cfg.payload == "fp8" and (4 * (cfg.H // 128)) % 16 else 0)
 

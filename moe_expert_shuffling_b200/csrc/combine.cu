@@ -145,6 +145,7 @@ struct CombineBulkParams {
     uint32_t per_cta;       // tokens of each CTA: [cta * per_cta, +per_cta)
 };
 
+template <int KMAX>
 __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const CombineBulkParams p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -211,17 +212,26 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
         return;
     }
 
-    // ---------------- consumers: thread v owns bytes [16v, 16v + 16) of every chunk
+    // ---------------- consumers: thread v owns bytes [16v, 16v + 16) of every chunk.
+    // A token's valid columns (bitmask) and weights are broadcast once per token and kept
+    // in registers; each chunk then costs k shared loads, 8k fmas and one 16-byte store.
     const uint32_t v16 = static_cast<uint32_t>(threadIdx.x - 32) * 16u;
-    int32_t s_cur = -1, s_nxt = -1;
-    float w_cur = 0.f, w_nxt = 0.f;
+    int32_t s_nxt = -1;
+    float w_nxt = 0.f;
     if (n_tok > 0 && lane < k) {
-        s_cur = __ldg(p.slot + static_cast<int64_t>(b) * k + lane);
-        w_cur = __ldg(p.w + static_cast<int64_t>(b) * k + lane);
+        s_nxt = __ldg(p.slot + static_cast<int64_t>(b) * k + lane);
+        w_nxt = __ldg(p.w + static_cast<int64_t>(b) * k + lane);
     }
     int i = 0;
     for (int m = 0; m < n_tok; ++m) {
         const uint32_t t = b + static_cast<uint32_t>(m);
+        const uint32_t vmask = __ballot_sync(
+            0xffffffffu,
+            lane < k && static_cast<uint32_t>(s_nxt) < static_cast<uint32_t>(p.n_rows));
+        float wv[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+            wv[j] = __shfl_sync(0xffffffffu, w_nxt, j);
         if (m + 1 < n_tok && lane < k) {
             s_nxt = __ldg(p.slot + static_cast<int64_t>(t + 1) * k + lane);
             w_nxt = __ldg(p.w + static_cast<int64_t>(t + 1) * k + lane);
@@ -237,33 +247,35 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
             const uint32_t off = c * kChunk;
             const uint32_t len = min(kChunk, p.row_bytes - off);
             const uint8_t *stage = ring + static_cast<size_t>(st) * p.stage_bytes + v16;
+            const bool mine = v16 < len;
             float acc[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
                 acc[e] = 0.f;
-            const bool mine = v16 < len;
-            for (int j0 = 0; j0 < k; j0 += 8) {
+#pragma unroll
+            for (int j0 = 0; j0 < KMAX; j0 += 8) {
+                if (j0 >= k)
+                    break;  // warp-uniform
                 uint4 q[8];
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
                     const int j = j0 + jj;
-                    const int32_t sj = __shfl_sync(0xffffffffu, s_cur, j & 31);
-                    const bool use = j < k && mine &&
-                                     static_cast<uint32_t>(sj) < static_cast<uint32_t>(p.n_rows);
-                    q[jj] = use ? lds_v4(stage + j * kChunk) : make_uint4(0u, 0u, 0u, 0u);
+                    q[jj] = (mine && ((vmask >> j) & 1u)) ? lds_v4(stage + j * kChunk)
+                                                          : make_uint4(0u, 0u, 0u, 0u);
+                }
+                if (j0 + 8 >= k) {
+                    // every row of this stage is in registers: release it to the producer
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&empty[st]);
                 }
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
                     const int j = j0 + jj;
-                    const int32_t sj = __shfl_sync(0xffffffffu, s_cur, j & 31);
-                    const float wj = __shfl_sync(0xffffffffu, w_cur, j & 31);
-                    if (j < k && static_cast<uint32_t>(sj) < static_cast<uint32_t>(p.n_rows))
-                        fma_bf16x8(acc, wj, q[jj]);
+                    if ((vmask >> j) & 1u)
+                        fma_bf16x8(acc, wv[j], q[jj]);
                 }
             }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&empty[st]);
             if (mine)
                 st_stream_v4(p.out + static_cast<int64_t>(t) * p.row_bytes + off + v16,
                              pack_bf16x8(acc));
@@ -273,8 +285,6 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
                 atomicOr(p.err, MOE_ERR_TIMEOUT);
             return;
         }
-        s_cur = s_nxt;
-        w_cur = w_nxt;
     }
 }
 
@@ -347,13 +357,13 @@ cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t s
     p.stages = static_cast<uint32_t>(S);
     p.bar_bytes = static_cast<uint32_t>(round_up(2 * S * 8, 128));
     const size_t smem = smem_for(S);
-    e = cudaFuncSetAttribute(combine_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kern = a.k <= 8 ? combine_bulk_kernel<8> : combine_bulk_kernel<32>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess)
         return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_bulk_kernel, kBulkThreads,
-                                                      smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBulkThreads, smem);
     if (e != cudaSuccess)
         return e;
     if (per_sm < 1)
@@ -369,7 +379,7 @@ cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t s
         per_cta = std::max<int64_t>(1, ceil_div(a.N, resident));
     p.per_cta = static_cast<uint32_t>(per_cta);
     const int64_t grid = std::max<int64_t>(1, ceil_div(a.N, per_cta));
-    combine_bulk_kernel<<<static_cast<unsigned>(grid), kBulkThreads, smem, stream>>>(p);
+    kern<<<static_cast<unsigned>(grid), kBulkThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
