@@ -112,7 +112,8 @@ MOE_API moe_status moe_plan_create(int32_t max_tokens, int32_t k, int32_t E, int
  *   rcnt[r] = #{t : some expert of t is on r}, rtok_off = exclusive scan of rcnt,
  *   rtok/fanout = the tokens of rank r in ascending order with the mask of their
  *   columns on r -- one move per (token, rank) pair.
- * Deterministic (no result depends on thread timing).  Enqueues three kernels.
+ * Deterministic (no result depends on thread timing).  Enqueues one cooperative kernel
+ * (three kernels where its grid cannot be co-resident).
  */
 MOE_API moe_status moe_plan(const int32_t *topk_idx, const float *topk_w, int32_t N, int32_t k,
                     int32_t E, int32_t R, void *stream, moe_plan_t *plan);
@@ -205,7 +206,8 @@ typedef enum {
     MOE_TUNE_COMBINE_ENGINE = 7,         /* 0 or 1: bulk-copy engine, 2: LSU engine */
     MOE_TUNE_COMBINE_SMEM_KB = 8,        /* bulk combine: shared-memory budget per CTA (KB) */
     MOE_TUNE_DISPATCH_UNITS_PER_WARP = 9, /* (token, chunk) units per dispatch warp */
-    MOE_TUNE_COMBINE_TOKENS_PER_CTA = 10 /* tokens per bulk-combine CTA */
+    MOE_TUNE_COMBINE_TOKENS_PER_CTA = 10, /* tokens per bulk-combine CTA */
+    MOE_TUNE_PLAN_ENGINE = 11            /* 0 or 1: one cooperative plan kernel, 2: three kernels */
 } moe_knob;
 
 MOE_API moe_status moe_tune(moe_knob knob, int32_t value);

@@ -34,7 +34,7 @@ KNOBS = {
     "dispatch_stages": 0, "dispatch_lag": 1, "dispatch_ctas_per_sm": 2,
     "dispatch_warps_per_cta": 3, "combine_vec_per_lane": 4, "combine_ctas_per_sm": 5,
     "combine_stages": 6, "combine_engine": 7, "combine_smem_kb": 8,
-    "dispatch_units_per_warp": 9, "combine_tokens_per_cta": 10,
+    "dispatch_units_per_warp": 9, "combine_tokens_per_cta": 10, "plan_engine": 11,
 }
 
 _i32 = ctypes.c_int32

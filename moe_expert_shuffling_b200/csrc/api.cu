@@ -134,6 +134,7 @@ moe_status moe_tune(moe_knob knob, int32_t value)
     case MOE_TUNE_COMBINE_SMEM_KB: t.combine_smem_kb = value; break;
     case MOE_TUNE_DISPATCH_UNITS_PER_WARP: t.dispatch_units_per_warp = value; break;
     case MOE_TUNE_COMBINE_TOKENS_PER_CTA: t.combine_tokens_per_cta = value; break;
+    case MOE_TUNE_PLAN_ENGINE: t.plan_engine = value; break;
     default: return fail(MOE_EINVAL, "unknown tuning knob %d", static_cast<int>(knob));
     }
     return ok();
@@ -181,6 +182,7 @@ moe_status moe_plan_create(int32_t max_tokens, int32_t k, int32_t E, int32_t R, 
         {reinterpret_cast<void **>(&p->rtok), sizeof(int32_t) * (p->rtok_cap > 0 ? p->rtok_cap : 1)},
         {reinterpret_cast<void **>(&p->fanout), sizeof(uint32_t) * (p->rtok_cap > 0 ? p->rtok_cap : 1)},
         {reinterpret_cast<void **>(&p->err), sizeof(uint32_t)},
+        {reinterpret_cast<void **>(&p->sync), 2 * sizeof(uint32_t)},
         {reinterpret_cast<void **>(&p->tile_cnt), sizeof(int32_t) * E * nt},
         {reinterpret_cast<void **>(&p->tile_rcnt), sizeof(int32_t) * R * nt},
         {reinterpret_cast<void **>(&p->tile_err), sizeof(uint32_t) * nt},

@@ -21,6 +21,7 @@ struct moe_plan_s {
             *rtok_off = nullptr, *slot = nullptr, *src_tok = nullptr, *src_j = nullptr,
             *rtok = nullptr;
     uint32_t *fanout = nullptr, *err = nullptr;
+    uint32_t *sync = nullptr;  // [2] grid-barrier words of the fused plan kernel (zero at rest)
     // scratch: per-tile counts [E][nt] and [R][nt] (then their column prefixes), tile flags
     int32_t *tile_cnt = nullptr, *tile_rcnt = nullptr;
     uint32_t *tile_err = nullptr;
@@ -49,6 +50,7 @@ struct Tuning {
     int combine_smem_kb = 0;
     int dispatch_units_per_warp = 0;
     int combine_tokens_per_cta = 0;
+    int plan_engine = 0;       // 0/1: one cooperative kernel when it fits, 2: three kernels
 };
 Tuning &tuning();
 

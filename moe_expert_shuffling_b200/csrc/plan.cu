@@ -4,18 +4,23 @@
 // transfers; DySHARP blog, section 5: the destination maps a token's logical index to a
 // local address -- slot[t, j] is that map.
 //
-// Three kernels, all deterministic (no result depends on thread timing):
-//   plan_count  one CTA per tile of 128 tokens: per-tile expert counts and per-tile
-//               counts of (token, rank) moves -> scratch [E][tiles], [R][tiles]
-//   plan_scan   one CTA per expert row and per rank row: exclusive scan over tiles,
-//               row totals -> cnt[E], rcnt[R]; CTA 0 also gathers the tile flags
-//   plan_rank   one CTA per tile: segment starts, then every entry's stable rank inside
-//               its segment as a popcount over a per-expert bitmask of the tile's tokens
-//               (bit t set when token t selects the expert), so no step is sequential.
+// Three phases, all deterministic (no result depends on thread timing):
+//   count  per tile of 128 tokens: expert counts and counts of (token, rank) moves
+//          -> scratch [E][tiles], [R][tiles], plus the tile's error flags
+//   scan   per expert row and per rank row: exclusive scan over tiles, row totals
+//          -> cnt[E], rcnt[R]; the tile flags are gathered into the error word
+//   rank   per tile: segment starts, then every entry's stable rank inside its segment
+//          as a popcount over a per-expert bitmask of the tile's tokens (bit t set when
+//          token t selects the expert), so no step is sequential.
+// By default the phases run in one cooperative kernel (plan_fused_kernel) whose CTAs
+// meet at two grid barriers; a barrier gives up after 1 s and reports MOE_ERR_TIMEOUT.
+// When the grid cannot be co-resident the phases run as three kernels instead.
 //
 // Inside a tile a warp looks at several tokens at once: lane = (token, column) with the
 // columns of one token in a segment of W = next power of two >= k lanes, so a token's
 // k ids are compared with width-W shuffles.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.cuh"
 
@@ -25,6 +30,18 @@ namespace {
 constexpr int kPlanThreads = kPlanWarps * 32;
 constexpr int kScanThreads = 256;
 constexpr uint32_t kFull = 0xffffffffu;  // all lanes of a warp
+
+// Kernel parameters: shape, routing, outputs and scratch.
+struct PlanK {
+    const int32_t *topk_idx;
+    int32_t N, k, E, R, epr, nt, n_rows;
+    int64_t rtok_cap;
+    int32_t *tile_cnt, *tile_rcnt;
+    uint32_t *tile_err;
+    int32_t *cnt, *expert_off, *rcnt, *rank_off, *rtok_off, *slot, *src_tok, *src_j, *rtok;
+    uint32_t *fanout, *err;
+    uint32_t *sync;  // [2] grid-barrier arrivals and departures (fused kernel), zero at rest
+};
 
 // Classification of one entry, shared by the count and rank kernels so both see the
 // same entries.  Entry (t, j) is valid when its id is in [0, E) and no earlier column of
@@ -134,7 +151,7 @@ __device__ void scan_into(const int32_t *src, int n, int32_t *dst, int32_t *warp
     int32_t carry = 0;
     for (int base = 0; base < n; base += blockDim.x) {
         const int i = base + threadIdx.x;
-        const int32_t v = i < n ? src[i] : 0;
+        const int32_t v = i < n ? __ldcg(src + i) : 0;
         int32_t tot;
         const int32_t ex = block_exclusive_scan(v, &tot, warp_sums);
         if (i < n)
@@ -145,44 +162,83 @@ __device__ void scan_into(const int32_t *src, int n, int32_t *dst, int32_t *warp
         dst[n] = carry;
 }
 
-__global__ void __launch_bounds__(kPlanThreads)
-    plan_count_kernel(const int32_t *__restrict__ topk_idx, int32_t N, int32_t k, int32_t E,
-                      int32_t epr, int32_t R, int32_t nt, int32_t *__restrict__ tile_cnt,
-                      int32_t *__restrict__ tile_rcnt, uint32_t *__restrict__ tile_err)
+// Shared-memory layout of every plan kernel (words).
+struct PlanSmem {
+    int32_t *eoff;      // [E+1] segment starts of the experts
+    int32_t *roff;      // [R+1] starts of the ranks' dedup lists
+    int32_t *ebase;     // [E]   tile base per expert; the histogram while counting
+    int32_t *rbase;     // [R]   tile base per rank; the rank histogram while counting
+    int32_t *rank_of;   // [E]   rank of each expert
+    uint32_t *emask;    // [E][4] tokens of the tile on each expert
+    uint32_t *rmask;    // [R][4] tokens of the tile on each rank
+    int32_t *ids;       // [kPlanTile * k] the tile's routing ids
+    int32_t *vid;       // [kPlanTile * k] valid id or -1
+    uint32_t *lead;     // [kPlanTile * k] leader masks
+};
+
+__host__ __device__ constexpr size_t plan_smem_words(int E, int R, int k)
 {
-    extern __shared__ int32_t smem[];
-    int32_t *hist = smem;            // [E]
-    int32_t *rhist = hist + E;       // [R]
-    int32_t *rank_of = rhist + R;    // [E]
-    int32_t *ids = rank_of + E;      // [kPlanTile * k]
-    __shared__ uint32_t s_err;
+    return static_cast<size_t>(E + 1) + (R + 1) + E + R + E + 4 * E + 4 * R +
+           3 * static_cast<size_t>(kPlanTile) * k;
+}
 
-    const int tile = blockIdx.x;
+__device__ PlanSmem carve(int32_t *w, int E, int R, int k)
+{
+    PlanSmem m;
+    m.eoff = w;
+    m.roff = m.eoff + E + 1;
+    m.ebase = m.roff + R + 1;
+    m.rbase = m.ebase + E;
+    m.rank_of = m.rbase + R;
+    m.emask = reinterpret_cast<uint32_t *>(m.rank_of + E);
+    m.rmask = m.emask + 4 * E;
+    m.ids = reinterpret_cast<int32_t *>(m.rmask + 4 * R);
+    m.vid = m.ids + kPlanTile * k;
+    m.lead = reinterpret_cast<uint32_t *>(m.vid + kPlanTile * k);
+    return m;
+}
+
+__device__ __forceinline__ int tile_tokens(const PlanK &p, int tile)
+{
+    const int64_t left = static_cast<int64_t>(p.N) - static_cast<int64_t>(tile) * kPlanTile;
+    return static_cast<int>(left <= 0 ? 0 : (left < kPlanTile ? left : kPlanTile));
+}
+
+__device__ void init_rank_of(const PlanK &p, const PlanSmem &m)
+{
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
+        m.rank_of[e] = e / p.epr;
+}
+
+__device__ void load_ids(const PlanK &p, const PlanSmem &m, int tile, int ntok)
+{
+    const int32_t *src = p.topk_idx + static_cast<int64_t>(tile) * kPlanTile * p.k;
+    for (int i = threadIdx.x; i < ntok * p.k; i += blockDim.x)
+        m.ids[i] = __ldg(src + i);
+}
+
+// Count phase for one tile.  All threads must call; rank_of must be ready.
+__device__ void count_tile(const PlanK &p, const PlanSmem &m, int tile, uint32_t *s_err)
+{
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t t0 = static_cast<int64_t>(tile) * kPlanTile;
-    const int64_t left = N - t0;
-    const int ntok = static_cast<int>(left < kPlanTile ? left : kPlanTile);
-
-    for (int i = threadIdx.x; i < E + R; i += blockDim.x)
-        smem[i] = 0;
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-        rank_of[e] = e / epr;
-    const int32_t *src = topk_idx + t0 * k;
-    for (int i = threadIdx.x; i < ntok * k; i += blockDim.x)
-        ids[i] = __ldg(src + i);
+    const int ntok = tile_tokens(p, tile);
+    int32_t *hist = m.ebase, *rhist = m.rbase;
+    for (int i = threadIdx.x; i < p.E + p.R; i += blockDim.x)
+        hist[i] = 0;  // ebase and rbase are contiguous
+    load_ids(p, m, tile, ntok);
     if (threadIdx.x == 0)
-        s_err = 0;
+        *s_err = 0;
     __syncthreads();
 
-    const LaneMap lm = lane_map(k);
+    const LaneMap lm = lane_map(p.k);
     const int j = lane & ((1 << lm.wbits) - 1);
     const int sub = lane >> lm.wbits;
     uint32_t flags = 0;
     for (int st = 0; st < lm.steps; ++st) {
         const int tw = st * lm.per_step + sub;           // token within the warp's 16
         const int tl = warp * kPlanTokensPerWarp + tw;
-        const bool present = tw < kPlanTokensPerWarp && tl < ntok && j < k;
-        const Entry c = classify(ids, rank_of, tl, j, present, k, E, 1 << lm.wbits);
+        const bool present = tw < kPlanTokensPerWarp && tl < ntok && j < p.k;
+        const Entry c = classify(m.ids, m.rank_of, tl, j, present, p.k, p.E, 1 << lm.wbits);
         flags |= c.flags;
         if (c.e >= 0)
             atomicAdd(&hist[c.e], 1);
@@ -190,112 +246,52 @@ __global__ void __launch_bounds__(kPlanThreads)
             atomicAdd(&rhist[c.r], 1);
     }
     if (flags)
-        atomicOr(&s_err, flags);
+        atomicOr(s_err, flags);
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-        tile_cnt[static_cast<int64_t>(e) * nt + tile] = hist[e];
-    for (int r = threadIdx.x; r < R; r += blockDim.x)
-        tile_rcnt[static_cast<int64_t>(r) * nt + tile] = rhist[r];
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
+        p.tile_cnt[static_cast<int64_t>(e) * p.nt + tile] = hist[e];
+    for (int r = threadIdx.x; r < p.R; r += blockDim.x)
+        p.tile_rcnt[static_cast<int64_t>(r) * p.nt + tile] = rhist[r];
     if (threadIdx.x == 0)
-        tile_err[tile] = s_err;
-}
-
-__global__ void __launch_bounds__(kScanThreads)
-    plan_scan_kernel(int32_t *__restrict__ tile_cnt, int32_t *__restrict__ tile_rcnt, int32_t E,
-                     int32_t R, int32_t nt, int32_t *__restrict__ cnt, int32_t *__restrict__ rcnt,
-                     const uint32_t *__restrict__ tile_err, uint32_t *__restrict__ err)
-{
-    __shared__ int32_t warp_sums[kScanThreads / 32];
-    __shared__ uint32_t s_err;
-    const int row = blockIdx.x;
-    int32_t *p = row < E ? tile_cnt + static_cast<int64_t>(row) * nt
-                         : tile_rcnt + static_cast<int64_t>(row - E) * nt;
-    int32_t carry = 0;
-    for (int base = 0; base < nt; base += blockDim.x) {
-        const int i = base + threadIdx.x;
-        const int32_t v = i < nt ? p[i] : 0;
-        int32_t tot;
-        const int32_t ex = block_exclusive_scan(v, &tot, warp_sums);
-        if (i < nt)
-            p[i] = carry + ex;
-        carry += tot;
-    }
-    if (threadIdx.x == 0) {
-        if (row < E)
-            cnt[row] = carry;
-        else
-            rcnt[row - E] = carry;
-    }
-    if (row == 0) {  // block-uniform
-        if (threadIdx.x == 0)
-            s_err = 0;
-        __syncthreads();
-        uint32_t f = 0;
-        for (int i = threadIdx.x; i < nt; i += blockDim.x)
-            f |= tile_err[i];
-        if (f)
-            atomicOr(&s_err, f);
-        __syncthreads();
-        if (threadIdx.x == 0)
-            *err = s_err;
-    }
-}
-
-__global__ void __launch_bounds__(kPlanThreads)
-    plan_rank_kernel(const int32_t *__restrict__ topk_idx, int32_t N, int32_t k, int32_t E,
-                     int32_t epr, int32_t R, int32_t nt, const int32_t *__restrict__ tile_cnt,
-                     const int32_t *__restrict__ tile_rcnt, const int32_t *__restrict__ cnt,
-                     const int32_t *__restrict__ rcnt, int32_t *__restrict__ expert_off,
-                     int32_t *__restrict__ rank_off, int32_t *__restrict__ rtok_off,
-                     int32_t *__restrict__ slot, int32_t *__restrict__ src_tok,
-                     int32_t *__restrict__ src_j, int32_t *__restrict__ rtok,
-                     uint32_t *__restrict__ fanout, int32_t n_rows, int64_t rtok_cap,
-                     uint32_t *__restrict__ err)
-{
-    extern __shared__ int32_t smem[];
-    int32_t *ebase = smem;                        // [E+1] segment starts, then tile bases
-    int32_t *rbase = ebase + E + 1;               // [R+1]
-    int32_t *rank_of = rbase + R + 1;             // [E]
-    uint32_t *emask = reinterpret_cast<uint32_t *>(rank_of + E);  // [E][4] tokens per expert
-    uint32_t *rmask = emask + 4 * E;              // [R][4] tokens per rank
-    int32_t *ids = reinterpret_cast<int32_t *>(rmask + 4 * R);    // [kPlanTile * k]
-    int32_t *vid = ids + kPlanTile * k;           // [kPlanTile * k] valid id or -1
-    uint32_t *lead = reinterpret_cast<uint32_t *>(vid + kPlanTile * k);  // [kPlanTile * k]
-    __shared__ int32_t warp_sums[kPlanThreads / 32];
-
-    const int tile = blockIdx.x;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t t0 = static_cast<int64_t>(tile) * kPlanTile;
-    const int64_t left = N - t0;
-    const int ntok = static_cast<int>(left <= 0 ? 0 : (left < kPlanTile ? left : kPlanTile));
-
-    // Segment starts: exclusive scans of the expert and rank totals.
-    scan_into(cnt, E, ebase, warp_sums);
-    scan_into(rcnt, R, rbase, warp_sums);
-    for (int i = threadIdx.x; i < 4 * (E + R); i += blockDim.x)
-        emask[i] = 0u;  // emask and rmask are contiguous
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-        rank_of[e] = e / epr;
-    const int32_t *src = topk_idx + t0 * k;
-    for (int i = threadIdx.x; i < ntok * k; i += blockDim.x)
-        ids[i] = __ldg(src + i);
+        p.tile_err[tile] = *s_err;
     __syncthreads();
-    if (tile == 0) {
-        for (int i = threadIdx.x; i <= E; i += blockDim.x)
-            expert_off[i] = ebase[i];
-        for (int i = threadIdx.x; i <= R; i += blockDim.x) {
-            rtok_off[i] = rbase[i];
-            rank_off[i] = ebase[i * epr];
+}
+
+// Segment starts from the totals; block 0 publishes them.  All threads must call.
+__device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_sums)
+{
+    scan_into(p.cnt, p.E, m.eoff, warp_sums);
+    scan_into(p.rcnt, p.R, m.roff, warp_sums);
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        for (int i = threadIdx.x; i <= p.E; i += blockDim.x)
+            p.expert_off[i] = m.eoff[i];
+        for (int i = threadIdx.x; i <= p.R; i += blockDim.x) {
+            p.rtok_off[i] = m.roff[i];
+            p.rank_off[i] = m.eoff[i * p.epr];
         }
     }
+}
+
+// Rank phase for one tile.  All threads must call; rank_prepare must have run.  With
+// ids_ready the tile's ids are already in shared memory.
+__device__ void rank_tile(const PlanK &p, const PlanSmem &m, int tile, bool ids_ready)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int ntok = tile_tokens(p, tile);
     if (ntok == 0)
-        return;  // block-uniform; no barrier follows for this block
-    __syncthreads();
+        return;  // block-uniform
+    const int k = p.k;
+    for (int i = threadIdx.x; i < 4 * (p.E + p.R); i += blockDim.x)
+        m.emask[i] = 0u;  // emask and rmask are contiguous
+    if (!ids_ready)
+        load_ids(p, m, tile, ntok);
     // This tile's first receive row per expert and first dedup entry per rank.
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-        ebase[e] += tile_cnt[static_cast<int64_t>(e) * nt + tile];
-    for (int r = threadIdx.x; r < R; r += blockDim.x)
-        rbase[r] += tile_rcnt[static_cast<int64_t>(r) * nt + tile];
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
+        m.ebase[e] = m.eoff[e] + __ldcg(p.tile_cnt + static_cast<int64_t>(e) * p.nt + tile);
+    for (int r = threadIdx.x; r < p.R; r += blockDim.x)
+        m.rbase[r] = m.roff[r] + __ldcg(p.tile_rcnt + static_cast<int64_t>(r) * p.nt + tile);
+    __syncthreads();
 
     // Pass A: classify, and mark each token in its expert's and rank's tile mask.
     const LaneMap lm = lane_map(k);
@@ -305,20 +301,21 @@ __global__ void __launch_bounds__(kPlanThreads)
         const int tw = st * lm.per_step + sub;
         const int tl = warp * kPlanTokensPerWarp + tw;
         const bool present = tw < kPlanTokensPerWarp && tl < ntok && j < k;
-        const Entry c = classify(ids, rank_of, tl, j, present, k, E, 1 << lm.wbits);
+        const Entry c = classify(m.ids, m.rank_of, tl, j, present, k, p.E, 1 << lm.wbits);
         if (present) {
-            vid[tl * k + j] = c.e;
-            lead[tl * k + j] = c.lead;
+            m.vid[tl * k + j] = c.e;
+            m.lead[tl * k + j] = c.lead;
             const uint32_t bit = 1u << (tl & 31);
             if (c.e >= 0)
-                atomicOr(&emask[4 * c.e + (tl >> 5)], bit);
+                atomicOr(&m.emask[4 * c.e + (tl >> 5)], bit);
             if (c.lead)
-                atomicOr(&rmask[4 * c.r + (tl >> 5)], bit);
+                atomicOr(&m.rmask[4 * c.r + (tl >> 5)], bit);
         }
     }
     __syncthreads();
 
     // Pass B: stable rank = tile base + earlier tokens of the tile on the same expert.
+    const int64_t t0 = static_cast<int64_t>(tile) * kPlanTile;
     uint32_t flags = 0;
     for (int st = 0; st < lm.steps; ++st) {
         const int tw = st * lm.per_step + sub;
@@ -327,111 +324,333 @@ __global__ void __launch_bounds__(kPlanThreads)
             continue;
         const int64_t t = t0 + tl;
         const int i = tl * k + j;
-        const int32_t e = vid[i];
+        const int32_t e = m.vid[i];
         int32_t s = -1;
         if (e >= 0) {
-            s = ebase[e] + bits_below(&emask[4 * e], tl);
-            if (static_cast<uint32_t>(s) < static_cast<uint32_t>(n_rows)) {
-                src_tok[s] = static_cast<int32_t>(t);
-                src_j[s] = j;
+            s = m.ebase[e] + bits_below(&m.emask[4 * e], tl);
+            if (static_cast<uint32_t>(s) < static_cast<uint32_t>(p.n_rows)) {
+                p.src_tok[s] = static_cast<int32_t>(t);
+                p.src_j[s] = j;
             } else {
                 flags |= MOE_ERR_BOUNDS;
                 s = -1;
             }
-            const uint32_t m = lead[i];
-            if (m) {
-                const int32_t r = rank_of[e];
-                const int32_t pos = rbase[r] + bits_below(&rmask[4 * r], tl);
-                if (pos >= 0 && pos < rtok_cap) {
-                    rtok[pos] = static_cast<int32_t>(t);
-                    fanout[pos] = m;
+            const uint32_t msk = m.lead[i];
+            if (msk) {
+                const int32_t r = m.rank_of[e];
+                const int32_t pos = m.rbase[r] + bits_below(&m.rmask[4 * r], tl);
+                if (pos >= 0 && pos < p.rtok_cap) {
+                    p.rtok[pos] = static_cast<int32_t>(t);
+                    p.fanout[pos] = msk;
                 } else {
                     flags |= MOE_ERR_BOUNDS;
                 }
             }
         }
-        slot[t * k + j] = s;
+        p.slot[t * k + j] = s;
     }
     if (flags)
-        atomicOr(err, flags);
+        atomicOr(p.err, flags);
+    __syncthreads();
 }
 
-size_t count_smem(int E, int R, int k) { return sizeof(int32_t) * (2 * E + R + kPlanTile * k); }
-size_t rank_smem(int E, int R, int k)
+// ------------------------------------------------------------- three-kernel path
+__global__ void __launch_bounds__(kPlanThreads) plan_count_kernel(const PlanK p)
 {
-    return sizeof(int32_t) * ((E + 1) + (R + 1) + E + 4 * (E + R) + 3 * kPlanTile * k);
+    extern __shared__ int32_t smem[];
+    __shared__ uint32_t s_err;
+    const PlanSmem m = carve(smem, p.E, p.R, p.k);
+    init_rank_of(p, m);
+    count_tile(p, m, blockIdx.x, &s_err);
+}
+
+__global__ void __launch_bounds__(kScanThreads) plan_scan_kernel(const PlanK p)
+{
+    __shared__ int32_t warp_sums[kScanThreads / 32];
+    __shared__ uint32_t s_err;
+    const int row = blockIdx.x;
+    int32_t *rp = row < p.E ? p.tile_cnt + static_cast<int64_t>(row) * p.nt
+                            : p.tile_rcnt + static_cast<int64_t>(row - p.E) * p.nt;
+    int32_t carry = 0;
+    for (int base = 0; base < p.nt; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        const int32_t v = i < p.nt ? rp[i] : 0;
+        int32_t tot;
+        const int32_t ex = block_exclusive_scan(v, &tot, warp_sums);
+        if (i < p.nt)
+            rp[i] = carry + ex;
+        carry += tot;
+    }
+    if (threadIdx.x == 0) {
+        if (row < p.E)
+            p.cnt[row] = carry;
+        else
+            p.rcnt[row - p.E] = carry;
+    }
+    if (row == 0) {  // block-uniform
+        if (threadIdx.x == 0)
+            s_err = 0;
+        __syncthreads();
+        uint32_t f = 0;
+        for (int i = threadIdx.x; i < p.nt; i += blockDim.x)
+            f |= p.tile_err[i];
+        if (f)
+            atomicOr(&s_err, f);
+        __syncthreads();
+        if (threadIdx.x == 0)
+            *p.err = s_err;
+    }
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_rank_kernel(const PlanK p)
+{
+    extern __shared__ int32_t smem[];
+    __shared__ int32_t warp_sums[kPlanThreads / 32];
+    const PlanSmem m = carve(smem, p.E, p.R, p.k);
+    init_rank_of(p, m);
+    rank_prepare(p, m, warp_sums);
+    rank_tile(p, m, blockIdx.x, false);
+}
+
+// ----------------------------------------------------------- fused (cooperative)
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *a)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+    return v;
+}
+
+// Grid barrier for a co-resident grid: arrivals count up to `target`.  Gives up after
+// kWaitLimitNs, sets MOE_ERR_TIMEOUT and returns false.  All threads must call.
+__device__ bool grid_barrier(const PlanK &p, uint32_t target, int *s_ok)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(&p.sync[0], 1u);
+        bool ok = true;
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t it = 0; ld_acquire_gpu(&p.sync[0]) < target; ++it) {
+            if ((it & 15u) == 15u && (global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30))) {
+                atomicOr(p.err, MOE_ERR_TIMEOUT);
+                ok = false;
+                break;
+            }
+            __nanosleep(64);
+        }
+        __threadfence();
+        *s_ok = ok;
+    }
+    __syncthreads();
+    return *s_ok != 0;
+}
+
+// The last CTA to leave resets the barrier words for the next launch.
+__device__ void grid_depart(const PlanK &p)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&p.sync[1], 1u) == gridDim.x - 1u) {
+            p.sync[0] = 0u;
+            p.sync[1] = 0u;
+            __threadfence();
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
+{
+    extern __shared__ int32_t smem[];
+    __shared__ uint32_t s_err;
+    __shared__ int32_t warp_sums[kPlanThreads / 32];
+    __shared__ int s_ok;
+    const PlanSmem m = carve(smem, p.E, p.R, p.k);
+    const uint32_t G = gridDim.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    init_rank_of(p, m);
+    for (int tile = blockIdx.x; tile < p.nt; tile += G)
+        count_tile(p, m, tile, &s_err);
+    if (!grid_barrier(p, G, &s_ok)) {
+        grid_depart(p);
+        return;
+    }
+
+    // Scan phase: one warp per expert row / rank row; lane l owns a contiguous run of
+    // ceil(tiles / 32) tiles.
+    const int per_lane = (p.nt + 31) / 32;
+    for (int row = blockIdx.x * kPlanWarps + warp; row < p.E + p.R;
+         row += static_cast<int>(G) * kPlanWarps) {
+        int32_t *rp = row < p.E ? p.tile_cnt + static_cast<int64_t>(row) * p.nt
+                                : p.tile_rcnt + static_cast<int64_t>(row - p.E) * p.nt;
+        const int a = lane * per_lane;
+        const int b = min(a + per_lane, p.nt);
+        int32_t sum = 0;
+        for (int i = a; i < b; ++i)
+            sum += __ldcg(rp + i);
+        int32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o)
+                incl += y;
+        }
+        int32_t run = incl - sum;
+        for (int i = a; i < b; ++i) {
+            const int32_t v = __ldcg(rp + i);
+            rp[i] = run;
+            run += v;
+        }
+        if (lane == 31) {
+            if (row < p.E)
+                p.cnt[row] = incl;
+            else
+                p.rcnt[row - p.E] = incl;
+        }
+    }
+    if (blockIdx.x == 0 && warp == 0) {
+        uint32_t f = 0;
+        for (int i = lane; i < p.nt; i += 32)
+            f |= __ldcg(p.tile_err + i);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            f |= __shfl_xor_sync(kFull, f, o);
+        if (lane == 0)
+            *p.err = f;
+    }
+    if (!grid_barrier(p, 2u * G, &s_ok)) {
+        grid_depart(p);
+        return;
+    }
+
+    rank_prepare(p, m, warp_sums);
+    const bool one_tile = static_cast<int>(G) >= p.nt;  // ids of the tile are still in smem
+    for (int tile = blockIdx.x; tile < p.nt; tile += G)
+        rank_tile(p, m, tile, one_tile);
+    grid_depart(p);
+}
+
+PlanK make_params(const int32_t *topk_idx, int32_t N, int32_t k, int32_t E, int32_t R,
+                  int64_t rtok_cap)
+{
+    PlanK p{};
+    p.topk_idx = topk_idx;
+    p.N = N;
+    p.k = k;
+    p.E = E;
+    p.R = R;
+    p.epr = E / R;
+    p.nt = static_cast<int32_t>(ceil_div(N, kPlanTile));
+    p.n_rows = N * k;
+    p.rtok_cap = rtok_cap;
+    return p;
+}
+
+bool ensure_attrs(int dev)
+{
+    static bool done[64] = {false};
+    if (dev < 0 || dev >= 64)
+        dev = 0;
+    if (done[dev])
+        return true;
+    const int bytes = static_cast<int>(sizeof(int32_t) *
+                                       plan_smem_words(kMaxExperts, kMaxExperts, kMaxTopk));
+    if (cudaFuncSetAttribute(plan_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(plan_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(plan_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess)
+        return false;
+    done[dev] = true;
+    return true;
+}
+
+cudaError_t launch_three(const PlanK &p, cudaStream_t stream)
+{
+    const size_t smem = sizeof(int32_t) * plan_smem_words(p.E, p.R, p.k);
+    if (p.nt > 0)
+        plan_count_kernel<<<p.nt, kPlanThreads, smem, stream>>>(p);
+    plan_scan_kernel<<<p.E + p.R, kScanThreads, 0, stream>>>(p);
+    plan_rank_kernel<<<p.nt > 0 ? p.nt : 1, kPlanThreads, smem, stream>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_plan(moe_plan_s *p, const int32_t *topk_idx, cudaStream_t stream)
+cudaError_t launch_plan(moe_plan_s *pl, const int32_t *topk_idx, cudaStream_t stream)
 {
-    static bool attrs_set[64] = {false};
-    const int dev = p->device >= 0 && p->device < 64 ? p->device : 0;
-    if (!attrs_set[dev]) {
-        const int max_rank = static_cast<int>(rank_smem(kMaxExperts, kMaxExperts, kMaxTopk));
-        const int max_count = static_cast<int>(count_smem(kMaxExperts, kMaxExperts, kMaxTopk));
-        cudaError_t e1 = cudaFuncSetAttribute(plan_rank_kernel,
-                                              cudaFuncAttributeMaxDynamicSharedMemorySize, max_rank);
-        if (e1 != cudaSuccess)
-            return e1;
-        e1 = cudaFuncSetAttribute(plan_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  max_count);
-        if (e1 != cudaSuccess)
-            return e1;
-        attrs_set[dev] = true;
+    if (!ensure_attrs(pl->device))
+        return cudaGetLastError() != cudaSuccess ? cudaGetLastError() : cudaErrorUnknown;
+    PlanK p = make_params(topk_idx, pl->N, pl->k, pl->E, pl->R, pl->rtok_cap);
+    p.tile_cnt = pl->tile_cnt;
+    p.tile_rcnt = pl->tile_rcnt;
+    p.tile_err = pl->tile_err;
+    p.cnt = pl->cnt;
+    p.expert_off = pl->expert_off;
+    p.rcnt = pl->rcnt;
+    p.rank_off = pl->rank_off;
+    p.rtok_off = pl->rtok_off;
+    p.slot = pl->slot;
+    p.src_tok = pl->src_tok;
+    p.src_j = pl->src_j;
+    p.rtok = pl->rtok;
+    p.fanout = pl->fanout;
+    p.err = pl->err;
+    p.sync = pl->sync;
+
+    if (tuning().plan_engine != 2) {
+        // One cooperative launch when the grid fits on the device at once.
+        static int coop[64] = {0};
+        const int dev = pl->device >= 0 && pl->device < 64 ? pl->device : 0;
+        if (coop[dev] == 0) {
+            int v = 0;
+            cudaDeviceGetAttribute(&v, cudaDevAttrCooperativeLaunch, pl->device);
+            coop[dev] = v ? 1 : -1;
+        }
+        const size_t smem = sizeof(int32_t) * plan_smem_words(p.E, p.R, p.k);
+        int per_sm = 0;
+        if (coop[dev] > 0 &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_fused_kernel,
+                                                          kPlanThreads, smem) == cudaSuccess &&
+            per_sm > 0) {
+            const int64_t fit = static_cast<int64_t>(sm_count(pl->device)) * per_sm;
+            const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(p.nt, fit)));
+            void *args[] = {&p};
+            return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(plan_fused_kernel),
+                                               dim3(grid), dim3(kPlanThreads), args, smem, stream);
+        }
+        (void)cudaGetLastError();
     }
-    const int32_t N = p->N, k = p->k, E = p->E, R = p->R, epr = p->epr;
-    const int32_t nt = static_cast<int32_t>(ceil_div(N, kPlanTile));
-    const int32_t n_rows = N * k;
-    if (nt > 0) {
-        plan_count_kernel<<<nt, kPlanThreads, count_smem(E, R, k), stream>>>(
-            topk_idx, N, k, E, epr, R, nt, p->tile_cnt, p->tile_rcnt, p->tile_err);
-    }
-    plan_scan_kernel<<<E + R, kScanThreads, 0, stream>>>(p->tile_cnt, p->tile_rcnt, E, R, nt,
-                                                          p->cnt, p->rcnt, p->tile_err, p->err);
-    plan_rank_kernel<<<nt > 0 ? nt : 1, kPlanThreads, rank_smem(E, R, k), stream>>>(
-        topk_idx, N, k, E, epr, R, nt, p->tile_cnt, p->tile_rcnt, p->cnt, p->rcnt, p->expert_off,
-        p->rank_off, p->rtok_off, p->slot, p->src_tok, p->src_j, p->rtok, p->fanout, n_rows,
-        p->rtok_cap, p->err);
-    return cudaGetLastError();
+    return launch_three(p, stream);
 }
 
 cudaError_t launch_plan_arrays(const PlanArrays &a, cudaStream_t stream)
 {
-    static bool attrs_set[64] = {false};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
-    if (dev < 0 || dev >= 64)
-        dev = 0;
-    if (!attrs_set[dev]) {
-        const int max_rank = static_cast<int>(rank_smem(kMaxExperts, kMaxExperts, kMaxTopk));
-        const int max_count = static_cast<int>(count_smem(kMaxExperts, kMaxExperts, kMaxTopk));
-        e = cudaFuncSetAttribute(plan_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 max_rank);
-        if (e != cudaSuccess)
-            return e;
-        e = cudaFuncSetAttribute(plan_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 max_count);
-        if (e != cudaSuccess)
-            return e;
-        attrs_set[dev] = true;
-    }
-    const int32_t N = a.N, k = a.k, E = a.E, R = a.R, epr = E / R;
-    const int32_t nt = static_cast<int32_t>(ceil_div(N, kPlanTile));
-    if (nt > 0) {
-        plan_count_kernel<<<nt, kPlanThreads, count_smem(E, R, k), stream>>>(
-            a.topk_idx, N, k, E, epr, R, nt, a.tile_cnt, a.tile_rcnt, a.tile_err);
-    }
-    plan_scan_kernel<<<E + R, kScanThreads, 0, stream>>>(a.tile_cnt, a.tile_rcnt, E, R, nt, a.cnt,
-                                                          a.rcnt, a.tile_err, a.err);
-    plan_rank_kernel<<<nt > 0 ? nt : 1, kPlanThreads, rank_smem(E, R, k), stream>>>(
-        a.topk_idx, N, k, E, epr, R, nt, a.tile_cnt, a.tile_rcnt, a.cnt, a.rcnt, a.expert_off,
-        a.rank_off, a.rtok_off, a.slot, a.src_tok, a.src_j, a.rtok, a.fanout, N * k, a.rtok_cap,
-        a.err);
-    return cudaGetLastError();
+    if (!ensure_attrs(dev))
+        return cudaGetLastError() != cudaSuccess ? cudaGetLastError() : cudaErrorUnknown;
+    PlanK p = make_params(a.topk_idx, a.N, a.k, a.E, a.R, a.rtok_cap);
+    p.tile_cnt = a.tile_cnt;
+    p.tile_rcnt = a.tile_rcnt;
+    p.tile_err = a.tile_err;
+    p.cnt = a.cnt;
+    p.expert_off = a.expert_off;
+    p.rcnt = a.rcnt;
+    p.rank_off = a.rank_off;
+    p.rtok_off = a.rtok_off;
+    p.slot = a.slot;
+    p.src_tok = a.src_tok;
+    p.src_j = a.src_j;
+    p.rtok = a.rtok;
+    p.fanout = a.fanout;
+    p.err = a.err;
+    p.sync = nullptr;
+    return launch_three(p, stream);
 }
 
 }  // namespace moe

@@ -199,6 +199,8 @@ def test_invalid_routing_is_flagged_and_contained():
     {"combine_engine": 2, "combine_vec_per_lane": 2},
     {"combine_engine": 2, "combine_vec_per_lane": 4},
     {"combine_stages": 2},
+    {"plan_engine": 2},
+    {"dispatch_units_per_warp": 10000, "combine_tokens_per_cta": 10000},
     {"combine_smem_kb": 64, "combine_ctas_per_sm": 2},
 ])
 def test_launch_configuration_does_not_change_results(knobs):
