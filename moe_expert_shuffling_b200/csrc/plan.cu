@@ -477,36 +477,43 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
         return;
     }
 
-    // Scan phase: one warp per expert row / rank row; lane l owns a contiguous run of
-    // ceil(tiles / 32) tiles.
-    const int per_lane = (p.nt + 31) / 32;
+    // Scan phase: one warp per expert row / rank row, in coalesced rounds of 32 tiles;
+    // each group of up to 16 rounds is loaded before any of it is scanned.
+    constexpr int kRounds = 16;
     for (int row = blockIdx.x * kPlanWarps + warp; row < p.E + p.R;
          row += static_cast<int>(G) * kPlanWarps) {
         int32_t *rp = row < p.E ? p.tile_cnt + static_cast<int64_t>(row) * p.nt
                                 : p.tile_rcnt + static_cast<int64_t>(row - p.E) * p.nt;
-        const int a = lane * per_lane;
-        const int b = min(a + per_lane, p.nt);
-        int32_t sum = 0;
-        for (int i = a; i < b; ++i)
-            sum += __ldcg(rp + i);
-        int32_t incl = sum;
+        int32_t carry = 0;
+        for (int g0 = 0; g0 < p.nt; g0 += 32 * kRounds) {
+            int32_t v[kRounds];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int32_t y = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o)
-                incl += y;
+            for (int q = 0; q < kRounds; ++q) {
+                const int i = g0 + q * 32 + lane;
+                v[q] = i < p.nt ? __ldcg(rp + i) : 0;
+            }
+#pragma unroll
+            for (int q = 0; q < kRounds; ++q) {
+                if (g0 + q * 32 < p.nt) {  // warp-uniform
+                    const int i = g0 + q * 32 + lane;
+                    int32_t incl = v[q];
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int32_t y = __shfl_up_sync(kFull, incl, o);
+                        if (lane >= o)
+                            incl += y;
+                    }
+                    if (i < p.nt)
+                        rp[i] = carry + incl - v[q];
+                    carry += __shfl_sync(kFull, incl, 31);
+                }
+            }
         }
-        int32_t run = incl - sum;
-        for (int i = a; i < b; ++i) {
-            const int32_t v = __ldcg(rp + i);
-            rp[i] = run;
-            run += v;
-        }
-        if (lane == 31) {
+        if (lane == 0) {
             if (row < p.E)
-                p.cnt[row] = incl;
+                p.cnt[row] = carry;
             else
-                p.rcnt[row - p.E] = incl;
+                p.rcnt[row - p.E] = carry;
         }
     }
     if (blockIdx.x == 0 && warp == 0) {
