@@ -151,7 +151,7 @@ __device__ void scan_into(const int32_t *src, int n, int32_t *dst, int32_t *warp
     int32_t carry = 0;
     for (int base = 0; base < n; base += blockDim.x) {
         const int i = base + threadIdx.x;
-        const int32_t v = i < n ? __ldcg(src + i) : 0;
+        const int32_t v = i < n ? src[i] : 0;
         int32_t tot;
         const int32_t ex = block_exclusive_scan(v, &tot, warp_sums);
         if (i < n)
@@ -258,10 +258,14 @@ __device__ void count_tile(const PlanK &p, const PlanSmem &m, int tile, uint32_t
 }
 
 // Segment starts from the totals; block 0 publishes them.  All threads must call.
+// Both totals arrays are staged in shared memory with their loads in flight together.
 __device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_sums)
 {
-    scan_into(p.cnt, p.E, m.eoff, warp_sums);
-    scan_into(p.rcnt, p.R, m.roff, warp_sums);
+    for (int i = threadIdx.x; i < p.E + p.R; i += blockDim.x)
+        m.ebase[i] = i < p.E ? __ldcg(p.cnt + i) : __ldcg(p.rcnt + (i - p.E));  // ebase|rbase
+    __syncthreads();
+    scan_into(m.ebase, p.E, m.eoff, warp_sums);
+    scan_into(m.rbase, p.R, m.roff, warp_sums);
     __syncthreads();
     if (blockIdx.x == 0) {
         for (int i = threadIdx.x; i <= p.E; i += blockDim.x)
