@@ -146,6 +146,20 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------ ours
+def dist_init(backend: str, rank: int, world: int, local: int | None = None):
+    """Join the process group (no-op for world == 1).  NCCL for GPU ranks, gloo on CPU."""
+    if world == 1:
+        return
+    import datetime
+
+    import torch.distributed as dist
+    kw = {}
+    if backend == "nccl":
+        kw["device_id"] = torch.device("cuda", local)
+    dist.init_process_group(backend, rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120), **kw)
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -153,22 +167,29 @@ def dist_setup(args):
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    dist_init("nccl", rank, world, local)
     return world, rank, local
 
 
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank runs an independent replica on its own seeded batch."""
+    return seed + rank
+
+
 def max_over_ranks(v: float, world: int) -> float:
+    """Slowest rank's value (device timing is per rank; the job ends with the last one)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(bytes_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job GB/s: every rank's bytes over the slowest rank's time."""
+    return bytes_per_rank_step * steps * world / (max_ms * 1e-3) / 1e9
 
 
 def barrier(world: int):
@@ -186,7 +207,7 @@ def run_ours(args):
     cfg = CONFIGS[args.config]
     if args.tokens > 0:
         cfg = cfg.with_tokens(args.tokens)
-    seed = args.seed + rank
+    seed = rank_seed(args.seed, rank)
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(device=dev)
 
@@ -245,8 +266,7 @@ def run_ours(args):
     ms_per_step = elapsed_ms / args.steps
 
     db, cb = dispatch_bytes(cfg), combine_bytes(cfg)
-    job_bytes = (db + cb) * args.steps * world
-    value = job_bytes / (elapsed_ms * 1e-3) / 1e9
+    value = job_throughput(db + cb, args.steps, world, elapsed_ms)
     tokens_per_s = cfg.N * args.steps * world / (elapsed_ms * 1e-3)
     peak, peak_kind = measured_hbm_peak()
     disp_us = 1e3 * statistics.mean(t_disp)
@@ -294,7 +314,7 @@ def run_ours(args):
         b.record(stream)
         b.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(b), world)
-        e2e = {"value": round((db + cb) * args.e2e_steps * world / (e_ms * 1e-3) / 1e9, 3),
+        e2e = {"value": round(job_throughput(db + cb, args.e2e_steps, world, e_ms), 3),
                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(e_ms / args.e2e_steps, 3), "steps": args.e2e_steps}
 
