@@ -75,14 +75,20 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_traffic(kernel: str, units: int):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+def kernel_traffic(kernel: str, cfg: Config):
+    """DRAM bytes per launch from the committed ncu summary: the captured bytes per token
+    scaled to this launch's tokens, if the capture was of this row shape and the kernel's
+    sources are unchanged since; else None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[kernel]
     except Exception:
         return None
+    shape = rec.get("shape", {})
+    if (shape.get("H"), shape.get("k"), shape.get("payload")) != (cfg.H, cfg.k, cfg.payload):
+        return None
+    units = cfg.N
     h = hashlib.sha256()
     for rel in rec["sources"]:
         with open(os.path.join(ROOT, rel), "rb") as f:
@@ -106,9 +112,9 @@ class ClockSampler:
 
     def start(self):
         try:
-            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{self.gpu}.csv")
-            self.fh = open(self.path, "w")
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix=f"clocks_gpu{self.gpu}_", suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", str(self.period)],
@@ -127,7 +133,10 @@ class ClockSampler:
         self.fh.close()
         rows = []
         with open(self.path) as f:
-            for line in f:
+            lines = f.readlines()
+        os.unlink(self.path)
+        if True:
+            for line in lines:
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) < 9:
                     continue
@@ -349,7 +358,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": kernel_traffic(dom, cfg.N)},
+                     "traffic": kernel_traffic(dom, cfg)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "e2e": e2e,
