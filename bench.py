@@ -285,7 +285,10 @@ def run_ours(args):
     else:
         dom, dom_bytes, dom_us = "combine_bulk_kernel", cb, comb_us
     achieved = dom_bytes / (dom_us * 1e-6) / 1e9
-    launches_per_step = 5 + (1 if cfg.payload == "fp8" and (4 * (cfg.H // 128)) % 16 else 0)
+    # plan (1 cooperative kernel or 3) + dispatch (+ the scale kernel for fp8 scale rows
+    # that are not a multiple of 16 bytes) + combine
+    launches_per_step = (plan.plan_kernels + 1 + 1 +
+                         (1 if cfg.payload == "fp8" and (4 * (cfg.H // 128)) % 16 else 0))
 
     # end to end: pinned host inputs -> device, step, result -> pinned host
     e2e = None

@@ -79,6 +79,7 @@ typedef struct {
     uint32_t *fanout;              /* [sum rcnt] bit j: column j of that token is on rank r */
     uint32_t *err;                 /* [1]    MOE_ERR_* bits of the last moe_plan call */
     const float *topk_w;           /* the weights given to the last moe_plan call */
+    int32_t plan_kernels;          /* kernels the last moe_plan call enqueued (1 or 3) */
 } moe_plan_view;
 
 /*

@@ -46,7 +46,7 @@ class _PlanView(ctypes.Structure):
         ("N", _i32), ("k", _i32), ("E", _i32), ("R", _i32), ("experts_per_rank", _i32),
         ("capacity_tokens", _i32), ("cnt", _vp), ("expert_off", _vp), ("rcnt", _vp),
         ("rank_off", _vp), ("rtok_off", _vp), ("slot", _vp), ("src_tok", _vp), ("src_j", _vp),
-        ("rtok", _vp), ("fanout", _vp), ("err", _vp), ("topk_w", _vp),
+        ("rtok", _vp), ("fanout", _vp), ("err", _vp), ("topk_w", _vp), ("plan_kernels", _i32),
     ]
 
 
@@ -169,6 +169,11 @@ class Plan:
     @property
     def capacity(self) -> int:
         return self._view().capacity_tokens
+
+    @property
+    def plan_kernels(self) -> int:
+        """Kernels the last moe_plan call enqueued (1 cooperative kernel, or 3)."""
+        return self._view().plan_kernels
 
     def arrays(self) -> dict[str, torch.Tensor]:
         """Zero-copy int32 views of the plan's device arrays (fanout/err as bit patterns)."""

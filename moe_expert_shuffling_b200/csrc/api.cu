@@ -359,6 +359,7 @@ moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *v)
     v->fanout = p->fanout;
     v->err = p->err;
     v->topk_w = p->topk_w;
+    v->plan_kernels = p->plan_kernels;
     return ok();
 }
 

@@ -26,6 +26,7 @@ struct moe_plan_s {
     int32_t *tile_cnt = nullptr, *tile_rcnt = nullptr;
     uint32_t *tile_err = nullptr;
     const float *topk_w = nullptr;
+    int32_t plan_kernels = 0;  // kernels the last launch_plan enqueued
 };
 
 namespace moe {

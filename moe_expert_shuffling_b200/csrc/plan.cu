@@ -629,11 +629,13 @@ cudaError_t launch_plan(moe_plan_s *pl, const int32_t *topk_idx, cudaStream_t st
             const int64_t fit = static_cast<int64_t>(sm_count(pl->device)) * per_sm;
             const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(p.nt, fit)));
             void *args[] = {&p};
+            pl->plan_kernels = 1;
             return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(plan_fused_kernel),
                                                dim3(grid), dim3(kPlanThreads), args, smem, stream);
         }
         (void)cudaGetLastError();
     }
+    pl->plan_kernels = 3;
     return launch_three(p, stream);
 }
 
