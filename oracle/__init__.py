@@ -11,13 +11,12 @@ from __future__ import annotations
 
 import ctypes
 import os
+from contextlib import contextmanager
 from dataclasses import dataclass
 
 import numpy as np
 
 from .build import build as _build
-
-_LIB = None
 
 _i32p = ctypes.POINTER(ctypes.c_int32)
 _u32p = ctypes.POINTER(ctypes.c_uint32)
@@ -29,27 +28,47 @@ _i64 = ctypes.c_int64
 _i32 = ctypes.c_int32
 
 
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    lib.oracle_plan.restype = ctypes.c_int
+    lib.oracle_plan.argtypes = [_i32p, _i64, _i32, _i32, _i32, _i32p, _i32p, _i32p, _i32p,
+                                _i32p, _i32p, _i32p, _i32p, _i32p, _u32p, _i64]
+    lib.oracle_validate.restype = ctypes.c_int
+    lib.oracle_validate.argtypes = [_i32p, _i64, _i32, _i32]
+    lib.oracle_dedup_count.restype = ctypes.c_int64
+    lib.oracle_dedup_count.argtypes = [_i32p, _i64, _i32, _i32, _i32]
+    lib.oracle_dispatch.restype = None
+    lib.oracle_dispatch.argtypes = [_u8p, _u8p, _i32p, _i64, _i32, _i64, _i64, _u8p, _u8p]
+    lib.oracle_combine.restype = None
+    lib.oracle_combine.argtypes = [_u16p, _i32p, _f32p, _i64, _i32, _i64, _u16p]
+    lib.oracle_combine_f64.restype = None
+    lib.oracle_combine_f64.argtypes = [_u16p, _i32p, _f32p, _i64, _i32, _i64, _f64p]
+    lib.oracle_f32_to_bf16.restype = None
+    lib.oracle_f32_to_bf16.argtypes = [_f32p, _i64, _u16p]
+    return lib
+
+
+_DEFAULT = None
+
+
 def _lib():
-    global _LIB
-    if _LIB is None:
-        lib = ctypes.CDLL(_build())
-        lib.oracle_plan.restype = ctypes.c_int
-        lib.oracle_plan.argtypes = [_i32p, _i64, _i32, _i32, _i32, _i32p, _i32p, _i32p, _i32p,
-                                    _i32p, _i32p, _i32p, _i32p, _i32p, _u32p, _i64]
-        lib.oracle_validate.restype = ctypes.c_int
-        lib.oracle_validate.argtypes = [_i32p, _i64, _i32, _i32]
-        lib.oracle_dedup_count.restype = ctypes.c_int64
-        lib.oracle_dedup_count.argtypes = [_i32p, _i64, _i32, _i32, _i32]
-        lib.oracle_dispatch.restype = None
-        lib.oracle_dispatch.argtypes = [_u8p, _u8p, _i32p, _i64, _i32, _i64, _i64, _u8p, _u8p]
-        lib.oracle_combine.restype = None
-        lib.oracle_combine.argtypes = [_u16p, _i32p, _f32p, _i64, _i32, _i64, _u16p]
-        lib.oracle_combine_f64.restype = None
-        lib.oracle_combine_f64.argtypes = [_u16p, _i32p, _f32p, _i64, _i32, _i64, _f64p]
-        lib.oracle_f32_to_bf16.restype = None
-        lib.oracle_f32_to_bf16.argtypes = [_f32p, _i64, _u16p]
-        _LIB = lib
-    return _LIB
+    global _DEFAULT
+    if _DEFAULT is None:
+        _DEFAULT = _bind(_build())
+    return _DEFAULT
+
+
+@contextmanager
+def using_library(path: str):
+    """Run the oracle functions on another build of oracle.c for the duration of the block
+    (the pin tests use this to check that planted mistakes are caught)."""
+    global _DEFAULT
+    prev = _lib()
+    _DEFAULT = _bind(path)
+    try:
+        yield
+    finally:
+        _DEFAULT = prev
 
 
 def _p(a: np.ndarray, ptype):

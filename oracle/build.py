@@ -20,5 +20,15 @@ def build(force: bool = False) -> str:
     return LIB
 
 
+def build_variant(source: str, lib_path: str) -> str:
+    """Compile another version of oracle.c (given as text) to `lib_path`."""
+    src = lib_path + ".c"
+    with open(src, "w") as f:
+        f.write(source)
+    subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-fPIC",
+                    "-shared", src, "-o", lib_path, "-lm"], check=True)
+    return lib_path
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv))

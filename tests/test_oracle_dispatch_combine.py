@@ -79,6 +79,31 @@ def exact_combine(y_bits, slot, w, tokens, cols):
     return out
 
 
+def fma_chain_at_scale(y_bits, slot, w):
+    """Exact fp32 fma chain (then bf16 RNE) for every output, vectorised.
+
+    Each product of an fp32 weight and a bf16 value is exact in float64.  The float64 sum
+    with the fp32 accumulator is exact too unless their exponents are far apart; a two-sum
+    finds those rare sums, which are then redone with exact rationals, so every step equals
+    a single rounding of the exact value to fp32."""
+    from fractions import Fraction
+    yv = bits_to_f32(y_bits).astype(np.float64)
+    N, k = slot.shape
+    acc = np.zeros((N, yv.shape[1]), np.float32)
+    for j in range(k):
+        prod = w[:, j:j + 1].astype(np.float64) * yv[slot[:, j]]
+        a64 = acc.astype(np.float64)
+        s = prod + a64
+        bb = s - prod
+        err = (prod - (s - bb)) + (a64 - bb)
+        nxt = s.astype(np.float32)
+        for t, c in zip(*np.nonzero(err != 0)):
+            exact = Fraction(float(prod[t, c])) + Fraction(float(a64[t, c]))
+            nxt[t, c] = np.float32(float(f32_round(exact)))
+        acc = nxt
+    return bf16_bits_of(acc)
+
+
 # --------------------------------------------------------------------------- dispatch
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_dispatch_brute_force_tiny(seed):
@@ -146,6 +171,16 @@ def test_combine_exact_rational_tiny():
     got = bits_to_f32(out)
     for (t, c), v in ref.items():
         assert Fraction(float(got[t, c])) == v, (t, c)
+
+
+@pytest.mark.parametrize("name,N", [("dsv3", 256), ("long", 128)])
+def test_combine_matches_exact_fma_chain_at_scale(name, N):
+    """Every output of a few hundred tokens equals the exact fp32-fma-chain result."""
+    cfg = CONFIGS[name].with_tokens(N)
+    idx, w = make_routing(cfg, 4)
+    p = oracle.plan(idx, cfg.E, cfg.R)
+    yb = bits16(make_payload_y(cfg.replace(y="normal"), 4))
+    assert np.array_equal(oracle.combine(yb, p.slot, w), fma_chain_at_scale(yb, p.slot, w))
 
 
 def test_combine_golden_ties_and_identity():
