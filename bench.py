@@ -245,7 +245,8 @@ def run_ours(args):
             ms.moe_dispatch(x, plan, recv=recv, stream=stream)
         if ev is not None:
             ev[2].record(stream)
-        ms.moe_combine(recv if identity else y, plan, out=out, stream=stream)
+        ms.moe_combine(recv if identity else y, plan, out=out, stream=stream,
+                       ranked=args.combine == "ranked")
         if ev is not None:
             ev[3].record(stream)
 
@@ -345,7 +346,9 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if cfg.payload == "bf16" else "fp8e4m3", "accum_dtype": "f32",
         "data": "synthetic (seeded routing and N(0,1) payload; no traces or weights exist)",
-        "config": {"workload": workload_name(cfg), "model": f"{cfg.name}-shaped MoE layer shuffle",
+        "config": {"workload": workload_name(cfg) + ("" if args.combine == "chain" else
+                                                      ", combine grouped by rank"),
+                   "model": f"{cfg.name}-shaped MoE layer shuffle",
                    "global_batch": cfg.N * world, "seq_len": cfg.N, "parallelism": f"replicas{world}",
                    "ep_ranks_logical": cfg.R,
                    "l2": "no flush: every input (x, y) and output is larger than the 126 MB L2"},
@@ -470,6 +473,8 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (small cases for profiling)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--combine", default="chain", choices=["chain", "ranked"],
+                    help="combine order: one fma chain per token, or grouped by rank first")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -175,6 +175,20 @@ MOE_API moe_status moe_plan_noalloc(const int32_t *topk_idx, int32_t N, int32_t 
                                     int32_t *src_tok, int32_t *src_j, int32_t *rtok,
                                     uint32_t *fanout, uint32_t *err, void *stream);
 
+/*
+ * moe_combine_ranked -- the combine with the reduction grouped by rank, the combine-side
+ * counterpart of the per-rank dedup (DySHARP blog, section 2: the partial results that
+ * several destinations produce for one token could be summed before travelling back;
+ * section 5: a reducing load returns one result).  For each rank holding experts of token
+ * t, in ascending rank order, a partial is formed as the fp32 fma chain over t's columns
+ * on that rank (ascending column, from +0); the partials are added in fp32 in ascending
+ * rank order (from +0) and the sum is rounded to bf16 (nearest even).  Arguments as for
+ * moe_combine.  The result differs from moe_combine only by rounding order (within the
+ * same error bound).  Uses the bulk-copy engine.
+ */
+MOE_API moe_status moe_combine_ranked(const void *y, int32_t H, moe_plan_t plan, void *out,
+                                      void *stream);
+
 /* moe_plan_query -- fill *view with the plan's shape and device pointers. */
 MOE_API moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *view);
 

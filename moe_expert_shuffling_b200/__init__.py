@@ -65,6 +65,8 @@ def _load():
     lib.moe_dispatch.argtypes = [_vp, ctypes.c_int, _vp, _i32, _vp, _vp, _vp, _vp]
     lib.moe_combine.restype = st
     lib.moe_combine.argtypes = [_vp, _i32, _vp, _vp, _vp]
+    lib.moe_combine_ranked.restype = st
+    lib.moe_combine_ranked.argtypes = [_vp, _i32, _vp, _vp, _vp]
     lib.moe_plan_query.restype = st
     lib.moe_plan_query.argtypes = [_vp, ctypes.POINTER(_PlanView)]
     lib.moe_plan_check.restype = st
@@ -274,8 +276,10 @@ def moe_dispatch(x: torch.Tensor, plan: Plan, recv: torch.Tensor | None = None,
     return (recv, recv_scale) if fp8 else recv
 
 
-def moe_combine(y: torch.Tensor, plan: Plan, out: torch.Tensor | None = None, stream=None):
-    """out[t] = bf16(sum_j w[t,j] * y[slot[t,j]]) with an fp32 fma chain in column order."""
+def moe_combine(y: torch.Tensor, plan: Plan, out: torch.Tensor | None = None, stream=None,
+                ranked: bool = False):
+    """out[t] = bf16(sum_j w[t,j] * y[slot[t,j]]) with an fp32 fma chain in column order;
+    with ranked=True the sum is grouped by rank first (moe_combine_ranked)."""
     _need_cuda(y, "y", (torch.bfloat16,), 2)
     N, k, _, _ = plan.shape
     rows, H = y.shape
@@ -286,6 +290,6 @@ def moe_combine(y: torch.Tensor, plan: Plan, out: torch.Tensor | None = None, st
     _need_cuda(out, "out", (torch.bfloat16,), 2)
     if tuple(out.shape) != (N, H):
         raise ValueError(f"out must have shape {(N, H)}")
-    _check(_lib.moe_combine(_vp(y.data_ptr()), H, plan._h, _vp(out.data_ptr()),
-                            _vp(_stream_ptr(stream))))
+    fn = _lib.moe_combine_ranked if ranked else _lib.moe_combine
+    _check(fn(_vp(y.data_ptr()), H, plan._h, _vp(out.data_ptr()), _vp(_stream_ptr(stream))))
     return out

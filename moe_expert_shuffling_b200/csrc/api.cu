@@ -306,7 +306,8 @@ moe_status moe_dispatch(const void *x, moe_dtype dtype, const float *x_scale, in
     return ok();
 }
 
-moe_status moe_combine(const void *y, int32_t H, moe_plan_t plan, void *out, void *stream)
+static moe_status combine_impl(const void *y, int32_t H, moe_plan_t plan, void *out, void *stream,
+                               bool ranked)
 {
     if (!plan)
         return fail(MOE_EINVAL, "plan must not be NULL");
@@ -330,10 +331,23 @@ moe_status moe_combine(const void *y, int32_t H, moe_plan_t plan, void *out, voi
     a.k = p->k;
     a.n_rows = p->N * p->k;
     a.H = H;
+    a.rank_off = p->rank_off;
+    a.R = p->R;
+    a.ranked = ranked;
     cudaError_t e = moe::launch_combine(a, p->device, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return cuda_fail(e, "combine kernel");
     return ok();
+}
+
+moe_status moe_combine(const void *y, int32_t H, moe_plan_t plan, void *out, void *stream)
+{
+    return combine_impl(y, H, plan, out, stream, false);
+}
+
+moe_status moe_combine_ranked(const void *y, int32_t H, moe_plan_t plan, void *out, void *stream)
+{
+    return combine_impl(y, H, plan, out, stream, true);
 }
 
 moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *v)

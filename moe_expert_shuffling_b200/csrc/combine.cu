@@ -123,9 +123,14 @@ __global__ void __launch_bounds__(kCombineThreads) combine_lsu_kernel(const Comb
 
 
 // ------------------------------------------------------------------ bulk engine
-constexpr uint32_t kChunk = 2048;                       // bytes of each row per unit
-constexpr int kConsumerWarps = kChunk / 16 / 32;        // one 16-byte vector per thread
-constexpr int kBulkThreads = 32 * (1 + kConsumerWarps);
+// A unit covers CW * 512 bytes of each of the token's k rows: one 16-byte vector per
+// consumer thread, CW consumer warps.  Wider k gets narrower chunks so that a stage
+// (k x chunk) stays at 16 KB: CW = 4 for k <= 8, 2 for k <= 16, 1 for k <= 32.
+template <int CW>
+struct Shape {
+    static constexpr uint32_t kChunk = 512u * CW;
+    static constexpr int kThreads = 32 * (1 + CW);
+};
 constexpr int kMaxBulkStages = 16;
 // Measured on B200 (dsv3 and long shapes): a ring of 32-36 KB per CTA, 3 CTAs per SM and
 // short runs of 4 tokens per CTA (the block scheduler evens out the tail) are fastest;
@@ -143,11 +148,20 @@ struct CombineBulkParams {
     int32_t N, k, n_rows;
     uint32_t row_bytes, nchunks, stages, stage_bytes, bar_bytes;
     uint32_t per_cta;       // tokens of each CTA: [cta * per_cta, +per_cta)
+    const int32_t *rank_off;  // [R+1] first receive row of each rank (rank-grouped order)
+    int32_t R;
+    uint32_t ring_bytes;    // bytes of the stage ring (the rank tables follow it)
 };
 
-template <int KMAX>
-__global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const CombineBulkParams p)
+// RANKED: the rank-grouped order -- per rank (ascending) an fp32 fma chain over the
+// token's columns on that rank (ascending), and the partials added in ascending rank
+// order; otherwise one fma chain over the columns in order.
+template <int KMAX, int CW, bool RANKED>
+__global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
+    combine_bulk_kernel(const CombineBulkParams p)
 {
+    constexpr uint32_t kChunk_ = Shape<CW>::kChunk;
+    constexpr int32_t kNoRank = 0x7fffffff;
     extern __shared__ __align__(128) uint8_t smem[];
     const int S = static_cast<int>(p.stages);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
@@ -155,11 +169,20 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
     uint8_t *ring = smem + p.bar_bytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int k = p.k;
+    // rank-grouped order: rank offsets, then per consumer warp the token's columns sorted
+    // by (rank, column) with their weights and ranks
+    int32_t *roff_s = reinterpret_cast<int32_t *>(ring + p.ring_bytes);
+    int32_t *ord_s = roff_s + (RANKED ? p.R + 1 : 0) + (warp > 0 ? (warp - 1) * 96 : 0);
+    float *wo_s = reinterpret_cast<float *>(ord_s + 32);
+    int32_t *ro_s = ord_s + 64;
+    if (RANKED)
+        for (int i = threadIdx.x; i <= p.R; i += blockDim.x)
+            roff_s[i] = __ldg(p.rank_off + i);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
+            mbar_init(&empty[s], CW);
         }
         mbar_init_fence();
     }
@@ -190,13 +213,13 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
                     ok = false;
                     break;
                 }
-                const uint32_t off = c * kChunk;
-                const uint32_t len = min(kChunk, p.row_bytes - off);
+                const uint32_t off = c * kChunk_;
+                const uint32_t len = min(kChunk_, p.row_bytes - off);
                 if (lane == 0)
                     mbar_arrive_expect_tx(&full[st], nv * len);
                 __syncwarp();
                 if (valid)
-                    bulk_load(ring + static_cast<size_t>(st) * p.stage_bytes + lane * kChunk,
+                    bulk_load(ring + static_cast<size_t>(st) * p.stage_bytes + lane * kChunk_,
                               p.y + static_cast<int64_t>(s_cur) * p.row_bytes + off, len,
                               &full[st]);
             }
@@ -228,10 +251,39 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
         const uint32_t vmask = __ballot_sync(
             0xffffffffu,
             lane < k && static_cast<uint32_t>(s_nxt) < static_cast<uint32_t>(p.n_rows));
-        float wv[KMAX];
+        float wv[RANKED ? 1 : KMAX];
+        if (!RANKED) {
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j)
-            wv[j] = __shfl_sync(0xffffffffu, w_nxt, j);
+            for (int j = 0; j < (RANKED ? 1 : KMAX); ++j)
+                wv[j] = __shfl_sync(0xffffffffu, w_nxt, j);
+        } else {
+            // rank of each column from the plan's rank offsets, then its position in the
+            // (rank, column) order
+            int32_t rj = kNoRank;
+            if ((vmask >> lane) & 1u) {
+                int lo = 0, hi = p.R;  // roff_s[lo] <= slot < roff_s[hi]
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (roff_s[mid] <= s_nxt)
+                        lo = mid;
+                    else
+                        hi = mid;
+                }
+                rj = lo;
+            }
+            int pos = 0;
+            for (int q = 0; q < k; ++q) {
+                const int32_t rq = __shfl_sync(0xffffffffu, rj, q);
+                pos += (rq < rj || (rq == rj && q < lane)) ? 1 : 0;
+            }
+            __syncwarp();
+            if (lane < k) {
+                ord_s[pos] = lane;
+                wo_s[pos] = w_nxt;
+                ro_s[pos] = rj;
+            }
+            __syncwarp();
+        }
         if (m + 1 < n_tok && lane < k) {
             s_nxt = __ldg(p.slot + static_cast<int64_t>(t + 1) * k + lane);
             w_nxt = __ldg(p.w + static_cast<int64_t>(t + 1) * k + lane);
@@ -244,14 +296,60 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
                 ok = false;
                 break;
             }
-            const uint32_t off = c * kChunk;
-            const uint32_t len = min(kChunk, p.row_bytes - off);
+            const uint32_t off = c * kChunk_;
+            const uint32_t len = min(kChunk_, p.row_bytes - off);
             const uint8_t *stage = ring + static_cast<size_t>(st) * p.stage_bytes + v16;
             const bool mine = v16 < len;
             float acc[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
                 acc[e] = 0.f;
+            if (RANKED) {
+                float part[8];
+                int32_t prev = -1;  // rank of the open partial
+#pragma unroll
+                for (int p0 = 0; p0 < KMAX; p0 += 8) {
+                    if (p0 >= k)
+                        break;  // warp-uniform
+                    uint4 q[8];
+#pragma unroll
+                    for (int pp = 0; pp < 8; ++pp) {
+                        const int pq = p0 + pp;
+                        const bool use = pq < k && ro_s[pq] != kNoRank;
+                        q[pp] = (mine && use) ? lds_v4(stage + ord_s[pq] * kChunk_)
+                                              : make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    if (p0 + 8 >= k) {
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(&empty[st]);
+                    }
+#pragma unroll
+                    for (int pp = 0; pp < 8; ++pp) {
+                        const int pq = p0 + pp;
+                        const int32_t rr = pq < k ? ro_s[pq] : kNoRank;
+                        if (rr == kNoRank)
+                            continue;
+                        if (rr != prev) {
+                            if (prev >= 0) {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    acc[e] = __fadd_rn(acc[e], part[e]);
+                            }
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                part[e] = 0.f;
+                            prev = rr;
+                        }
+                        fma_bf16x8(part, wo_s[pq], q[pp]);
+                    }
+                }
+                if (prev >= 0) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        acc[e] = __fadd_rn(acc[e], part[e]);
+                }
+            } else {
 #pragma unroll
             for (int j0 = 0; j0 < KMAX; j0 += 8) {
                 if (j0 >= k)
@@ -260,7 +358,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
                     const int j = j0 + jj;
-                    q[jj] = (mine && ((vmask >> j) & 1u)) ? lds_v4(stage + j * kChunk)
+                    q[jj] = (mine && ((vmask >> j) & 1u)) ? lds_v4(stage + j * kChunk_)
                                                           : make_uint4(0u, 0u, 0u, 0u);
                 }
                 if (j0 + 8 >= k) {
@@ -273,8 +371,9 @@ __global__ void __launch_bounds__(kBulkThreads, 1) combine_bulk_kernel(const Com
                 for (int jj = 0; jj < 8; ++jj) {
                     const int j = j0 + jj;
                     if ((vmask >> j) & 1u)
-                        fma_bf16x8(acc, wv[j], q[jj]);
+                        fma_bf16x8(acc, wv[RANKED ? 0 : j], q[jj]);
                 }
+            }
             }
             if (mine)
                 st_stream_v4(p.out + static_cast<int64_t>(t) * p.row_bytes + off + v16,
@@ -320,8 +419,11 @@ cudaError_t launch_kb(const CombineParams &p, int vpl, int device, int ctas, cud
 
 }  // namespace
 
-cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t stream)
+template <int KMAX, int CW, bool RANKED>
+cudaError_t launch_bulk_shape(const CombineArgs &a, int device, cudaStream_t stream)
 {
+    constexpr uint32_t chunk = Shape<CW>::kChunk;
+    constexpr int threads = Shape<CW>::kThreads;
     const Tuning &tu = tuning();
     CombineBulkParams p;
     p.y = reinterpret_cast<const uint8_t *>(a.y);
@@ -333,8 +435,8 @@ cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t s
     p.k = a.k;
     p.n_rows = a.n_rows;
     p.row_bytes = static_cast<uint32_t>(a.H) * 2u;
-    p.nchunks = static_cast<uint32_t>(ceil_div(p.row_bytes, kChunk));
-    p.stage_bytes = static_cast<uint32_t>(a.k) * kChunk;
+    p.nchunks = static_cast<uint32_t>(ceil_div(p.row_bytes, chunk));
+    p.stage_bytes = static_cast<uint32_t>(a.k) * chunk;
 
     int max_optin = 0;
     cudaError_t e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
@@ -346,9 +448,13 @@ cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t s
                                               : std::min(kDefaultSmemBudget, max_optin);
     int S = tu.combine_stages > 0 ? tu.combine_stages : kMaxBulkStages;
     S = std::min(S, kMaxBulkStages);
+    p.rank_off = a.rank_off;
+    p.R = a.R;
+    // rank-grouped order: the rank offsets plus 96 words per consumer warp
+    const size_t tables = RANKED ? sizeof(int32_t) * (static_cast<size_t>(a.R) + 1 + 96 * CW) : 0;
     auto smem_for = [&](int st) {
         return static_cast<size_t>(round_up(2 * st * 8, 128)) +
-               static_cast<size_t>(st) * p.stage_bytes;
+               static_cast<size_t>(st) * p.stage_bytes + tables;
     };
     while (S > 2 && smem_for(S) > static_cast<size_t>(budget))
         --S;
@@ -356,20 +462,22 @@ cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t s
         return cudaErrorInvalidValue;
     p.stages = static_cast<uint32_t>(S);
     p.bar_bytes = static_cast<uint32_t>(round_up(2 * S * 8, 128));
+    p.ring_bytes = static_cast<uint32_t>(S) * p.stage_bytes;
     const size_t smem = smem_for(S);
-    auto kern = a.k <= 8 ? combine_bulk_kernel<8> : combine_bulk_kernel<32>;
+    auto kern = combine_bulk_kernel<KMAX, CW, RANKED>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess)
         return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBulkThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
     if (e != cudaSuccess)
         return e;
     if (per_sm < 1)
         return cudaErrorInvalidConfiguration;
+    // the default keeps about 12 consumer warps per SM whatever the chunk width
     per_sm = std::min(per_sm, tu.combine_ctas_per_sm > 0 ? tu.combine_ctas_per_sm
-                                                          : kDefaultCtasPerSm);
+                                                          : kDefaultCtasPerSm * 4 / CW);
     // Contiguous runs of tokens per CTA; the grid covers all tokens so that CTAs that
     // finish early are replaced by the block scheduler.
     const int64_t resident = static_cast<int64_t>(sm_count(device)) * per_sm;
@@ -379,8 +487,18 @@ cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t s
         per_cta = std::max<int64_t>(1, ceil_div(a.N, resident));
     p.per_cta = static_cast<uint32_t>(per_cta);
     const int64_t grid = std::max<int64_t>(1, ceil_div(a.N, per_cta));
-    kern<<<static_cast<unsigned>(grid), kBulkThreads, smem, stream>>>(p);
+    kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(p);
     return cudaGetLastError();
+}
+
+template <bool RANKED>
+cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t stream)
+{
+    if (a.k <= 8)
+        return launch_bulk_shape<8, 4, RANKED>(a, device, stream);
+    if (a.k <= 16)
+        return launch_bulk_shape<16, 2, RANKED>(a, device, stream);
+    return launch_bulk_shape<32, 1, RANKED>(a, device, stream);
 }
 
 cudaError_t launch_combine(const CombineArgs &a, int device, cudaStream_t stream)
@@ -388,8 +506,10 @@ cudaError_t launch_combine(const CombineArgs &a, int device, cudaStream_t stream
     if (a.N == 0)
         return cudaSuccess;
     const Tuning &tu = tuning();
+    if (a.ranked)
+        return launch_combine_bulk<true>(a, device, stream);
     if (tu.combine_mode != 2)
-        return launch_combine_bulk(a, device, stream);
+        return launch_combine_bulk<false>(a, device, stream);
     int vpl = tu.combine_vec_per_lane > 0 ? tu.combine_vec_per_lane : 1;
     if (vpl != 1 && vpl != 2 && vpl != 4)
         vpl = 1;

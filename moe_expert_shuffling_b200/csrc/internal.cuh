@@ -94,6 +94,9 @@ struct CombineArgs {
     uint16_t *out;         // bf16 [N, H]
     uint32_t *err;
     int32_t N, k, n_rows, H;
+    const int32_t *rank_off = nullptr;  // [R+1], for the rank-grouped order
+    int32_t R = 0;
+    bool ranked = false;   // rank-grouped summation order instead of one chain
 };
 cudaError_t launch_combine(const CombineArgs &a, int device, cudaStream_t stream);
 

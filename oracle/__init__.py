@@ -41,6 +41,9 @@ def _bind(path: str):
     lib.oracle_dispatch.argtypes = [_u8p, _u8p, _i32p, _i64, _i32, _i64, _i64, _u8p, _u8p]
     lib.oracle_combine.restype = None
     lib.oracle_combine.argtypes = [_u16p, _i32p, _f32p, _i64, _i32, _i64, _u16p]
+    lib.oracle_combine_ranked.restype = None
+    lib.oracle_combine_ranked.argtypes = [_u16p, _i32p, _f32p, _i32p, _i64, _i32, _i64, _i32,
+                                          _i32, _u16p]
     lib.oracle_combine_f64.restype = None
     lib.oracle_combine_f64.argtypes = [_u16p, _i32p, _f32p, _i64, _i32, _i64, _f64p]
     lib.oracle_f32_to_bf16.restype = None
@@ -164,6 +167,21 @@ def combine(y_bf16_bits: np.ndarray, slot: np.ndarray, w: np.ndarray) -> np.ndar
     H = y.shape[1]
     out = np.zeros((N, H), np.uint16)
     _lib().oracle_combine(_p(y, _u16p), _p(sl, _i32p), _p(ww, _f32p), N, k, H, _p(out, _u16p))
+    return out
+
+
+def combine_ranked(y_bf16_bits: np.ndarray, slot: np.ndarray, w: np.ndarray,
+                   topk_idx: np.ndarray, E: int, R: int) -> np.ndarray:
+    """Rank-grouped combine: per-rank fp32 fma chains, then fp32 adds across ranks."""
+    y = np.ascontiguousarray(y_bf16_bits.view(np.uint16))
+    sl = np.ascontiguousarray(slot, dtype=np.int32)
+    ww = np.ascontiguousarray(w, dtype=np.float32)
+    idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    N, k = sl.shape
+    H = y.shape[1]
+    out = np.zeros((N, H), np.uint16)
+    _lib().oracle_combine_ranked(_p(y, _u16p), _p(sl, _i32p), _p(ww, _f32p), _p(idx, _i32p), N,
+                                 k, H, E, R, _p(out, _u16p))
     return out
 
 

@@ -26,7 +26,7 @@
  *                bf16_rne( fp32 fma chain over j = 0..k-1 of w[t,j] * y[slot[t,j]] ).
  *                The chain order and fp32 accumulation are fixed by the accuracy
  *                target; combine_f64 is the exact-order-free float64 sum used to bound
- *                the rounding error.
+ *                the rounding error; combine_ranked reduces per rank first.
  *
  * Readings where the pages are silent: expert e lives on rank e / (E/R); segments are
  * tight (no padding); ids of one token are distinct and in [0, E) -- anything else is
@@ -207,6 +207,40 @@ void oracle_combine(const uint16_t *y, const int32_t *slot, const float *w, int6
                 acc = fmaf(w[t * k + j], bf16_to_f32(y[s * H + c]), acc);
             }
             out[t * H + c] = f32_to_bf16_rne(acc);
+        }
+}
+
+/*
+ * Rank-grouped combine (the combine-side counterpart of the per-rank dedup; DySHARP blog,
+ * section 2: the partial results that several destinations produce for one token could be
+ * summed before they travel back, and section 5: dymultimem.ld_reduce returns one reduced
+ * result).  For each rank r in ascending order that holds some expert of token t, the
+ * rank's partial is the fp32 fma chain over the token's columns on r in ascending column
+ * order, starting from +0; the partials are then added in ascending rank order in fp32,
+ * starting from +0; the result is rounded to bf16 (nearest even).
+ */
+void oracle_combine_ranked(const uint16_t *y, const int32_t *slot, const float *w,
+                           const int32_t *topk_idx, int64_t N, int32_t k, int64_t H, int32_t E,
+                           int32_t R, uint16_t *out)
+{
+    const int32_t epr = E / R;
+    for (int64_t t = 0; t < N; ++t)
+        for (int64_t c = 0; c < H; ++c) {
+            float total = 0.0f;
+            for (int32_t r = 0; r < R; ++r) {
+                int any = 0;
+                float part = 0.0f;
+                for (int32_t j = 0; j < k; ++j) {
+                    if (topk_idx[t * k + j] / epr != r)
+                        continue;
+                    int64_t s = slot[t * k + j];
+                    part = fmaf(w[t * k + j], bf16_to_f32(y[s * H + c]), part);
+                    any = 1;
+                }
+                if (any)
+                    total = total + part;
+            }
+            out[t * H + c] = f32_to_bf16_rne(total);
         }
 }
 

@@ -75,6 +75,42 @@ def test_more_seeds(name, seed):
     assert np.array_equal(r["got_out"], r["ref_out"])
 
 
+@pytest.mark.parametrize("name", ["dsv3_k16", "dsv3_k32"])
+def test_wide_topk_parity(name):
+    """Top-16 and top-32 of 256 experts (the wider-fan-out settings), 4096 tokens."""
+    cfg = CONFIGS[name].with_tokens(4096)
+    r = run_all(cfg, 0)
+    assert_plan_equal(r["gp"], r["ref"])
+    assert np.array_equal(r["got_recv"], r["ref_recv"])
+    assert_combine_close(r["got_out"], r["ref_out"])
+    assert np.array_equal(r["got_out"], r["ref_out"])
+
+
+@pytest.mark.parametrize("cfg", [
+    CONFIGS["dsv3"].with_tokens(2000),
+    CONFIGS["skew"].with_tokens(1000),
+    CONFIGS["long"].with_tokens(3000),
+    CONFIGS["mixtral"].with_tokens(1000),
+    CONFIGS["tiny"],
+    CONFIGS["dsv3_k16"].with_tokens(500),
+    CONFIGS["dsv3_k32"].with_tokens(500),
+    CONFIGS["dsv3"].replace(N=300, H=64, E=1024, k=8, R=1024),
+    CONFIGS["dsv3"].replace(N=300, H=64, E=1024, k=8, R=1),
+], ids=lambda c: f"{c.name}-N{c.N}-E{c.E}-k{c.k}-R{c.R}")
+def test_ranked_combine_parity(cfg):
+    """moe_combine_ranked matches the oracle's rank-grouped order bit for bit."""
+    import moe_expert_shuffling_b200 as ms
+    idx, w, x, xs, y = make_inputs(cfg, 3)
+    p, ti, tw = gpu_plan(idx, w, cfg.E, cfg.R)
+    out = ms.moe_combine(y, p, ranked=True)
+    torch.cuda.synchronize()
+    ref = oracle.plan(idx, cfg.E, cfg.R)
+    want = oracle.combine_ranked(bits16(y), ref.slot, w, idx, cfg.E, cfg.R)
+    got = bits16(out)
+    assert_combine_close(got, want)
+    assert np.array_equal(got, want)
+
+
 @pytest.mark.parametrize("name", ["mixtral", "dsv3"])
 def test_identity_experts_return_x(name):
     """combine(dispatch(x)) == x with y = recv and weights summing to 1."""

@@ -65,6 +65,26 @@ def bf16_round(q):
     return _round_binary(q, 7, -126)
 
 
+def exact_combine_ranked(y_bits, slot, w, idx, E, R, tokens, cols):
+    """Rank-grouped order in exact rationals: per rank an fp32 fma chain, then fp32 adds."""
+    y = bits_to_f32(y_bits)
+    epr = E // R
+    out = {}
+    for t in tokens:
+        for c in cols:
+            total = Fraction(0)
+            for r in range(R):
+                cols_r = [j for j in range(slot.shape[1]) if idx[t, j] // epr == r]
+                if not cols_r:
+                    continue
+                part = Fraction(0)
+                for j in cols_r:
+                    part = f32_round(Fraction(float(w[t, j])) * Fraction(float(y[slot[t, j], c])) + part)
+                total = f32_round(total + part)
+            out[(t, c)] = bf16_round(total)
+    return out
+
+
 def exact_combine(y_bits, slot, w, tokens, cols):
     """fp32 fma chain from +0 in column order j = 0..k-1, then bf16 RNE, in exact rationals."""
     y = bits_to_f32(y_bits)
@@ -102,6 +122,36 @@ def fma_chain_at_scale(y_bits, slot, w):
             nxt[t, c] = np.float32(float(f32_round(exact)))
         acc = nxt
     return bf16_bits_of(acc)
+
+
+def _round32_sum(p64, a64):
+    """fp32 rounding of the exact sum of two float64 arrays holding exact values."""
+    from fractions import Fraction
+    s = p64 + a64
+    bb = s - p64
+    err = (p64 - (s - bb)) + (a64 - bb)
+    out = s.astype(np.float32)
+    for i in zip(*np.nonzero(err != 0)):
+        out[i] = np.float32(float(f32_round(Fraction(float(p64[i])) + Fraction(float(a64[i])))))
+    return out
+
+
+def ranked_at_scale(y_bits, slot, w, idx, E, R):
+    """Exact rank-grouped order for every output: per rank an fp32 fma chain, fp32 adds."""
+    yv = bits_to_f32(y_bits).astype(np.float64)
+    N, k = slot.shape
+    epr = E // R
+    out = np.zeros((N, yv.shape[1]), np.float32)
+    for t in range(N):
+        total = np.zeros(yv.shape[1], np.float32)
+        for r in sorted({int(e) // epr for e in idx[t]}):
+            part = np.zeros(yv.shape[1], np.float32)
+            for j in range(k):
+                if idx[t, j] // epr == r:
+                    part = _round32_sum(np.float64(w[t, j]) * yv[slot[t, j]], part.astype(np.float64))
+            total = _round32_sum(total.astype(np.float64), part.astype(np.float64))
+        out[t] = total
+    return bf16_bits_of(out)
 
 
 # --------------------------------------------------------------------------- dispatch
@@ -181,6 +231,64 @@ def test_combine_matches_exact_fma_chain_at_scale(name, N):
     p = oracle.plan(idx, cfg.E, cfg.R)
     yb = bits16(make_payload_y(cfg.replace(y="normal"), 4))
     assert np.array_equal(oracle.combine(yb, p.slot, w), fma_chain_at_scale(yb, p.slot, w))
+
+
+def test_ranked_combine_exact_rational():
+    cfg = CONFIGS["dsv3"].with_tokens(12).replace(H=48)
+    wl = make_workload(cfg, 5)
+    p = oracle.plan(wl.topk_idx, cfg.E, cfg.R)
+    yb = bits16(wl.y)
+    out = bits_to_f32(oracle.combine_ranked(yb, p.slot, wl.topk_w, wl.topk_idx, cfg.E, cfg.R))
+    ref = exact_combine_ranked(yb, p.slot, wl.topk_w, wl.topk_idx, cfg.E, cfg.R,
+                               range(cfg.N), range(cfg.H))
+    for (t, c), v in ref.items():
+        assert Fraction(float(out[t, c])) == v, (t, c)
+
+
+def test_ranked_combine_matches_exact_order_at_scale():
+    cfg = CONFIGS["dsv3"].with_tokens(256)
+    wl = make_workload(cfg, 8)
+    p = oracle.plan(wl.topk_idx, cfg.E, cfg.R)
+    yb = bits16(wl.y)
+    assert np.array_equal(oracle.combine_ranked(yb, p.slot, wl.topk_w, wl.topk_idx, cfg.E, cfg.R),
+                          ranked_at_scale(yb, p.slot, wl.topk_w, wl.topk_idx, cfg.E, cfg.R))
+
+
+def test_ranked_combine_with_one_rank_is_the_plain_chain():
+    cfg = CONFIGS["dsv3"].with_tokens(64).replace(H=128, R=1)
+    wl = make_workload(cfg, 6)
+    p = oracle.plan(wl.topk_idx, cfg.E, cfg.R)
+    yb = bits16(wl.y)
+    assert np.array_equal(oracle.combine_ranked(yb, p.slot, wl.topk_w, wl.topk_idx, cfg.E, 1),
+                          oracle.combine(yb, p.slot, wl.topk_w))
+
+
+def test_ranked_combine_differs_from_the_chain_only_by_rounding():
+    cfg = CONFIGS["dsv3"].with_tokens(128)
+    wl = make_workload(cfg, 7)
+    p = oracle.plan(wl.topk_idx, cfg.E, cfg.R)
+    yb = bits16(wl.y)
+    a = oracle.combine_ranked(yb, p.slot, wl.topk_w, wl.topk_idx, cfg.E, cfg.R)
+    b = oracle.combine(yb, p.slot, wl.topk_w)
+    exact = oracle.combine_f64(yb, p.slot, wl.topk_w)
+    assert not np.array_equal(a, b)          # the order matters somewhere
+    fa = bits_to_f32(a).astype(np.float64)
+    yv = bits_to_f32(yb).astype(np.float64)
+    mag = sum(np.abs(wl.topk_w[:, j:j + 1].astype(np.float64) * yv[p.slot[:, j]])
+              for j in range(cfg.k))
+    gamma = 2 * cfg.k * 2.0 ** -24 / (1 - 2 * cfg.k * 2.0 ** -24)
+    assert np.all(np.abs(fa - exact) <= np.abs(exact) * 2.0 ** -8 + 2.0 ** -134 + 1.01 * gamma * mag)
+
+
+@pytest.mark.parametrize("name,N", [("dsv3", 96), ("long", 96)])
+def test_ranked_identity_experts_return_x(name, N):
+    cfg = CONFIGS[name].with_tokens(N).replace(payload="bf16")
+    wl = make_workload(cfg, 0, with_y=False)
+    p = oracle.plan(wl.topk_idx, cfg.E, cfg.R)
+    xb = bits16(wl.x)
+    recv = oracle.dispatch(xb.view(np.uint8).reshape(N, -1), p.slot).view(np.uint16).reshape(-1, cfg.H)
+    out = oracle.combine_ranked(recv, p.slot, wl.topk_w, wl.topk_idx, cfg.E, cfg.R)
+    assert np.array_equal(bits_to_f32(out), bits_to_f32(xb))
 
 
 def test_combine_golden_ties_and_identity():

@@ -14,7 +14,8 @@ import torch
 import oracle
 from oracle.build import SRC, build_variant
 from tests.test_oracle_dispatch_combine import (
-    bf16_bits_of, bits16, bits_to_f32, exact_combine, fma_chain_at_scale,
+    bf16_bits_of, bits16, bits_to_f32, exact_combine, exact_combine_ranked, fma_chain_at_scale,
+    ranked_at_scale,
 )
 from tests.test_oracle_plan import GOLDEN, brute_plan, check_invariants
 from workloads import CONFIGS, make_routing, make_workload
@@ -48,6 +49,9 @@ MUTANTS = {
     "bf16_truncate": ("u += 0x7fffu + lsb;", "u += 0u * lsb;"),
     # rounding ties away from zero instead of to even
     "bf16_ties_away": ("u += 0x7fffu + lsb;", "u += 0x8000u + 0u * lsb;"),
+    # rank-grouped combine visits the ranks in descending order
+    "ranked_descending": ("for (int32_t r = 0; r < R; ++r) {\n                int any = 0;",
+                          "for (int32_t r = R - 1; r >= 0; --r) {\n                int any = 0;"),
     # drops the last expert of each token
     "skip_last_column": ("    for (int64_t t = 0; t < N; ++t)\n        for (int32_t j = 0; j < k; ++j)\n            cnt[topk_idx[t * k + j]] += 1;",
                          "    for (int64_t t = 0; t < N; ++t)\n        for (int32_t j = 0; j + 1 < k; ++j)\n            cnt[topk_idx[t * k + j]] += 1;"),
@@ -119,13 +123,22 @@ def run_pins():
         yb = bits16(make_payload_y(cfg, 4))
         assert np.array_equal(oracle.combine(yb, p.slot, w), fma_chain_at_scale(yb, p.slot, w))
 
+    def ranked():
+        cfg = CONFIGS["dsv3"].with_tokens(256)
+        wl = make_workload(cfg, 8)
+        p = oracle.plan(wl.topk_idx, cfg.E, cfg.R)
+        yb = bits16(wl.y)
+        assert np.array_equal(
+            oracle.combine_ranked(yb, p.slot, wl.topk_w, wl.topk_idx, cfg.E, cfg.R),
+            ranked_at_scale(yb, p.slot, wl.topk_w, wl.topk_idx, cfg.E, cfg.R))
+
     def rounding():
         vals = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, 257.0, 259.0, 1.2345], np.float32)
         assert np.array_equal(oracle.f32_to_bf16(vals), bf16_bits_of(vals))
 
     for name, fn in (("golden", golden), ("brute", brute), ("invariants", invariants),
                      ("dispatch", dispatch_rows), ("exact_combine", exact),
-                     ("chain_at_scale", chain_at_scale),
+                     ("chain_at_scale", chain_at_scale), ("ranked", ranked),
                      ("rounding", rounding)):
         pin(name, fn)
     return failures

@@ -112,7 +112,8 @@ def test_brute_force_tiny(seed):
     check_invariants(p, idx, cfg.E, cfg.R)
 
 
-@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "skew", "long"])
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "skew", "long", "dsv3_k16",
+                                  "dsv3_k32"])
 def test_invariants_all_configs(name):
     cfg = CONFIGS[name]
     idx, _ = make_routing(cfg, 0)
@@ -153,7 +154,7 @@ def test_empty_input():
     assert np.all(p.expert_off == 0) and np.all(p.rtok_off == 0)
 
 
-@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "long"])
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "dsv3", "long", "dsv3_k16", "dsv3_k32"])
 def test_distinct_rank_closed_form(name):
     """Mean distinct ranks per token matches R * (1 - C(E-E/R, k)/C(E, k)) within 5 s.e."""
     cfg = CONFIGS[name]

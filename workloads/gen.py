@@ -88,6 +88,12 @@ CONFIGS = {
                    routing="zipf", weights="sigmoid", y="normal"),
     "long": Config("long", N=65536, H=4096, E=64, k=6, R=16, payload="fp8",
                    routing="uniform", weights="softmax", y="normal"),
+    # DeepSeek-V3 with wider top-k, the medium and large settings of the DySHARP study
+    # (topk 16 and 32; "Accelerating MoE with Dynamic In-Switch Computing", section 7)
+    "dsv3_k16": Config("dsv3_k16", N=16384, H=7168, E=256, k=16, R=32, payload="bf16",
+                       routing="uniform", weights="sigmoid", y="normal"),
+    "dsv3_k32": Config("dsv3_k32", N=16384, H=7168, E=256, k=32, R=32, payload="bf16",
+                       routing="uniform", weights="sigmoid", y="normal"),
 }
 
 
