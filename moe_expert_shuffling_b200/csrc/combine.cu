@@ -252,6 +252,9 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
             0xffffffffu,
             lane < k && static_cast<uint32_t>(s_nxt) < static_cast<uint32_t>(p.n_rows));
         float wv[RANKED ? 1 : KMAX];
+        constexpr int KR = (RANKED && KMAX <= 8) ? KMAX : 1;
+        int32_t ordr[KR], ror[KR];
+        float wor[KR];
         if (!RANKED) {
 #pragma unroll
             for (int j = 0; j < (RANKED ? 1 : KMAX); ++j)
@@ -283,6 +286,15 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
                 ro_s[pos] = rj;
             }
             __syncwarp();
+            if (KMAX <= 8) {
+                // small k: keep the token's order in registers for all of its chunks
+#pragma unroll
+                for (int pq = 0; pq < (KMAX <= 8 ? KMAX : 1); ++pq) {
+                    ordr[pq] = pq < k ? ord_s[pq] : 0;
+                    wor[pq] = pq < k ? wo_s[pq] : 0.f;
+                    ror[pq] = pq < k ? ro_s[pq] : kNoRank;
+                }
+            }
         }
         if (m + 1 < n_tok && lane < k) {
             s_nxt = __ldg(p.slot + static_cast<int64_t>(t + 1) * k + lane);
@@ -315,9 +327,10 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
 #pragma unroll
                     for (int pp = 0; pp < 8; ++pp) {
                         const int pq = p0 + pp;
-                        const bool use = pq < k && ro_s[pq] != kNoRank;
-                        q[pp] = (mine && use) ? lds_v4(stage + ord_s[pq] * kChunk_)
-                                              : make_uint4(0u, 0u, 0u, 0u);
+                        const int32_t rr = KMAX <= 8 ? ror[pp] : (pq < k ? ro_s[pq] : kNoRank);
+                        const int32_t jr = KMAX <= 8 ? ordr[pp] : ord_s[pq < k ? pq : 0];
+                        q[pp] = (mine && rr != kNoRank) ? lds_v4(stage + jr * kChunk_)
+                                                        : make_uint4(0u, 0u, 0u, 0u);
                     }
                     if (p0 + 8 >= k) {
                         __syncwarp();
@@ -327,7 +340,7 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
 #pragma unroll
                     for (int pp = 0; pp < 8; ++pp) {
                         const int pq = p0 + pp;
-                        const int32_t rr = pq < k ? ro_s[pq] : kNoRank;
+                        const int32_t rr = KMAX <= 8 ? ror[pp] : (pq < k ? ro_s[pq] : kNoRank);
                         if (rr == kNoRank)
                             continue;
                         if (rr != prev) {
@@ -341,7 +354,7 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
                                 part[e] = 0.f;
                             prev = rr;
                         }
-                        fma_bf16x8(part, wo_s[pq], q[pp]);
+                        fma_bf16x8(part, KMAX <= 8 ? wor[pp] : wo_s[pq], q[pp]);
                     }
                 }
                 if (prev >= 0) {

@@ -33,6 +33,9 @@ def _bind(path: str):
     lib.oracle_plan.restype = ctypes.c_int
     lib.oracle_plan.argtypes = [_i32p, _i64, _i32, _i32, _i32, _i32p, _i32p, _i32p, _i32p,
                                 _i32p, _i32p, _i32p, _i32p, _i32p, _u32p, _i64]
+    lib.oracle_plan_ex.restype = ctypes.c_int
+    lib.oracle_plan_ex.argtypes = [_i32p, _i64, _i32, _i32, _i32, _i32, _i32p, _i32p, _i32p,
+                                   _i32p, _i32p, _i32p, _i32p, _i32p, _i32p, _u32p, _i64]
     lib.oracle_validate.restype = ctypes.c_int
     lib.oracle_validate.argtypes = [_i32p, _i64, _i32, _i32]
     lib.oracle_dedup_count.restype = ctypes.c_int64
@@ -94,11 +97,17 @@ class Plan:
     rcnt: np.ndarray        # int32 [R]
     rank_off: np.ndarray    # int32 [R+1]
     rtok_off: np.ndarray    # int32 [R+1]
-    slot: np.ndarray        # int32 [N, k]
-    src_tok: np.ndarray     # int32 [N*k]
-    src_j: np.ndarray       # int32 [N*k]
+    slot: np.ndarray        # int32 [N, k] (-1 for a dropped entry)
+    src_tok: np.ndarray     # int32 [rows] (-1 for padding and unused rows)
+    src_j: np.ndarray       # int32 [rows]
     rtok: np.ndarray        # int32 [sum rcnt]
     fanout: np.ndarray      # uint32 [sum rcnt]
+    align: int = 1
+
+    @property
+    def rows(self) -> int:
+        """Receive rows a buffer must hold: N*k + E*(align - 1)."""
+        return self.N * self.k + self.E * (self.align - 1)
 
 
 def validate(topk_idx: np.ndarray, E: int) -> bool:
@@ -113,42 +122,48 @@ def dedup_count(topk_idx: np.ndarray, E: int, R: int) -> int:
     return int(_lib().oracle_dedup_count(_p(idx, _i32p), N, k, E, R))
 
 
-def plan(topk_idx: np.ndarray, E: int, R: int) -> Plan:
+def plan(topk_idx: np.ndarray, E: int, R: int, align: int = 1) -> Plan:
+    """The segment plan; ids of -1 are dropped entries; segments start on multiples of align."""
     idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
     N, k = idx.shape
     cap = max(1, N * min(k, R))
+    rows = N * k + E * (max(align, 1) - 1)
     cnt = np.zeros(E, np.int32)
     expert_off = np.zeros(E + 1, np.int32)
     rcnt = np.zeros(R, np.int32)
     rank_off = np.zeros(R + 1, np.int32)
     rtok_off = np.zeros(R + 1, np.int32)
     slot = np.zeros((N, k), np.int32)
-    src_tok = np.zeros(max(1, N * k), np.int32)
-    src_j = np.zeros(max(1, N * k), np.int32)
+    src_tok = np.zeros(max(1, rows), np.int32)
+    src_j = np.zeros(max(1, rows), np.int32)
     rtok = np.zeros(cap, np.int32)
     fanout = np.zeros(cap, np.uint32)
-    rc = _lib().oracle_plan(_p(idx, _i32p), N, k, E, R, _p(cnt, _i32p), _p(expert_off, _i32p),
-                            _p(rcnt, _i32p), _p(rank_off, _i32p), _p(rtok_off, _i32p),
-                            _p(slot, _i32p), _p(src_tok, _i32p), _p(src_j, _i32p),
-                            _p(rtok, _i32p), _p(fanout, _u32p), cap)
+    rc = _lib().oracle_plan_ex(_p(idx, _i32p), N, k, E, R, align, _p(cnt, _i32p),
+                               _p(expert_off, _i32p), _p(rcnt, _i32p), _p(rank_off, _i32p),
+                               _p(rtok_off, _i32p), _p(slot, _i32p), _p(src_tok, _i32p),
+                               _p(src_j, _i32p), _p(rtok, _i32p), _p(fanout, _u32p), cap)
     if rc != 0:
         raise OracleError("invalid routing or shape")
     n = int(rtok_off[R])
     return Plan(N, k, E, R, cnt, expert_off, rcnt, rank_off, rtok_off, slot,
-                src_tok[:N * k].copy(), src_j[:N * k].copy(), rtok[:n].copy(), fanout[:n].copy())
+                src_tok[:rows].copy(), src_j[:rows].copy(), rtok[:n].copy(), fanout[:n].copy(),
+                align)
 
 
-def dispatch(x_rows: np.ndarray, slot: np.ndarray, x_scale_rows: np.ndarray | None = None):
-    """x_rows: uint8 [N, row_bytes]; returns recv uint8 [N*k, row_bytes] (and scales)."""
+def dispatch(x_rows: np.ndarray, slot: np.ndarray, x_scale_rows: np.ndarray | None = None,
+             rows: int | None = None):
+    """x_rows: uint8 [N, row_bytes]; returns recv uint8 [rows, row_bytes] (and scales), rows
+    defaulting to N*k; rows no entry maps to stay zero."""
     x = np.ascontiguousarray(x_rows.view(np.uint8).reshape(x_rows.shape[0], -1))
     sl = np.ascontiguousarray(slot, dtype=np.int32)
     N, k = sl.shape
     rb = x.shape[1]
-    recv = np.zeros((N * k, rb), np.uint8)
+    nrows = N * k if rows is None else rows
+    recv = np.zeros((nrows, rb), np.uint8)
     if x_scale_rows is not None:
         xs = np.ascontiguousarray(x_scale_rows.view(np.uint8).reshape(N, -1))
         sb = xs.shape[1]
-        rs = np.zeros((N * k, sb), np.uint8)
+        rs = np.zeros((nrows, sb), np.uint8)
         _lib().oracle_dispatch(_p(x, _u8p), _p(xs, _u8p), _p(sl, _i32p), N, k, rb, sb,
                                _p(recv, _u8p), _p(rs, _u8p))
         return recv, rs

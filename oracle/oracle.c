@@ -29,7 +29,10 @@
  *                the rounding error; combine_ranked reduces per rank first.
  *
  * Readings where the pages are silent: expert e lives on rank e / (E/R); segments are
- * tight (no padding); ids of one token are distinct and in [0, E) -- anything else is
+ * tight unless an alignment is asked for, in which case each expert's segment starts on a
+ * multiple of `align` rows and the rows after its entries are padding (no token); an id
+ * of -1 marks an entry the router dropped (no receive row, no contribution, not an
+ * error); other ids are distinct within a token and in [0, E) -- anything else is
  * rejected with ORACLE_EINVAL.  Build: gcc -O2 -ffp-contract=off (no contraction, so
  * every fma below is the only fused operation).
  */
@@ -50,12 +53,16 @@ static int valid_shape(int64_t N, int32_t k, int32_t E, int32_t R)
     return 1;
 }
 
-/* 1 if every id is in [0,E) and no token lists an expert twice. */
+#define DROPPED (-1)
+
+/* 1 if every id is -1 (dropped) or in [0,E), and no token lists an expert twice. */
 int oracle_validate(const int32_t *topk_idx, int64_t N, int32_t k, int32_t E)
 {
     for (int64_t t = 0; t < N; ++t) {
         for (int32_t j = 0; j < k; ++j) {
             int32_t e = topk_idx[t * k + j];
+            if (e == DROPPED)
+                continue;
             if (e < 0 || e >= E)
                 return 0;
             for (int32_t i = 0; i < j; ++i)
@@ -64,6 +71,14 @@ int oracle_validate(const int32_t *topk_idx, int64_t N, int32_t k, int32_t E)
         }
     }
     return 1;
+}
+
+/* 1 when column j of token t is routed to an expert of rank r (dropped entries are not). */
+static int on_rank(const int32_t *topk_idx, int64_t t, int32_t j, int32_t k, int32_t epr,
+                   int32_t r)
+{
+    int32_t e = topk_idx[t * k + j];
+    return e != DROPPED && e / epr == r;
 }
 
 /* Number of (token, rank) moves: tokens counted once per distinct rank they touch. */
@@ -75,7 +90,7 @@ int64_t oracle_dedup_count(const int32_t *topk_idx, int64_t N, int32_t k, int32_
         for (int64_t t = 0; t < N; ++t) {
             int hit = 0;
             for (int32_t j = 0; j < k; ++j)
-                if (topk_idx[t * k + j] / epr == r)
+                if (on_rank(topk_idx, t, j, k, epr, r))
                     hit = 1;
             total += hit;
         }
@@ -84,47 +99,60 @@ int64_t oracle_dedup_count(const int32_t *topk_idx, int64_t N, int32_t k, int32_
 
 /*
  * Outputs (all caller-allocated):
- *   cnt[E]          entries routed to each expert
- *   expert_off[E+1] exclusive prefix sum of cnt (segment starts, expert-major)
+ *   cnt[E]          entries routed to each expert (dropped entries excluded)
+ *   expert_off[E+1] segment starts, expert-major: expert_off[e+1] = expert_off[e] +
+ *                   cnt[e] rounded up to a multiple of `align`
  *   rcnt[R]         tokens with at least one expert on rank r (dedup moves)
  *   rank_off[R+1]   first receive row of each rank = expert_off[r * E/R]
  *   rtok_off[R+1]   exclusive prefix sum of rcnt
- *   slot[N*k]       receive row of entry (t,j): expert_off[e] + #{t' < t routed to e}
- *   src_tok[N*k]    token of each receive row (inverse of slot)
- *   src_j[N*k]      top-k column of each receive row
+ *   slot[N*k]       receive row of entry (t,j): expert_off[e] + #{t' < t routed to e},
+ *                   or -1 for a dropped entry
+ *   src_tok[rows]   token of each receive row, -1 for padding and unused rows
+ *   src_j[rows]     top-k column of each receive row, -1 for padding and unused rows
  *   rtok[cap]       rtok[rtok_off[r] + i] = i-th smallest token touching rank r
  *   fanout[cap]     bit j set when column j of that token is an expert of rank r
+ * rows = N*k + E*(align - 1), the receive rows a buffer must hold.
  */
-int oracle_plan(const int32_t *topk_idx, int64_t N, int32_t k, int32_t E, int32_t R,
-                int32_t *cnt, int32_t *expert_off, int32_t *rcnt, int32_t *rank_off,
-                int32_t *rtok_off, int32_t *slot, int32_t *src_tok, int32_t *src_j,
-                int32_t *rtok, uint32_t *fanout, int64_t rtok_cap)
+int oracle_plan_ex(const int32_t *topk_idx, int64_t N, int32_t k, int32_t E, int32_t R,
+                   int32_t align, int32_t *cnt, int32_t *expert_off, int32_t *rcnt,
+                   int32_t *rank_off, int32_t *rtok_off, int32_t *slot, int32_t *src_tok,
+                   int32_t *src_j, int32_t *rtok, uint32_t *fanout, int64_t rtok_cap)
 {
-    if (!valid_shape(N, k, E, R) || !oracle_validate(topk_idx, N, k, E))
+    if (!valid_shape(N, k, E, R) || align < 1 || !oracle_validate(topk_idx, N, k, E))
         return ORACLE_EINVAL;
     const int32_t epr = E / R;
+    const int64_t rows = N * k + (int64_t)E * (align - 1);
 
     /* histogram over experts */
     for (int32_t e = 0; e < E; ++e)
         cnt[e] = 0;
     for (int64_t t = 0; t < N; ++t)
         for (int32_t j = 0; j < k; ++j)
-            cnt[topk_idx[t * k + j]] += 1;
+            if (topk_idx[t * k + j] != DROPPED)
+                cnt[topk_idx[t * k + j]] += 1;
 
-    /* exclusive scan: segment starts */
+    /* exclusive scan of the (aligned) segment sizes: segment starts */
     expert_off[0] = 0;
     for (int32_t e = 0; e < E; ++e)
-        expert_off[e + 1] = expert_off[e] + cnt[e];
+        expert_off[e + 1] = expert_off[e] + (cnt[e] + align - 1) / align * align;
     for (int32_t r = 0; r <= R; ++r)
         rank_off[r] = expert_off[r * epr];
 
     /* stable rank inside each segment: tokens in ascending order */
+    for (int64_t i = 0; i < rows; ++i) {
+        src_tok[i] = -1;
+        src_j[i] = -1;
+    }
     int32_t *fill = (int32_t *)calloc((size_t)E, sizeof(int32_t));
     if (!fill)
         return ORACLE_EINVAL;
     for (int64_t t = 0; t < N; ++t)
         for (int32_t j = 0; j < k; ++j) {
             int32_t e = topk_idx[t * k + j];
+            if (e == DROPPED) {
+                slot[t * k + j] = -1;
+                continue;
+            }
             int32_t s = expert_off[e] + fill[e];
             fill[e] += 1;
             slot[t * k + j] = s;
@@ -140,7 +168,7 @@ int oracle_plan(const int32_t *topk_idx, int64_t N, int32_t k, int32_t E, int32_
         for (int64_t t = 0; t < N; ++t) {
             uint32_t mask = 0;
             for (int32_t j = 0; j < k; ++j)
-                if (topk_idx[t * k + j] / epr == r)
+                if (on_rank(topk_idx, t, j, k, epr, r))
                     mask |= 1u << j;
             if (mask) {
                 int64_t pos = (int64_t)rtok_off[r] + n;
@@ -157,6 +185,16 @@ int oracle_plan(const int32_t *topk_idx, int64_t N, int32_t k, int32_t E, int32_
     return ORACLE_OK;
 }
 
+/* The plan with tight segments (align = 1). */
+int oracle_plan(const int32_t *topk_idx, int64_t N, int32_t k, int32_t E, int32_t R,
+                int32_t *cnt, int32_t *expert_off, int32_t *rcnt, int32_t *rank_off,
+                int32_t *rtok_off, int32_t *slot, int32_t *src_tok, int32_t *src_j,
+                int32_t *rtok, uint32_t *fanout, int64_t rtok_cap)
+{
+    return oracle_plan_ex(topk_idx, N, k, E, R, 1, cnt, expert_off, rcnt, rank_off, rtok_off,
+                          slot, src_tok, src_j, rtok, fanout, rtok_cap);
+}
+
 /*
  * recv[slot[t,j]] = x[t] for every entry; row_bytes payload bytes per row.  With
  * scale_bytes > 0 the per-row scale block x_scale[t] moves to recv_scale[slot[t,j]].
@@ -168,6 +206,8 @@ void oracle_dispatch(const uint8_t *x, const uint8_t *x_scale, const int32_t *sl
     for (int64_t t = 0; t < N; ++t)
         for (int32_t j = 0; j < k; ++j) {
             int64_t s = slot[t * k + j];
+            if (s < 0)
+                continue; /* dropped entry: no receive row */
             memcpy(recv + s * row_bytes, x + t * row_bytes, (size_t)row_bytes);
             if (scale_bytes > 0)
                 memcpy(recv_scale + s * scale_bytes, x_scale + t * scale_bytes,
@@ -204,6 +244,8 @@ void oracle_combine(const uint16_t *y, const int32_t *slot, const float *w, int6
             float acc = 0.0f;
             for (int32_t j = 0; j < k; ++j) {
                 int64_t s = slot[t * k + j];
+                if (s < 0)
+                    continue; /* dropped entry contributes nothing */
                 acc = fmaf(w[t * k + j], bf16_to_f32(y[s * H + c]), acc);
             }
             out[t * H + c] = f32_to_bf16_rne(acc);
@@ -231,7 +273,7 @@ void oracle_combine_ranked(const uint16_t *y, const int32_t *slot, const float *
                 int any = 0;
                 float part = 0.0f;
                 for (int32_t j = 0; j < k; ++j) {
-                    if (topk_idx[t * k + j] / epr != r)
+                    if (!on_rank(topk_idx, t, j, k, epr, r))
                         continue;
                     int64_t s = slot[t * k + j];
                     part = fmaf(w[t * k + j], bf16_to_f32(y[s * H + c]), part);
@@ -255,6 +297,8 @@ void oracle_combine_f64(const uint16_t *y, const int32_t *slot, const float *w, 
             double acc = 0.0;
             for (int32_t j = 0; j < k; ++j) {
                 int64_t s = slot[t * k + j];
+                if (s < 0)
+                    continue;
                 acc += (double)w[t * k + j] * (double)bf16_to_f32(y[s * H + c]);
             }
             out[t * H + c] = acc;

@@ -359,3 +359,30 @@ def test_combine_within_float64_error_bound(name, N):
     chain_err = gamma * mag
     half_ulp = np.abs(exact) * 2.0 ** -8 + 2.0 ** -134  # >= half a bf16 ulp (7 fraction bits)
     assert np.all(np.abs(out - exact) <= half_ulp + chain_err * 1.01)
+
+
+def test_dispatch_and_combine_skip_dropped_entries():
+    """A dropped entry gets no row and adds nothing: combine equals the chain over the
+    token's remaining columns (computed with k-1 columns by moving the dropped one out)."""
+    cfg = CONFIGS["tiny"].replace(k=3)
+    wl = make_workload(cfg, 2)
+    idx = wl.topk_idx.copy()
+    idx[::3, 2] = -1                        # drop the last column of every third token
+    p = oracle.plan(idx, cfg.E, cfg.R, align=4)
+    xb = bits16(wl.x)
+    recv = oracle.dispatch(xb.view(np.uint8).reshape(cfg.N, -1), p.slot, rows=p.rows)
+    rows16 = recv.view(np.uint16).reshape(p.rows, cfg.H)
+    used = p.src_tok >= 0
+    assert np.array_equal(rows16[used], xb[p.src_tok[used]])
+    assert not rows16[~used].any()          # rows no entry maps to are left untouched
+    y = np.random.default_rng(1).standard_normal((p.rows, cfg.H)).astype(np.float32)
+    yb = bf16_bits_of(y)
+    out = oracle.combine(yb, p.slot, wl.topk_w)
+    # reference: for dropped tokens use only columns 0..1 (a k=2 chain), else all three
+    w2 = wl.topk_w.copy()
+    sl2 = p.slot.copy()
+    keep = idx[:, 2] >= 0
+    ref_full = oracle.combine(yb, np.where(sl2 < 0, 0, sl2), w2)
+    ref_two = oracle.combine(yb, np.ascontiguousarray(sl2[:, :2]), np.ascontiguousarray(w2[:, :2]))
+    assert np.array_equal(out[keep], ref_full[keep])
+    assert np.array_equal(out[~keep], ref_two[~keep])

@@ -17,21 +17,21 @@ from tests.test_oracle_dispatch_combine import (
     bf16_bits_of, bits16, bits_to_f32, exact_combine, exact_combine_ranked, fma_chain_at_scale,
     ranked_at_scale,
 )
-from tests.test_oracle_plan import GOLDEN, brute_plan, check_invariants
+from tests.test_oracle_plan import GOLDEN, GOLDEN_DA, brute_plan, check_aligned, check_invariants, drop_some
 from workloads import CONFIGS, make_routing, make_workload
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 MUTANTS = {
     # stable order broken: fill segments with tokens in descending order
-    "descending_fill": ("for (int64_t t = 0; t < N; ++t)\n        for (int32_t j = 0; j < k; ++j) {\n            int32_t e = topk_idx[t * k + j];\n            int32_t s = expert_off[e] + fill[e];",
-                        "for (int64_t t = N - 1; t >= 0; --t)\n        for (int32_t j = 0; j < k; ++j) {\n            int32_t e = topk_idx[t * k + j];\n            int32_t s = expert_off[e] + fill[e];"),
+    "descending_fill": ("for (int64_t t = 0; t < N; ++t)\n        for (int32_t j = 0; j < k; ++j) {\n            int32_t e = topk_idx[t * k + j];\n            if (e == DROPPED) {",
+                        "for (int64_t t = N - 1; t >= 0; --t)\n        for (int32_t j = 0; j < k; ++j) {\n            int32_t e = topk_idx[t * k + j];\n            if (e == DROPPED) {"),
     # inclusive instead of exclusive segment starts
-    "inclusive_scan": ("expert_off[e + 1] = expert_off[e] + cnt[e];",
-                       "expert_off[e + 1] = expert_off[e] + cnt[e] + (e == 0 ? cnt[0] : 0);"),
+    "inclusive_scan": ("expert_off[e + 1] = expert_off[e] + (cnt[e] + align - 1) / align * align;",
+                       "expert_off[e + 1] = expert_off[e] + (cnt[e] + align - 1) / align * align + (e == 0 ? cnt[0] : 0);"),
     # wrong expert -> rank map in the dedup (modulo instead of blocks)
-    "rank_modulo": ("if (topk_idx[t * k + j] / epr == r)\n                    mask |= 1u << j;",
-                    "if (topk_idx[t * k + j] % R == r)\n                    mask |= 1u << j;"),
+    "rank_modulo": ("return e != DROPPED && e / epr == r;",
+                    "return e != DROPPED && (e + 1) / epr == r;"),
     # rank segment starts taken from the wrong expert
     "rank_off_index": ("rank_off[r] = expert_off[r * epr];", "rank_off[r] = expert_off[r];"),
     # inverse map records the token instead of the column
@@ -40,8 +40,8 @@ MUTANTS = {
     "dispatch_neighbour": ("memcpy(recv + s * row_bytes, x + t * row_bytes, (size_t)row_bytes);",
                            "memcpy(recv + s * row_bytes, x + ((t + 1) % N) * row_bytes, (size_t)row_bytes);"),
     # combine sums the columns in reverse order
-    "combine_reversed": ("for (int32_t j = 0; j < k; ++j) {\n                int64_t s = slot[t * k + j];\n                acc = fmaf(",
-                         "for (int32_t j = k - 1; j >= 0; --j) {\n                int64_t s = slot[t * k + j];\n                acc = fmaf("),
+    "combine_reversed": ("for (int32_t j = 0; j < k; ++j) {\n                int64_t s = slot[t * k + j];\n                if (s < 0)\n                    continue; /* dropped entry contributes nothing */",
+                         "for (int32_t j = k - 1; j >= 0; --j) {\n                int64_t s = slot[t * k + j];\n                if (s < 0)\n                    continue; /* dropped entry contributes nothing */"),
     # multiply then add (two roundings) instead of a fused multiply-add
     "combine_mul_add": ("acc = fmaf(w[t * k + j], bf16_to_f32(y[s * H + c]), acc);",
                         "acc = w[t * k + j] * bf16_to_f32(y[s * H + c]) + acc;"),
@@ -52,9 +52,15 @@ MUTANTS = {
     # rank-grouped combine visits the ranks in descending order
     "ranked_descending": ("for (int32_t r = 0; r < R; ++r) {\n                int any = 0;",
                           "for (int32_t r = R - 1; r >= 0; --r) {\n                int any = 0;"),
+    # segments not padded to the requested alignment
+    "align_ignored": ("expert_off[e + 1] = expert_off[e] + (cnt[e] + align - 1) / align * align;",
+                      "expert_off[e + 1] = expert_off[e] + cnt[e] + 0 * align;"),
+    # dropped entries still placed (as expert 0)
+    "dropped_placed": ("            if (e == DROPPED) {\n                slot[t * k + j] = -1;\n                continue;\n            }",
+                       "            if (e == DROPPED) {\n                e = 0;\n            }"),
     # drops the last expert of each token
-    "skip_last_column": ("    for (int64_t t = 0; t < N; ++t)\n        for (int32_t j = 0; j < k; ++j)\n            cnt[topk_idx[t * k + j]] += 1;",
-                         "    for (int64_t t = 0; t < N; ++t)\n        for (int32_t j = 0; j + 1 < k; ++j)\n            cnt[topk_idx[t * k + j]] += 1;"),
+    "skip_last_column": ("for (int32_t j = 0; j < k; ++j)\n            if (topk_idx[t * k + j] != DROPPED)\n                cnt[topk_idx[t * k + j]] += 1;",
+                         "for (int32_t j = 0; j + 1 < k; ++j)\n            if (topk_idx[t * k + j] != DROPPED)\n                cnt[topk_idx[t * k + j]] += 1;"),
 }
 
 
@@ -132,6 +138,15 @@ def run_pins():
             oracle.combine_ranked(yb, p.slot, wl.topk_w, wl.topk_idx, cfg.E, cfg.R),
             ranked_at_scale(yb, p.slot, wl.topk_w, wl.topk_idx, cfg.E, cfg.R))
 
+    def dropped_aligned():
+        g = json.load(open(GOLDEN_DA))
+        p = oracle.plan(np.array(g["topk_idx"], np.int32), g["E"], g["R"], align=g["align"])
+        for name in ("cnt", "expert_off", "slot", "src_tok", "rtok", "fanout"):
+            assert np.array_equal(getattr(p, name), np.array(g["expected"][name])), name
+        cfg = CONFIGS["dsv3"].with_tokens(400)
+        idx = drop_some(make_routing(cfg, 3)[0], 0.1, 9)
+        check_aligned(oracle.plan(idx, cfg.E, cfg.R, align=16), idx, cfg.E, cfg.R, 16)
+
     def rounding():
         vals = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, 257.0, 259.0, 1.2345], np.float32)
         assert np.array_equal(oracle.f32_to_bf16(vals), bf16_bits_of(vals))
@@ -139,6 +154,7 @@ def run_pins():
     for name, fn in (("golden", golden), ("brute", brute), ("invariants", invariants),
                      ("dispatch", dispatch_rows), ("exact_combine", exact),
                      ("chain_at_scale", chain_at_scale), ("ranked", ranked),
+                     ("dropped_aligned", dropped_aligned),
                      ("rounding", rounding)):
         pin(name, fn)
     return failures

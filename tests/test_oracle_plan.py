@@ -16,6 +16,7 @@ import oracle
 from workloads import CONFIGS, ZIPF_ALPHA, distinct_rank_expectation, find_zipf_alpha, make_routing
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "token_ab_example.json")
+GOLDEN_DA = os.path.join(os.path.dirname(__file__), "golden", "token_ab_dropped_aligned.json")
 
 
 def brute_plan(idx, E, R):
@@ -202,7 +203,7 @@ def test_invalid_routing_rejected(bad):
     elif bad == "range_hi":
         idx[0, 0] = 8
     else:
-        idx[1, 0] = -1
+        idx[1, 0] = -2          # -1 would be a dropped entry, not an error
     assert not oracle.validate(idx, 8)
     with pytest.raises(oracle.OracleError):
         oracle.plan(idx, 8, 4)
@@ -215,3 +216,85 @@ def test_invalid_shape_rejected(E, R, k):
         idx[0] = np.arange(k) % E
     with pytest.raises(oracle.OracleError):
         oracle.plan(idx[:, :max(k, 1)] if k else np.zeros((1, 0), np.int32), E, R)
+
+
+# ------------------------------------------------- dropped entries and aligned segments
+def drop_some(idx, frac, seed):
+    rng = np.random.default_rng(seed)
+    out = idx.copy()
+    out[rng.random(idx.shape) < frac] = -1
+    return out
+
+
+def test_golden_dropped_and_aligned():
+    g = json.load(open(GOLDEN_DA))
+    p = oracle.plan(np.array(g["topk_idx"], np.int32), g["E"], g["R"], align=g["align"])
+    ex = g["expected"]
+    assert p.rows == ex["rows"]
+    for name in ("cnt", "expert_off", "rank_off", "slot", "src_tok", "src_j", "rcnt",
+                 "rtok_off", "rtok", "fanout"):
+        assert np.array_equal(getattr(p, name), np.array(ex[name])), name
+
+
+def check_aligned(p, idx, E, R, align):
+    valid = idx >= 0
+    assert np.all(p.expert_off % align == 0)
+    seg = np.diff(p.expert_off.astype(np.int64))
+    assert np.array_equal(seg, (p.cnt + align - 1) // align * align)
+    assert int(p.cnt.sum()) == int(valid.sum())
+    assert np.all(p.slot[~valid] == -1)
+    e = idx[valid]
+    s = p.slot[valid]
+    assert np.all(p.expert_off[e] <= s) and np.all(s < p.expert_off[e] + p.cnt[e])
+    assert len(np.unique(s)) == s.size
+    # every row that no entry maps to is marked -1 in the inverse maps
+    used = np.zeros(p.rows, bool)
+    used[s] = True
+    assert np.all(p.src_tok[~used] == -1) and np.all(p.src_j[~used] == -1)
+    t_of = np.nonzero(valid)[0]
+    assert np.array_equal(p.src_tok[s], t_of)
+    # the dedup ignores dropped entries
+    epr = E // R
+    for r in range(R):
+        toks = p.rtok[p.rtok_off[r]:p.rtok_off[r + 1]]
+        hit = valid & (np.where(valid, idx, 0) // epr == r)
+        assert np.array_equal(toks, np.nonzero(hit.any(axis=1))[0])
+
+
+@pytest.mark.parametrize("name,frac,align", [("tiny", 0.2, 1), ("tiny", 0.3, 8),
+                                             ("dsv3", 0.1, 128), ("long", 0.05, 64),
+                                             ("mixtral", 0.5, 16)])
+def test_dropped_and_aligned_invariants(name, frac, align):
+    cfg = CONFIGS[name].with_tokens(min(CONFIGS[name].N, 2000))
+    idx = drop_some(make_routing(cfg, 3)[0], frac, 9)
+    p = oracle.plan(idx, cfg.E, cfg.R, align=align)
+    check_aligned(p, idx, cfg.E, cfg.R, align)
+    # alignment only shifts segments: the rank inside a segment is the tight plan's
+    t = oracle.plan(idx, cfg.E, cfg.R, align=1)
+    valid = idx >= 0
+    e = idx[valid]
+    assert np.array_equal(p.slot[valid] - p.expert_off[e], t.slot[valid] - t.expert_off[e])
+    assert np.array_equal(p.rtok, t.rtok) and np.array_equal(p.fanout, t.fanout)
+
+
+def test_brute_force_with_drops():
+    cfg = CONFIGS["tiny"]
+    idx = drop_some(make_routing(cfg, 4)[0], 0.25, 11)
+    p = oracle.plan(idx, cfg.E, cfg.R)
+    rows = [[int(v) for v in row] for row in idx]
+    for t in range(cfg.N):
+        for j in range(cfg.k):
+            e = rows[t][j]
+            if e < 0:
+                assert p.slot[t, j] == -1
+                continue
+            below = sum(1 for row in rows for v in row if 0 <= v < e)
+            earlier = sum(1 for tp in range(t) if e in rows[tp])
+            assert p.slot[t, j] == below + earlier
+
+
+def test_all_dropped():
+    idx = -np.ones((50, 4), np.int32)
+    p = oracle.plan(idx, 16, 4, align=8)
+    assert p.cnt.sum() == 0 and p.rcnt.sum() == 0 and np.all(p.slot == -1)
+    assert np.all(p.expert_off == 0) and np.all(p.src_tok == -1)
