@@ -34,7 +34,10 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from workloads import CONFIGS, Config, make_payload_x, make_payload_y, make_routing  # noqa: E402
+from workloads import (  # noqa: E402
+    CONFIGS, Config, drop_entries, make_expert_outputs, make_payload_x, make_payload_y,
+    make_routing,
+)
 
 METRIC = "dispatch+combine effective HBM GB/s and % of B200 roofline; tokens/s"
 NOMINAL_HBM_GBS = 8000.0
@@ -42,16 +45,18 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 # ----------------------------------------------------------------------------- bytes
-def dispatch_bytes(cfg: Config, N: int | None = None) -> int:
-    """x rows read once, N*k receive rows written once, N*k slots read."""
+def dispatch_bytes(cfg: Config, N: int | None = None, entries: int | None = None) -> int:
+    """x rows read once, one receive row written per routed entry, N*k slots read."""
     N = cfg.N if N is None else N
-    return N * cfg.row_bytes + N * cfg.k * cfg.row_bytes + 4 * N * cfg.k
+    V = N * cfg.k if entries is None else entries
+    return N * cfg.row_bytes + V * cfg.row_bytes + 4 * N * cfg.k
 
 
-def combine_bytes(cfg: Config, N: int | None = None) -> int:
-    """N*k bf16 rows of y read, N bf16 out rows written, slots and weights read."""
+def combine_bytes(cfg: Config, N: int | None = None, entries: int | None = None) -> int:
+    """One bf16 row of y read per routed entry, N bf16 out rows written, slots and weights."""
     N = cfg.N if N is None else N
-    return 2 * N * cfg.k * cfg.H + 2 * N * cfg.H + 8 * N * cfg.k
+    V = N * cfg.k if entries is None else entries
+    return 2 * V * cfg.H + 2 * N * cfg.H + 8 * N * cfg.k
 
 
 def plan_bytes(cfg: Config, N: int | None = None) -> int:
@@ -220,18 +225,23 @@ def run_ours(args):
     stream = torch.cuda.Stream(device=dev)
 
     idx_h, w_h = make_routing(cfg, seed)
+    if args.drop > 0:
+        idx_h = drop_entries(idx_h, args.drop, seed)
+    entries = int((idx_h >= 0).sum())
+    rows = cfg.N * cfg.k + cfg.E * (args.align - 1)
     with torch.cuda.stream(stream):
         x, xs = make_payload_x(cfg, seed, dev)
-        y = make_payload_y(cfg, seed, dev)
+        y = (make_payload_y(cfg, seed, dev) if rows == cfg.N * cfg.k
+             else make_expert_outputs(rows, cfg.H, seed, dev) if cfg.y != "identity" else None)
         idx = torch.from_numpy(idx_h).to(dev)
         w = torch.from_numpy(w_h).to(dev)
-        recv = torch.empty((cfg.N * cfg.k, cfg.H), dtype=x.dtype, device=dev)
-        rs = (torch.empty((cfg.N * cfg.k, cfg.H // 128), dtype=torch.float32, device=dev)
+        recv = torch.empty((rows, cfg.H), dtype=x.dtype, device=dev)
+        rs = (torch.empty((rows, cfg.H // 128), dtype=torch.float32, device=dev)
               if cfg.payload == "fp8" else None)
         out = torch.empty((cfg.N, cfg.H), dtype=torch.bfloat16, device=dev)
     stream.synchronize()
     identity = y is None
-    plan = ms.moe_plan_create(cfg.N, cfg.k, cfg.E, cfg.R)
+    plan = ms.moe_plan_create(cfg.N, cfg.k, cfg.E, cfg.R, align=args.align)
 
     def step(ev=None):
         if ev is not None:
@@ -274,7 +284,7 @@ def run_ours(args):
     elapsed_ms = max_over_ranks(elapsed_ms, world)
     ms_per_step = elapsed_ms / args.steps
 
-    db, cb = dispatch_bytes(cfg), combine_bytes(cfg)
+    db, cb = dispatch_bytes(cfg, entries=entries), combine_bytes(cfg, entries=entries)
     value = job_throughput(db + cb, args.steps, world, elapsed_ms)
     tokens_per_s = cfg.N * args.steps * world / (elapsed_ms * 1e-3)
     peak, peak_kind = measured_hbm_peak()
@@ -346,8 +356,10 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if cfg.payload == "bf16" else "fp8e4m3", "accum_dtype": "f32",
         "data": "synthetic (seeded routing and N(0,1) payload; no traces or weights exist)",
-        "config": {"workload": workload_name(cfg) + ("" if args.combine == "chain" else
-                                                      ", combine grouped by rank"),
+        "config": {"workload": workload_name(cfg)
+                   + ("" if args.combine == "chain" else ", combine grouped by rank")
+                   + (f", segments aligned to {args.align} rows" if args.align > 1 else "")
+                   + (f", {args.drop:.0%} of entries dropped" if args.drop > 0 else ""),
                    "model": f"{cfg.name}-shaped MoE layer shuffle",
                    "global_batch": cfg.N * world, "seq_len": cfg.N, "parallelism": f"replicas{world}",
                    "ep_ranks_logical": cfg.R,
@@ -473,6 +485,10 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (small cases for profiling)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--align", type=int, default=1,
+                    help="start every expert segment on a multiple of this many rows")
+    ap.add_argument("--drop", type=float, default=0.0,
+                    help="fraction of routing entries marked dropped (id -1), seeded")
     ap.add_argument("--combine", default="chain", choices=["chain", "ranked"],
                     help="combine order: one fma chain per token, or grouped by rank first")
     ap.add_argument("--seed", type=int, default=0)

@@ -72,14 +72,16 @@ typedef struct {
     int32_t *rcnt;                 /* [R]    tokens that touch rank r (dedup moves) */
     int32_t *rank_off;             /* [R+1]  first receive row of each rank */
     int32_t *rtok_off;             /* [R+1]  start of each rank's dedup list */
-    int32_t *slot;                 /* [N*k]  receive row of entry (t, j), or -1 if invalid */
-    int32_t *src_tok;              /* [N*k]  token of each receive row */
-    int32_t *src_j;                /* [N*k]  top-k column of each receive row */
+    int32_t *slot;                 /* [N*k]  receive row of entry (t, j); -1 if dropped/invalid */
+    int32_t *src_tok;              /* [recv_rows] token of each receive row, -1 if none */
+    int32_t *src_j;                /* [recv_rows] top-k column of each receive row, -1 if none */
     int32_t *rtok;                 /* [sum rcnt] tokens of rank r, ascending */
     uint32_t *fanout;              /* [sum rcnt] bit j: column j of that token is on rank r */
     uint32_t *err;                 /* [1]    MOE_ERR_* bits of the last moe_plan call */
     const float *topk_w;           /* the weights given to the last moe_plan call */
     int32_t plan_kernels;          /* kernels the last moe_plan call enqueued (1 or 3) */
+    int32_t align;                 /* expert segments start on multiples of this many rows */
+    int32_t recv_rows;             /* rows a receive buffer needs: N*k + E*(align-1) */
 } moe_plan_view;
 
 /*
@@ -89,6 +91,18 @@ typedef struct {
  */
 MOE_API moe_status moe_plan_create(int32_t max_tokens, int32_t k, int32_t E, int32_t R,
                            moe_plan_t *out);
+
+/*
+ * moe_plan_create_aligned -- as moe_plan_create, with every expert segment of the receive
+ * buffer starting on a multiple of `align` rows (1 <= align <= 65536), e.g. the row tile of
+ * a grouped GEMM over the experts.  The rows between an expert's last entry and the next
+ * segment are padding: dispatch does not write them, combine does not read them, and
+ * src_tok/src_j mark them -1.  Receive buffers then need N*k + E*(align-1) rows
+ * (moe_plan_view.recv_rows).  The logical segments are the pages' (FUSCO summary,
+ * Group 3); the alignment is this library's option for the consumer of the segments.
+ */
+MOE_API moe_status moe_plan_create_aligned(int32_t max_tokens, int32_t k, int32_t E, int32_t R,
+                                           int32_t align, moe_plan_t *out);
 
 /*
  * moe_plan -- build the logical-segment plan of one routing (FUSCO abstract: the
@@ -106,8 +120,12 @@ MOE_API moe_status moe_plan_create(int32_t max_tokens, int32_t k, int32_t E, int
  *             allocation); otherwise *plan is reused and must have been created with
  *             the same (k, E, R) and capacity >= N, else MOE_EINVAL.
  *
+ * An id of -1 marks an entry the router dropped: it gets slot -1, no receive row and no
+ * share of the combine, and it is not an error.
+ *
  * Computes, for expert e on rank e / (E/R):
- *   cnt[e], expert_off = exclusive scan of cnt, rank_off[r] = expert_off[r*E/R];
+ *   cnt[e], expert_off = exclusive scan of cnt (each rounded up to the plan's alignment),
+ *   rank_off[r] = expert_off[r*E/R];
  *   slot[t,j] = expert_off[e] + #{t' < t : e in topk_idx[t',:]} (stable, ascending t);
  *   src_tok/src_j = inverse of slot;
  *   rcnt[r] = #{t : some expert of t is on r}, rtok_off = exclusive scan of rcnt,
@@ -130,8 +148,9 @@ MOE_API moe_status moe_plan(const int32_t *topk_idx, const float *topk_w, int32_
  *   x_scale     device fp32 [N, H/128] for fp8 (moved with its row), NULL for bf16
  *   H           elements per row
  *   plan        a plan built by moe_plan (its N and k are used)
- *   recv        device [N*k, H] of `dtype`, caller-allocated, fully overwritten
- *   recv_scale  device fp32 [N*k, H/128] for fp8, NULL for bf16
+ *   recv        device [recv_rows, H] of `dtype`, caller-allocated (recv_rows = N*k for a
+ *               tight plan); every row an entry maps to is written, others are untouched
+ *   recv_scale  device fp32 [recv_rows, H/128] for fp8, NULL for bf16
  * Rows are copied bit for bit; nothing is converted.
  */
 MOE_API moe_status moe_dispatch(const void *x, moe_dtype dtype, const float *x_scale, int32_t H,
@@ -143,7 +162,8 @@ MOE_API moe_status moe_dispatch(const void *x, moe_dtype dtype, const float *x_s
  * experts' results for a token are brought back and summed).  The chain order is the
  * top-k column order, so the result does not depend on the launch configuration.
  *
- *   y     device bf16 [N*k, H]  expert outputs in the receive layout
+ *   y     device bf16 [recv_rows, H]  expert outputs in the receive layout (rows no
+ *         entry maps to are not read)
  *   H     elements per row (H % 8 == 0)
  *   plan  the plan whose slots laid out y; its weights pointer is read
  *   out   device bf16 [N, H], caller-allocated, fully overwritten

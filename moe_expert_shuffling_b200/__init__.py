@@ -47,6 +47,7 @@ class _PlanView(ctypes.Structure):
         ("capacity_tokens", _i32), ("cnt", _vp), ("expert_off", _vp), ("rcnt", _vp),
         ("rank_off", _vp), ("rtok_off", _vp), ("slot", _vp), ("src_tok", _vp), ("src_j", _vp),
         ("rtok", _vp), ("fanout", _vp), ("err", _vp), ("topk_w", _vp), ("plan_kernels", _i32),
+        ("align", _i32), ("recv_rows", _i32),
     ]
 
 
@@ -59,6 +60,8 @@ def _load():
     st = ctypes.c_int
     lib.moe_plan_create.restype = st
     lib.moe_plan_create.argtypes = [_i32, _i32, _i32, _i32, ctypes.POINTER(_vp)]
+    lib.moe_plan_create_aligned.restype = st
+    lib.moe_plan_create_aligned.argtypes = [_i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp)]
     lib.moe_plan.restype = st
     lib.moe_plan.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, ctypes.POINTER(_vp)]
     lib.moe_dispatch.restype = st
@@ -173,6 +176,15 @@ class Plan:
         return self._view().capacity_tokens
 
     @property
+    def rows(self) -> int:
+        """Rows a receive buffer needs for the last plan: N*k + E*(align - 1)."""
+        return self._view().recv_rows
+
+    @property
+    def align(self) -> int:
+        return self._view().align
+
+    @property
     def plan_kernels(self) -> int:
         """Kernels the last moe_plan call enqueued (1 cooperative kernel, or 3)."""
         return self._view().plan_kernels
@@ -195,7 +207,7 @@ class Plan:
             "rcnt": arr(v.rcnt, R), "rank_off": arr(v.rank_off, R + 1),
             "rtok_off": rtok_off, "slot": arr(v.slot, N * k).view(N, k) if N else
             torch.empty((0, k), dtype=torch.int32, device=dev),
-            "src_tok": arr(v.src_tok, N * k), "src_j": arr(v.src_j, N * k),
+            "src_tok": arr(v.src_tok, v.recv_rows), "src_j": arr(v.src_j, v.recv_rows),
             "rtok": arr(v.rtok, n_dedup), "fanout": arr(v.fanout, n_dedup),
             "err": arr(v.err, 1),
         }
@@ -219,9 +231,11 @@ class Plan:
             pass
 
 
-def moe_plan_create(max_tokens: int, k: int, E: int, R: int) -> Plan:
+def moe_plan_create(max_tokens: int, k: int, E: int, R: int, align: int = 1) -> Plan:
+    """Allocate a reusable plan; with align > 1 expert segments start on multiples of it."""
     h = _vp(0)
-    _check(_lib.moe_plan_create(int(max_tokens), int(k), int(E), int(R), ctypes.byref(h)))
+    _check(_lib.moe_plan_create_aligned(int(max_tokens), int(k), int(E), int(R), int(align),
+                                        ctypes.byref(h)))
     return Plan(h.value)
 
 
@@ -252,11 +266,12 @@ def moe_dispatch(x: torch.Tensor, plan: Plan, recv: torch.Tensor | None = None,
     if N != pN:
         raise ValueError(f"x has {N} rows but the plan has {pN} tokens")
     fp8 = x.dtype != torch.bfloat16
+    rows = plan.rows
     if recv is None:
-        recv = torch.empty((N * k, H), dtype=x.dtype, device=x.device)
+        recv = torch.empty((rows, H), dtype=x.dtype, device=x.device)
     _need_cuda(recv, "recv", (x.dtype,), 2)
-    if tuple(recv.shape) != (N * k, H):
-        raise ValueError(f"recv must have shape {(N * k, H)}")
+    if tuple(recv.shape) != (rows, H):
+        raise ValueError(f"recv must have shape {(rows, H)}")
     xs_ptr = rs_ptr = 0
     if fp8:
         if x_scale is None:
@@ -265,10 +280,10 @@ def moe_dispatch(x: torch.Tensor, plan: Plan, recv: torch.Tensor | None = None,
         if tuple(x_scale.shape) != (N, H // 128):
             raise ValueError(f"x_scale must have shape {(N, H // 128)}")
         if recv_scale is None:
-            recv_scale = torch.empty((N * k, H // 128), dtype=torch.float32, device=x.device)
+            recv_scale = torch.empty((rows, H // 128), dtype=torch.float32, device=x.device)
         _need_cuda(recv_scale, "recv_scale", (torch.float32,), 2)
-        if tuple(recv_scale.shape) != (N * k, H // 128):
-            raise ValueError(f"recv_scale must have shape {(N * k, H // 128)}")
+        if tuple(recv_scale.shape) != (rows, H // 128):
+            raise ValueError(f"recv_scale must have shape {(rows, H // 128)}")
         xs_ptr, rs_ptr = x_scale.data_ptr(), recv_scale.data_ptr()
     _check(_lib.moe_dispatch(_vp(x.data_ptr()), MOE_FP8E4M3 if fp8 else MOE_BF16, _vp(xs_ptr),
                              H, plan._h, _vp(recv.data_ptr()), _vp(rs_ptr),
@@ -283,8 +298,8 @@ def moe_combine(y: torch.Tensor, plan: Plan, out: torch.Tensor | None = None, st
     _need_cuda(y, "y", (torch.bfloat16,), 2)
     N, k, _, _ = plan.shape
     rows, H = y.shape
-    if rows != N * k:
-        raise ValueError(f"y must have {N * k} rows (got {rows})")
+    if rows != plan.rows:
+        raise ValueError(f"y must have {plan.rows} rows (got {rows})")
     if out is None:
         out = torch.empty((N, H), dtype=torch.bfloat16, device=y.device)
     _need_cuda(out, "out", (torch.bfloat16,), 2)

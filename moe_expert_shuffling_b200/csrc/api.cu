@@ -142,12 +142,22 @@ moe_status moe_tune(moe_knob knob, int32_t value)
 
 moe_status moe_plan_create(int32_t max_tokens, int32_t k, int32_t E, int32_t R, moe_plan_t *out)
 {
+    return moe_plan_create_aligned(max_tokens, k, E, R, 1, out);
+}
+
+moe_status moe_plan_create_aligned(int32_t max_tokens, int32_t k, int32_t E, int32_t R,
+                                   int32_t align, moe_plan_t *out)
+{
     if (!out)
         return fail(MOE_EINVAL, "out must not be NULL");
     *out = nullptr;
     moe_status st = check_shape(max_tokens, k, E, R);
     if (st != MOE_OK)
         return st;
+    if (align < 1 || align > (1 << 16))
+        return fail(MOE_EINVAL, "align must be in [1, 65536] (got %d)", align);
+    if (moe::recv_rows(max_tokens, k, E, align) >= (int64_t(1) << 31))
+        return fail(MOE_EINVAL, "N*k + E*(align-1) must be < 2^31");
     int dev = 0;
     if ((st = current_device(&dev)) != MOE_OK)
         return st;
@@ -163,7 +173,10 @@ moe_status moe_plan_create(int32_t max_tokens, int32_t k, int32_t E, int32_t R, 
     p->device = dev;
     p->nt_cap = static_cast<int32_t>(moe::ceil_div(max_tokens, moe::kPlanTile));
     p->rtok_cap = static_cast<int64_t>(max_tokens) * (k < R ? k : R);
+    p->align = align;
+    p->rows_cap = moe::recv_rows(max_tokens, k, E, align);
     const int64_t rows = static_cast<int64_t>(max_tokens) * k;
+    const int64_t all_rows = p->rows_cap;
     const int64_t nt = p->nt_cap > 0 ? p->nt_cap : 1;
 
     // One allocation, every array 256-byte aligned.
@@ -177,8 +190,8 @@ moe_status moe_plan_create(int32_t max_tokens, int32_t k, int32_t E, int32_t R, 
         {reinterpret_cast<void **>(&p->rank_off), sizeof(int32_t) * (R + 1)},
         {reinterpret_cast<void **>(&p->rtok_off), sizeof(int32_t) * (R + 1)},
         {reinterpret_cast<void **>(&p->slot), sizeof(int32_t) * (rows > 0 ? rows : 1)},
-        {reinterpret_cast<void **>(&p->src_tok), sizeof(int32_t) * (rows > 0 ? rows : 1)},
-        {reinterpret_cast<void **>(&p->src_j), sizeof(int32_t) * (rows > 0 ? rows : 1)},
+        {reinterpret_cast<void **>(&p->src_tok), sizeof(int32_t) * (all_rows > 0 ? all_rows : 1)},
+        {reinterpret_cast<void **>(&p->src_j), sizeof(int32_t) * (all_rows > 0 ? all_rows : 1)},
         {reinterpret_cast<void **>(&p->rtok), sizeof(int32_t) * (p->rtok_cap > 0 ? p->rtok_cap : 1)},
         {reinterpret_cast<void **>(&p->fanout), sizeof(uint32_t) * (p->rtok_cap > 0 ? p->rtok_cap : 1)},
         {reinterpret_cast<void **>(&p->err), sizeof(uint32_t)},
@@ -297,7 +310,7 @@ moe_status moe_dispatch(const void *x, moe_dtype dtype, const float *x_scale, in
     a.err = p->err;
     a.N = p->N;
     a.k = p->k;
-    a.n_rows = p->N * p->k;
+    a.n_rows = static_cast<int32_t>(moe::recv_rows(p->N, p->k, p->E, p->align));
     a.row_bytes = static_cast<uint32_t>(H) * elem;
     a.srow_bytes = srow;
     cudaError_t e = moe::launch_dispatch(a, p->device, static_cast<cudaStream_t>(stream));
@@ -329,7 +342,7 @@ static moe_status combine_impl(const void *y, int32_t H, moe_plan_t plan, void *
     a.err = p->err;
     a.N = p->N;
     a.k = p->k;
-    a.n_rows = p->N * p->k;
+    a.n_rows = static_cast<int32_t>(moe::recv_rows(p->N, p->k, p->E, p->align));
     a.H = H;
     a.rank_off = p->rank_off;
     a.R = p->R;
@@ -374,6 +387,8 @@ moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *v)
     v->err = p->err;
     v->topk_w = p->topk_w;
     v->plan_kernels = p->plan_kernels;
+    v->align = p->align;
+    v->recv_rows = static_cast<int32_t>(moe::recv_rows(p->N, p->k, p->E, p->align));
     return ok();
 }
 

@@ -11,8 +11,10 @@
 struct moe_plan_s {
     int32_t cap = 0;        // largest N accepted
     int32_t N = 0, k = 0, E = 0, R = 0, epr = 0;
+    int32_t align = 1;      // expert segments start on multiples of this many rows
     int32_t nt_cap = 0;     // tiles for `cap` tokens
     int64_t rtok_cap = 0;   // entries of rtok/fanout: cap * min(k, R)
+    int64_t rows_cap = 0;   // receive rows for `cap` tokens: cap * k + E * (align - 1)
     int device = 0;
     void *mem = nullptr;
     size_t mem_bytes = 0;
@@ -30,6 +32,12 @@ struct moe_plan_s {
 };
 
 namespace moe {
+
+// Receive rows of a plan: N * k entries plus up to align - 1 padding rows per expert.
+inline int64_t recv_rows(int64_t N, int32_t k, int32_t E, int32_t align)
+{
+    return N * k + static_cast<int64_t>(E) * (align - 1);
+}
 
 // Tokens per plan tile (one CTA of the count and rank kernels).
 constexpr int kPlanWarps = 8;
@@ -64,6 +72,7 @@ cudaError_t launch_plan(moe_plan_s *p, const int32_t *topk_idx, cudaStream_t str
 struct PlanArrays {
     const int32_t *topk_idx;
     int32_t N, k, E, R;
+    int32_t align = 1;
     int64_t rtok_cap;
     int32_t *cnt, *expert_off, *rcnt, *rank_off, *rtok_off, *slot, *src_tok, *src_j, *rtok;
     uint32_t *fanout, *err;

@@ -34,7 +34,7 @@ constexpr uint32_t kFull = 0xffffffffu;  // all lanes of a warp
 // Kernel parameters: shape, routing, outputs and scratch.
 struct PlanK {
     const int32_t *topk_idx;
-    int32_t N, k, E, R, epr, nt, n_rows;
+    int32_t N, k, E, R, epr, nt, n_rows, align;
     int64_t rtok_cap;
     int32_t *tile_cnt, *tile_rcnt;
     uint32_t *tile_err;
@@ -84,7 +84,8 @@ __device__ __forceinline__ Entry classify(const int32_t *ids, const int32_t *ran
         if (q < j && iq == id)
             valid = false;
     }
-    c.flags = (present && !in_range ? MOE_ERR_ID_RANGE : 0u) |
+    // -1 marks an entry the router dropped: no row, no contribution, not an error
+    c.flags = (present && !in_range && id != -1 ? MOE_ERR_ID_RANGE : 0u) |
               (in_range && !valid ? MOE_ERR_ID_DUP : 0u);
     c.e = valid ? id : -1;
     c.r = valid ? rank_of[id] : -1;
@@ -259,10 +260,19 @@ __device__ void count_tile(const PlanK &p, const PlanSmem &m, int tile, uint32_t
 
 // Segment starts from the totals; block 0 publishes them.  All threads must call.
 // Both totals arrays are staged in shared memory with their loads in flight together.
+// Segment sizes are the counts rounded up to the alignment.  Also marks every receive
+// row that no entry maps to (segment padding and rows after the last segment) with -1
+// in src_tok/src_j, spread over all CTAs of the grid.
 __device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_sums)
 {
-    for (int i = threadIdx.x; i < p.E + p.R; i += blockDim.x)
-        m.ebase[i] = i < p.E ? __ldcg(p.cnt + i) : __ldcg(p.rcnt + (i - p.E));  // ebase|rbase
+    for (int i = threadIdx.x; i < p.E + p.R; i += blockDim.x) {
+        if (i < p.E) {
+            const int32_t c = __ldcg(p.cnt + i);
+            m.ebase[i] = (c + p.align - 1) / p.align * p.align;
+        } else {
+            m.rbase[i - p.E] = __ldcg(p.rcnt + (i - p.E));
+        }
+    }
     __syncthreads();
     scan_into(m.ebase, p.E, m.eoff, warp_sums);
     scan_into(m.rbase, p.R, m.roff, warp_sums);
@@ -274,6 +284,20 @@ __device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_su
             p.rtok_off[i] = m.roff[i];
             p.rank_off[i] = m.eoff[i * p.epr];
         }
+    }
+    if (p.align > 1) {
+        for (int e = blockIdx.x; e < p.E; e += gridDim.x) {
+            const int32_t first = m.eoff[e] + __ldcg(p.cnt + e);
+            for (int32_t r = first + threadIdx.x; r < m.eoff[e + 1]; r += blockDim.x) {
+                p.src_tok[r] = -1;
+                p.src_j[r] = -1;
+            }
+        }
+    }
+    for (int64_t r = m.eoff[p.E] + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+         r < p.n_rows; r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        p.src_tok[r] = -1;
+        p.src_j[r] = -1;
     }
 }
 
@@ -543,7 +567,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
 }
 
 PlanK make_params(const int32_t *topk_idx, int32_t N, int32_t k, int32_t E, int32_t R,
-                  int64_t rtok_cap)
+                  int32_t align, int64_t rtok_cap)
 {
     PlanK p{};
     p.topk_idx = topk_idx;
@@ -553,7 +577,8 @@ PlanK make_params(const int32_t *topk_idx, int32_t N, int32_t k, int32_t E, int3
     p.R = R;
     p.epr = E / R;
     p.nt = static_cast<int32_t>(ceil_div(N, kPlanTile));
-    p.n_rows = N * k;
+    p.align = align;
+    p.n_rows = static_cast<int32_t>(recv_rows(N, k, E, align));
     p.rtok_cap = rtok_cap;
     return p;
 }
@@ -594,7 +619,7 @@ cudaError_t launch_plan(moe_plan_s *pl, const int32_t *topk_idx, cudaStream_t st
 {
     if (!ensure_attrs(pl->device))
         return cudaGetLastError() != cudaSuccess ? cudaGetLastError() : cudaErrorUnknown;
-    PlanK p = make_params(topk_idx, pl->N, pl->k, pl->E, pl->R, pl->rtok_cap);
+    PlanK p = make_params(topk_idx, pl->N, pl->k, pl->E, pl->R, pl->align, pl->rtok_cap);
     p.tile_cnt = pl->tile_cnt;
     p.tile_rcnt = pl->tile_rcnt;
     p.tile_err = pl->tile_err;
@@ -647,7 +672,7 @@ cudaError_t launch_plan_arrays(const PlanArrays &a, cudaStream_t stream)
         return e;
     if (!ensure_attrs(dev))
         return cudaGetLastError() != cudaSuccess ? cudaGetLastError() : cudaErrorUnknown;
-    PlanK p = make_params(a.topk_idx, a.N, a.k, a.E, a.R, a.rtok_cap);
+    PlanK p = make_params(a.topk_idx, a.N, a.k, a.E, a.R, a.align, a.rtok_cap);
     p.tile_cnt = a.tile_cnt;
     p.tile_rcnt = a.tile_rcnt;
     p.tile_err = a.tile_err;

@@ -14,6 +14,7 @@ from tests.shuffle_cases import (
     assert_combine_close, assert_plan_equal, bits16, bits_to_f32, gpu_plan, make_inputs,
     plan_to_host,
 )
+from tests.test_oracle_plan import drop_some
 from workloads import CONFIGS
 
 pytestmark = pytest.mark.gpu
@@ -268,3 +269,60 @@ def test_side_stream():
     s.synchronize()
     ref = oracle.plan(idx, cfg.E, cfg.R)
     assert np.array_equal(bits16(out), oracle.combine(bits16(y), ref.slot, w))
+
+
+@pytest.mark.parametrize("name,N,frac,align", [
+    ("tiny", 128, 0.2, 1), ("tiny", 300, 0.3, 8), ("dsv3", 2000, 0.1, 128),
+    ("long", 3000, 0.05, 64), ("mixtral", 2000, 0.5, 16), ("dsv3", 700, 1.0, 4),
+    ("dsv3_k32", 300, 0.2, 32),
+])
+def test_dropped_and_aligned_parity(name, N, frac, align):
+    """Dropped entries (id -1) and aligned expert segments match the oracle bit for bit."""
+    import moe_expert_shuffling_b200 as ms
+    cfg = CONFIGS[name].with_tokens(N)
+    idx, w, x, xs, _ = make_inputs(cfg, 5, y=False)
+    idx = drop_some(idx, frac, 13)
+    ref = oracle.plan(idx, cfg.E, cfg.R, align=align)
+    p = ms.moe_plan_create(N, cfg.k, cfg.E, cfg.R, align=align)
+    p, ti, tw = gpu_plan(idx, w, cfg.E, cfg.R, plan=p)
+    assert p.rows == ref.rows and p.align == align
+    got = plan_to_host(p)
+    for name_ in ("cnt", "expert_off", "rcnt", "rank_off", "rtok_off", "slot", "src_tok",
+                  "src_j", "rtok"):
+        assert np.array_equal(got[name_], getattr(ref, name_)), name_
+    assert np.array_equal(got["fanout"], ref.fanout)
+    assert int(got["err"][0]) == 0                       # drops are not errors
+    used = ref.src_tok >= 0
+    if cfg.payload == "fp8":
+        recv, rs = ms.moe_dispatch(x, p, x_scale=xs)
+        ref_recv, ref_rs = oracle.dispatch(x.cpu().numpy(), ref.slot, xs.cpu().numpy(), rows=ref.rows)
+        assert np.array_equal(rs.cpu().numpy().view(np.uint8)[used], ref_rs[used])
+        got_recv = recv.cpu().numpy()
+    else:
+        recv = ms.moe_dispatch(x, p)
+        ref_recv = oracle.dispatch(bits16(x).view(np.uint8).reshape(N, -1), ref.slot, rows=ref.rows)
+        got_recv = bits16(recv).view(np.uint8).reshape(ref.rows, -1)
+    assert np.array_equal(got_recv[used], ref_recv[used])
+    g = torch.Generator(device="cuda")
+    g.manual_seed(21)
+    y = torch.randn((ref.rows, cfg.H), generator=g, device="cuda").to(torch.bfloat16)
+    out = ms.moe_combine(y, p)
+    out_r = ms.moe_combine(y, p, ranked=True)
+    assert p.check() == 0
+    yb = bits16(y)
+    assert np.array_equal(bits16(out), oracle.combine(yb, ref.slot, w))
+    assert np.array_equal(bits16(out_r), oracle.combine_ranked(yb, ref.slot, w, idx, cfg.E, cfg.R))
+
+
+def test_drops_alone_raise_no_error():
+    import moe_expert_shuffling_b200 as ms
+    idx = -np.ones((257, 4), np.int32)
+    w = np.full((257, 4), 0.25, np.float32)
+    p, ti, tw = gpu_plan(idx, w, 16, 4)
+    x = torch.randn((257, 64), device="cuda").to(torch.bfloat16)
+    recv = ms.moe_dispatch(x, p)
+    out = ms.moe_combine(recv, p)
+    assert p.check() == 0
+    assert not bits16(out).any()              # nothing routed: out is +0
+    a = plan_to_host(p)
+    assert np.all(a["slot"] == -1) and np.all(a["src_tok"] == -1) and a["cnt"].sum() == 0

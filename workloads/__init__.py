@@ -12,8 +12,10 @@ from .gen import (  # noqa: F401
     Workload,
     ZIPF_ALPHA,
     distinct_rank_expectation,
+    drop_entries,
     find_zipf_alpha,
     make_payload_x,
+    make_expert_outputs,
     make_payload_y,
     make_routing,
     make_workload,

@@ -213,6 +213,19 @@ def make_payload_y(cfg: Config, seed: int, device="cpu"):
     return _randn_bf16(cfg.N * cfg.k, cfg.H, _stream_seed(seed, 2), device)
 
 
+def make_expert_outputs(rows: int, H: int, seed: int, device="cpu") -> torch.Tensor:
+    """bf16 [rows, H] ~ N(0,1): expert outputs for a receive layout of `rows` rows."""
+    return _randn_bf16(rows, H, _stream_seed(seed, 2), device)
+
+
+def drop_entries(topk_idx: np.ndarray, frac: float, seed: int) -> np.ndarray:
+    """Mark a seeded fraction of the routing entries as dropped (id -1)."""
+    out = topk_idx.copy()
+    rng = np.random.Generator(np.random.PCG64(_stream_seed(seed, 3)))
+    out[rng.random(out.shape) < frac] = -1
+    return out
+
+
 def make_workload(cfg: Config, seed: int = 0, device="cpu", with_y: bool = True) -> Workload:
     idx, w = make_routing(cfg, seed)
     x, xs = make_payload_x(cfg, seed, device)
