@@ -384,6 +384,98 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
+def run_micro_batches(args):
+    """The batch split into M micro-batches.  Without --overlap they run one after the
+    other; with it, dispatch of micro-batch m runs on a second stream while micro-batch
+    m-1 combines (concurrent dispatch and combine, ordered by events)."""
+    import moe_expert_shuffling_b200 as ms
+    from moe_expert_shuffling_b200 import build as lib_build
+
+    lib_build.build()
+    world, rank, local = dist_setup(args)
+    cfg = CONFIGS[args.config]
+    if args.tokens > 0:
+        cfg = cfg.with_tokens(args.tokens)
+    if cfg.payload != "bf16" or cfg.y == "identity":
+        raise SystemExit("micro-batch mode takes a bf16 workload with independent expert outputs")
+    seed = rank_seed(args.seed, rank)
+    dev = torch.device("cuda", local)
+    sa, sb = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    idx_h, w_h = make_routing(cfg, seed)
+    with torch.cuda.stream(sa):
+        x, _ = make_payload_x(cfg, seed, dev)
+        y = make_payload_y(cfg, seed, dev)
+        idx = torch.from_numpy(idx_h).to(dev)
+        w = torch.from_numpy(w_h).to(dev)
+        out = torch.empty((cfg.N, cfg.H), dtype=torch.bfloat16, device=dev)
+    sa.synchronize()
+    M = args.micro_batches
+    cuts = [cfg.N * m // M for m in range(M + 1)]
+    mbs = []
+    for m in range(M):
+        a, b = cuts[m], cuts[m + 1]
+        mbs.append(dict(idx=idx[a:b], w=w[a:b], x=x[a:b], y=y[a * cfg.k:b * cfg.k],
+                        out=out[a:b], plan=ms.moe_plan_create(b - a, cfg.k, cfg.E, cfg.R),
+                        recv=torch.empty(((b - a) * cfg.k, cfg.H), dtype=x.dtype, device=dev)))
+
+    def step(e0=None, e1=None):
+        if e0 is not None:
+            e0.record(sa)
+        for mb in mbs:
+            ms.moe_plan(mb["idx"], mb["w"], cfg.E, cfg.R, plan=mb["plan"], stream=sa)
+        ms.moe_dispatch(mbs[0]["x"], mbs[0]["plan"], recv=mbs[0]["recv"], stream=sa)
+        for m in range(1, M):
+            if args.overlap:
+                ready = torch.cuda.Event()
+                ready.record(sa)
+                sb.wait_event(ready)
+                ms.moe_dispatch(mbs[m]["x"], mbs[m]["plan"], recv=mbs[m]["recv"], stream=sb)
+                done = torch.cuda.Event()
+                done.record(sb)
+            else:
+                ms.moe_dispatch(mbs[m]["x"], mbs[m]["plan"], recv=mbs[m]["recv"], stream=sa)
+            ms.moe_combine(mbs[m - 1]["y"], mbs[m - 1]["plan"], out=mbs[m - 1]["out"], stream=sa)
+            if args.overlap:
+                sa.wait_event(done)
+        ms.moe_combine(mbs[-1]["y"], mbs[-1]["plan"], out=mbs[-1]["out"], stream=sa)
+        if e1 is not None:
+            e1.record(sa)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    step(e0, None)
+    for _ in range(args.steps - 2):
+        step()
+    step(None, e1)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    el = max_over_ranks(e0.elapsed_time(e1), world)
+    nbytes = dispatch_bytes(cfg) + combine_bytes(cfg)
+    value = job_throughput(nbytes, args.steps, world, el)
+    for mb in mbs:
+        assert mb["plan"].check(sa) == 0
+        mb["plan"].close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": workload_name(cfg) + f", {M} micro-batches"
+                   + (", dispatch of each overlapping the previous combine" if args.overlap
+                      else ", one after the other")},
+        "pct_roofline": {"of_nominal_8000": round(100 * value / world / NOMINAL_HBM_GBS, 2)},
+        "gpu_launches": (3 * M) * args.steps,
+    }), flush=True)
+
+
 # ------------------------------------------------------------------------ CPU oracle
 def oracle_sample_step(cfg: Config, idx_h, w_h, x_bytes, xs_bytes, y_bits, n):
     """One oracle plan + dispatch + combine over the first n tokens of the workload."""
@@ -489,6 +581,10 @@ def main(argv=None):
                     help="start every expert segment on a multiple of this many rows")
     ap.add_argument("--drop", type=float, default=0.0,
                     help="fraction of routing entries marked dropped (id -1), seeded")
+    ap.add_argument("--micro-batches", type=int, default=1,
+                    help="split each step's batch into this many micro-batches")
+    ap.add_argument("--overlap", action="store_true",
+                    help="with micro-batches: dispatch of one overlaps combine of the previous")
     ap.add_argument("--combine", default="chain", choices=["chain", "ranked"],
                     help="combine order: one fma chain per token, or grouped by rank first")
     ap.add_argument("--seed", type=int, default=0)
@@ -500,6 +596,8 @@ def main(argv=None):
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.micro_batches > 1:
+        run_micro_batches(args)
     else:
         run_ours(args)
 
