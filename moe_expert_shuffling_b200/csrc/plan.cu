@@ -5,7 +5,8 @@
 // local address -- slot[t, j] is that map.
 //
 // Three phases, all deterministic (no result depends on thread timing):
-//   count  per tile of 128 tokens: expert counts and counts of (token, rank) moves
+//   count  per tile of 128 tokens: classify the entries, mark each token in 128-bit
+//          per-expert and per-rank tile masks; the counts are their popcounts
 //          -> scratch [E][tiles], [R][tiles], plus the tile's error flags
 //   scan   per expert row and per rank row: exclusive scan over tiles, row totals
 //          -> cnt[E], rcnt[R]; the tile flags are gathered into the error word
@@ -218,48 +219,67 @@ __device__ void load_ids(const PlanK &p, const PlanSmem &m, int tile, int ntok)
         m.ids[i] = __ldg(src + i);
 }
 
-// Count phase for one tile.  All threads must call; rank_of must be ready.
-__device__ void count_tile(const PlanK &p, const PlanSmem &m, int tile, uint32_t *s_err)
+// Classify a tile's entries into shared memory: vid/lead per entry, and each token's bit
+// in its experts' and ranks' tile masks.  All threads must call; rank_of must be ready.
+// Returns this thread's MOE_ERR_* flags.
+__device__ uint32_t classify_tile(const PlanK &p, const PlanSmem &m, int tile, int ntok)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int ntok = tile_tokens(p, tile);
-    int32_t *hist = m.ebase, *rhist = m.rbase;
-    for (int i = threadIdx.x; i < p.E + p.R; i += blockDim.x)
-        hist[i] = 0;  // ebase and rbase are contiguous
+    const int k = p.k;
+    for (int i = threadIdx.x; i < 4 * (p.E + p.R); i += blockDim.x)
+        m.emask[i] = 0u;  // emask and rmask are contiguous
     load_ids(p, m, tile, ntok);
-    if (threadIdx.x == 0)
-        *s_err = 0;
     __syncthreads();
-
-    const LaneMap lm = lane_map(p.k);
+    const LaneMap lm = lane_map(k);
     const int j = lane & ((1 << lm.wbits) - 1);
     const int sub = lane >> lm.wbits;
     uint32_t flags = 0;
     for (int st = 0; st < lm.steps; ++st) {
         const int tw = st * lm.per_step + sub;           // token within the warp's 16
         const int tl = warp * kPlanTokensPerWarp + tw;
-        const bool present = tw < kPlanTokensPerWarp && tl < ntok && j < p.k;
-        const Entry c = classify(m.ids, m.rank_of, tl, j, present, p.k, p.E, 1 << lm.wbits);
+        const bool present = tw < kPlanTokensPerWarp && tl < ntok && j < k;
+        const Entry c = classify(m.ids, m.rank_of, tl, j, present, k, p.E, 1 << lm.wbits);
         flags |= c.flags;
-        if (c.e >= 0)
-            atomicAdd(&hist[c.e], 1);
-        if (c.lead)
-            atomicAdd(&rhist[c.r], 1);
+        if (present) {
+            m.vid[tl * k + j] = c.e;
+            m.lead[tl * k + j] = c.lead;
+            const uint32_t bit = 1u << (tl & 31);
+            if (c.e >= 0)
+                atomicOr(&m.emask[4 * c.e + (tl >> 5)], bit);
+            if (c.lead)
+                atomicOr(&m.rmask[4 * c.r + (tl >> 5)], bit);
+        }
     }
+    __syncthreads();
+    return flags;
+}
+
+// Count phase for one tile: the tile's count per expert (per rank) is the number of its
+// tokens on it, the popcount of the tile mask.  Leaves the tile's classification in
+// shared memory.  All threads must call; rank_of must be ready.
+__device__ void count_tile(const PlanK &p, const PlanSmem &m, int tile, uint32_t *s_err)
+{
+    if (threadIdx.x == 0)
+        *s_err = 0;
+    const uint32_t flags = classify_tile(p, m, tile, tile_tokens(p, tile));
     if (flags)
         atomicOr(s_err, flags);
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+        const uint32_t *mk = &m.emask[4 * e];
+        p.tile_cnt[static_cast<int64_t>(e) * p.nt + tile] =
+            __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+    }
+    for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
+        const uint32_t *mk = &m.rmask[4 * r];
+        p.tile_rcnt[static_cast<int64_t>(r) * p.nt + tile] =
+            __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+    }
     __syncthreads();
-    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
-        p.tile_cnt[static_cast<int64_t>(e) * p.nt + tile] = hist[e];
-    for (int r = threadIdx.x; r < p.R; r += blockDim.x)
-        p.tile_rcnt[static_cast<int64_t>(r) * p.nt + tile] = rhist[r];
     if (threadIdx.x == 0)
         p.tile_err[tile] = *s_err;
     __syncthreads();
 }
 
-// Segment starts from the totals; block 0 publishes them.  All threads must call.
-// Both totals arrays are staged in shared memory with their loads in flight together.
 // Segment sizes are the counts rounded up to the alignment.  Also marks every receive
 // row that no entry maps to (segment padding and rows after the last segment) with -1
 // in src_tok/src_j, spread over all CTAs of the grid.
@@ -302,18 +322,17 @@ __device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_su
 }
 
 // Rank phase for one tile.  All threads must call; rank_prepare must have run.  With
-// ids_ready the tile's ids are already in shared memory.
-__device__ void rank_tile(const PlanK &p, const PlanSmem &m, int tile, bool ids_ready)
+// tile_ready the tile's classification (count_tile of this tile) is still in shared
+// memory; otherwise it is rebuilt.
+__device__ void rank_tile(const PlanK &p, const PlanSmem &m, int tile, bool tile_ready)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int ntok = tile_tokens(p, tile);
     if (ntok == 0)
         return;  // block-uniform
     const int k = p.k;
-    for (int i = threadIdx.x; i < 4 * (p.E + p.R); i += blockDim.x)
-        m.emask[i] = 0u;  // emask and rmask are contiguous
-    if (!ids_ready)
-        load_ids(p, m, tile, ntok);
+    if (!tile_ready)
+        (void)classify_tile(p, m, tile, ntok);  // flags were reported by the count phase
     // This tile's first receive row per expert and first dedup entry per rank.
     for (int e = threadIdx.x; e < p.E; e += blockDim.x)
         m.ebase[e] = m.eoff[e] + __ldcg(p.tile_cnt + static_cast<int64_t>(e) * p.nt + tile);
@@ -321,28 +340,10 @@ __device__ void rank_tile(const PlanK &p, const PlanSmem &m, int tile, bool ids_
         m.rbase[r] = m.roff[r] + __ldcg(p.tile_rcnt + static_cast<int64_t>(r) * p.nt + tile);
     __syncthreads();
 
-    // Pass A: classify, and mark each token in its expert's and rank's tile mask.
+    // Stable rank = tile base + earlier tokens of the tile on the same expert.
     const LaneMap lm = lane_map(k);
     const int j = lane & ((1 << lm.wbits) - 1);
     const int sub = lane >> lm.wbits;
-    for (int st = 0; st < lm.steps; ++st) {
-        const int tw = st * lm.per_step + sub;
-        const int tl = warp * kPlanTokensPerWarp + tw;
-        const bool present = tw < kPlanTokensPerWarp && tl < ntok && j < k;
-        const Entry c = classify(m.ids, m.rank_of, tl, j, present, k, p.E, 1 << lm.wbits);
-        if (present) {
-            m.vid[tl * k + j] = c.e;
-            m.lead[tl * k + j] = c.lead;
-            const uint32_t bit = 1u << (tl & 31);
-            if (c.e >= 0)
-                atomicOr(&m.emask[4 * c.e + (tl >> 5)], bit);
-            if (c.lead)
-                atomicOr(&m.rmask[4 * c.r + (tl >> 5)], bit);
-        }
-    }
-    __syncthreads();
-
-    // Pass B: stable rank = tile base + earlier tokens of the tile on the same expert.
     const int64_t t0 = static_cast<int64_t>(tile) * kPlanTile;
     uint32_t flags = 0;
     for (int st = 0; st < lm.steps; ++st) {
@@ -560,7 +561,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
     }
 
     rank_prepare(p, m, warp_sums);
-    const bool one_tile = static_cast<int>(G) >= p.nt;  // ids of the tile are still in smem
+    // With one tile per CTA the count phase left that tile's classification in smem.
+    const bool one_tile = static_cast<int>(G) >= p.nt;
     for (int tile = blockIdx.x; tile < p.nt; tile += G)
         rank_tile(p, m, tile, one_tile);
     grid_depart(p);
