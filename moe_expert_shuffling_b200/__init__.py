@@ -156,6 +156,13 @@ class Plan:
     def __init__(self, handle: int):
         self._h = _vp(handle)
         self._refs = ()
+        self._meta = None  # (N, k, E, R, rows) of the last plan, cached for the hot calls
+
+    def _cached(self):
+        if self._meta is None:
+            v = self._view()
+            self._meta = (v.N, v.k, v.E, v.R, v.recv_rows)
+        return self._meta
 
     @property
     def handle(self) -> int:
@@ -168,8 +175,7 @@ class Plan:
 
     @property
     def shape(self) -> tuple[int, int, int, int]:
-        v = self._view()
-        return v.N, v.k, v.E, v.R
+        return self._cached()[:4]
 
     @property
     def capacity(self) -> int:
@@ -178,7 +184,7 @@ class Plan:
     @property
     def rows(self) -> int:
         """Rows a receive buffer needs for the last plan: N*k + E*(align - 1)."""
-        return self._view().recv_rows
+        return self._cached()[4]
 
     @property
     def align(self) -> int:
@@ -253,6 +259,8 @@ def moe_plan(topk_idx: torch.Tensor, topk_w: torch.Tensor, E: int, R: int,
     if plan is None:
         plan = Plan(h.value)
     plan._refs = (topk_idx, topk_w)
+    if plan._meta is None or plan._meta[0] != N:
+        plan._meta = None
     return plan
 
 

@@ -2,6 +2,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 
@@ -107,6 +108,76 @@ int sm_count(int device)
         cache[device] = n;
     }
     return cache[device];
+}
+
+int max_smem_optin(int device)
+{
+    static int cache[64] = {0};
+    if (device < 0 || device >= 64)
+        return 0;
+    if (cache[device] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) !=
+                cudaSuccess ||
+            v <= 0)
+            v = 48 * 1024;
+        cache[device] = v;
+    }
+    return cache[device];
+}
+
+namespace {
+struct FitEntry {
+    const void *kernel;
+    int device, threads;
+    size_t smem;
+    int per_sm;
+};
+struct LimitEntry {
+    const void *kernel;
+    int device;
+    size_t smem;
+};
+std::mutex g_fit_mu;
+FitEntry g_fit[128];
+int g_fit_n = 0;
+LimitEntry g_limit[64];
+int g_limit_n = 0;
+}  // namespace
+
+cudaError_t kernel_fit(const void *kernel, int device, int threads, size_t smem, int *per_sm)
+{
+    std::lock_guard<std::mutex> lock(g_fit_mu);
+    for (int i = 0; i < g_fit_n; ++i) {
+        const FitEntry &f = g_fit[i];
+        if (f.kernel == kernel && f.device == device && f.threads == threads && f.smem == smem) {
+            *per_sm = f.per_sm;
+            return cudaSuccess;
+        }
+    }
+    // raise the kernel's dynamic-shared-memory limit if this size needs more
+    int li = -1;
+    for (int i = 0; i < g_limit_n; ++i)
+        if (g_limit[i].kernel == kernel && g_limit[i].device == device)
+            li = i;
+    if (smem > 48 * 1024 && (li < 0 || g_limit[li].smem < smem)) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess)
+            return e;
+        if (li < 0 && g_limit_n < 64)
+            li = g_limit_n++;
+        if (li >= 0)
+            g_limit[li] = LimitEntry{kernel, device, smem};
+    }
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem);
+    if (e != cudaSuccess)
+        return e;
+    if (g_fit_n < 128)
+        g_fit[g_fit_n++] = FitEntry{kernel, device, threads, smem, n};
+    *per_sm = n;
+    return cudaSuccess;
 }
 
 }  // namespace moe

@@ -406,7 +406,7 @@ cudaError_t launch_one(const CombineParams &p, int device, int ctas_per_sm, cuda
     auto kern = combine_lsu_kernel<KB, VPL>;
     int per_sm = 0;
     cudaError_t e =
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCombineThreads, 0);
+        kernel_fit(reinterpret_cast<const void *>(kern), device, kCombineThreads, 0, &per_sm);
     if (e != cudaSuccess)
         return e;
     per_sm = std::max(per_sm, 1);
@@ -451,11 +451,8 @@ cudaError_t launch_bulk_shape(const CombineArgs &a, int device, cudaStream_t str
     p.nchunks = static_cast<uint32_t>(ceil_div(p.row_bytes, chunk));
     p.stage_bytes = static_cast<uint32_t>(a.k) * chunk;
 
-    int max_optin = 0;
-    cudaError_t e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
-                                           device);
-    if (e != cudaSuccess)
-        return e;
+    const int max_optin = max_smem_optin(device);
+    cudaError_t e = cudaSuccess;
     // Several CTAs per SM (more consumer warps) beat one CTA with a deeper ring.
     const int budget = tu.combine_smem_kb > 0 ? std::min(tu.combine_smem_kb * 1024, max_optin)
                                               : std::min(kDefaultSmemBudget, max_optin);
@@ -478,12 +475,8 @@ cudaError_t launch_bulk_shape(const CombineArgs &a, int device, cudaStream_t str
     p.ring_bytes = static_cast<uint32_t>(S) * p.stage_bytes;
     const size_t smem = smem_for(S);
     auto kern = combine_bulk_kernel<KMAX, CW, RANKED>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess)
-        return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+    e = kernel_fit(reinterpret_cast<const void *>(kern), device, threads, smem, &per_sm);
     if (e != cudaSuccess)
         return e;
     if (per_sm < 1)

@@ -178,11 +178,8 @@ cudaError_t launch_dispatch(const DispatchArgs &a, int device, cudaStream_t stre
     const uint32_t stage_bytes =
         static_cast<uint32_t>(round_up(scale_off + (bulk_scales ? a.srow_bytes : 0u), 128));
 
-    int max_optin = 0;
-    cudaError_t e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
-                                           device);
-    if (e != cudaSuccess)
-        return e;
+    const int max_optin = max_smem_optin(device);
+    cudaError_t e = cudaSuccess;
     auto smem_for = [&](int st) {
         return static_cast<size_t>(round_up(static_cast<int64_t>(wpc) * st * 8, 128)) +
                static_cast<size_t>(wpc) * st * stage_bytes;
@@ -196,13 +193,9 @@ cudaError_t launch_dispatch(const DispatchArgs &a, int device, cudaStream_t stre
     lag = std::min(lag, stages - 1);
     const size_t smem = smem_for(stages);
 
-    e = cudaFuncSetAttribute(dispatch_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess)
-        return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_bulk_kernel, wpc * 32,
-                                                      smem);
+    e = kernel_fit(reinterpret_cast<const void *>(dispatch_bulk_kernel), device, wpc * 32, smem,
+                   &per_sm);
     if (e != cudaSuccess)
         return e;
     if (per_sm < 1)

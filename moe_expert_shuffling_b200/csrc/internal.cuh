@@ -65,6 +65,14 @@ Tuning &tuning();
 
 int sm_count(int device);
 
+// Largest dynamic shared memory a CTA may opt into on `device` (cached).
+int max_smem_optin(int device);
+
+// Resident CTAs per SM of `kernel` with `threads` threads and `smem` bytes of dynamic shared
+// memory on `device`, raising the kernel's dynamic-shared-memory limit when needed.  Cached
+// per (kernel, device, threads, smem) so that repeated launches make no runtime queries.
+cudaError_t kernel_fit(const void *kernel, int device, int threads, size_t smem, int *per_sm);
+
 cudaError_t launch_plan(moe_plan_s *p, const int32_t *topk_idx, cudaStream_t stream);
 
 // The planner's kernels on explicit arrays (for callers that own every buffer).  The

@@ -650,8 +650,8 @@ cudaError_t launch_plan(moe_plan_s *pl, const int32_t *topk_idx, cudaStream_t st
         const size_t smem = sizeof(int32_t) * plan_smem_words(p.E, p.R, p.k);
         int per_sm = 0;
         if (coop[dev] > 0 &&
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_fused_kernel,
-                                                          kPlanThreads, smem) == cudaSuccess &&
+            kernel_fit(reinterpret_cast<const void *>(plan_fused_kernel), pl->device,
+                       kPlanThreads, smem, &per_sm) == cudaSuccess &&
             per_sm > 0) {
             const int64_t fit = static_cast<int64_t>(sm_count(pl->device)) * per_sm;
             const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(p.nt, fit)));
