@@ -269,8 +269,9 @@ def run_ours(args):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     graph = None
     if args.graph:
-        # one whole step (plan, dispatch, combine) captured once and replayed: no host work
-        # per step; the per-kernel times then come from an event-timed pass of the same steps
+        # One whole step (plan, dispatch, combine) captured once and replayed: no host work
+        # per step.  The per-kernel times come from an event-timed pass of the same steps on
+        # the same stream just before the timed replays.
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream):
             step()
@@ -605,8 +606,10 @@ def main(argv=None):
                     help="start every expert segment on a multiple of this many rows")
     ap.add_argument("--drop", type=float, default=0.0,
                     help="fraction of routing entries marked dropped (id -1), seeded")
-    ap.add_argument("--graph", action="store_true",
-                    help="capture one step in a CUDA graph and replay it (no per-step host work)")
+    ap.add_argument("--graph", dest="graph", action="store_true", default=True,
+                    help="capture one step in a CUDA graph and replay it (default)")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch every step from the host on a stream instead")
     ap.add_argument("--micro-batches", type=int, default=1,
                     help="split each step's batch into this many micro-batches")
     ap.add_argument("--overlap", action="store_true",
