@@ -214,7 +214,8 @@ MOE_API moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *view);
 
 /*
  * moe_plan_check -- wait for `stream`, then copy the plan's error word to *flags
- * (MOE_ERR_* bits; 0 = the routing was valid and every wait finished).
+ * (MOE_ERR_* bits; 0 = the routing was valid and every wait finished).  After a reported
+ * MOE_ERR_TIMEOUT it also rearms the plan's grid-barrier words.
  */
 MOE_API moe_status moe_plan_check(moe_plan_t plan, void *stream, uint32_t *flags);
 

@@ -473,6 +473,12 @@ moe_status moe_plan_check(moe_plan_t plan, void *stream, uint32_t *flags)
     e = cudaMemcpy(flags, plan->err, sizeof(uint32_t), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaMemcpy(err)");
+    if (*flags & MOE_ERR_TIMEOUT) {
+        // a grid barrier was abandoned: rearm its words for the next plan
+        e = cudaMemset(plan->sync, 0, 2 * sizeof(uint32_t));
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaMemset(sync)");
+    }
     return ok();
 }
 

@@ -14,7 +14,8 @@
 //          as a popcount over a per-expert bitmask of the tile's tokens (bit t set when
 //          token t selects the expert), so no step is sequential.
 // By default the phases run in one cooperative kernel (plan_fused_kernel) whose CTAs
-// meet at two grid barriers; a barrier gives up after 1 s and reports MOE_ERR_TIMEOUT.
+// meet at two sense-reversing grid barriers; a wait gives up after 1 s and reports
+// MOE_ERR_TIMEOUT.
 // When the grid cannot be co-resident the phases run as three kernels instead.
 //
 // Inside a tile a warp looks at several tokens at once: lane = (token, column) with the
@@ -41,7 +42,7 @@ struct PlanK {
     uint32_t *tile_err;
     int32_t *cnt, *expert_off, *rcnt, *rank_off, *rtok_off, *slot, *src_tok, *src_j, *rtok;
     uint32_t *fanout, *err;
-    uint32_t *sync;  // [2] grid-barrier arrivals and departures (fused kernel), zero at rest
+    uint32_t *sync;  // [2] grid-barrier arrival count (zero at rest) and generation
 };
 
 // Classification of one entry, shared by the count and rank kernels so both see the
@@ -449,43 +450,49 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *a)
     return v;
 }
 
-// Grid barrier for a co-resident grid: arrivals count up to `target`.  Gives up after
-// kWaitLimitNs, sets MOE_ERR_TIMEOUT and returns false.  All threads must call.
-__device__ bool grid_barrier(const PlanK &p, uint32_t target, int *s_ok)
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t *a, uint32_t v)
+{
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(a), "r"(v)
+                 : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t *a, uint32_t v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+
+// Sense-reversing grid barrier for a co-resident grid.  sync[0] counts arrivals; the last
+// CTA to arrive sets it back to 0 and advances the generation word sync[1], which the
+// others wait on, so the words are ready for the next barrier (and the next launch) with no
+// extra step.  A wait gives up after kWaitLimitNs, sets MOE_ERR_TIMEOUT and returns false.
+// All threads must call.
+__device__ bool grid_barrier(const PlanK &p, int *s_ok)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(&p.sync[0], 1u);
+        const uint32_t gen = ld_acquire_gpu(&p.sync[1]);
         bool ok = true;
-        const uint64_t t0 = global_timer_ns();
-        for (uint32_t it = 0; ld_acquire_gpu(&p.sync[0]) < target; ++it) {
-            if ((it & 15u) == 15u && (global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30))) {
-                atomicOr(p.err, MOE_ERR_TIMEOUT);
-                ok = false;
-                break;
+        if (atom_add_acq_rel_gpu(&p.sync[0], 1u) == gridDim.x - 1u) {
+            p.sync[0] = 0u;                // no CTA reads the count until the next barrier
+            st_release_gpu(&p.sync[1], gen + 1u);
+        } else {
+            const uint64_t t0 = global_timer_ns();
+            for (uint32_t it = 0; ld_acquire_gpu(&p.sync[1]) == gen; ++it) {
+                if ((it & 15u) == 15u &&
+                    (global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30))) {
+                    atomicOr(p.err, MOE_ERR_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+                __nanosleep(32);
             }
-            __nanosleep(64);
         }
-        __threadfence();
         *s_ok = ok;
     }
     __syncthreads();
     return *s_ok != 0;
-}
-
-// The last CTA to leave resets the barrier words for the next launch.
-__device__ void grid_depart(const PlanK &p)
-{
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        if (atomicAdd(&p.sync[1], 1u) == gridDim.x - 1u) {
-            p.sync[0] = 0u;
-            p.sync[1] = 0u;
-            __threadfence();
-        }
-    }
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
@@ -501,10 +508,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
     init_rank_of(p, m);
     for (int tile = blockIdx.x; tile < p.nt; tile += G)
         count_tile(p, m, tile, &s_err);
-    if (!grid_barrier(p, G, &s_ok)) {
-        grid_depart(p);
+    if (!grid_barrier(p, &s_ok))
         return;
-    }
 
     // Scan phase: one warp per expert row / rank row, in coalesced rounds of 32 tiles;
     // each group of up to 16 rounds is loaded before any of it is scanned.
@@ -555,17 +560,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
         if (lane == 0)
             *p.err = f;
     }
-    if (!grid_barrier(p, 2u * G, &s_ok)) {
-        grid_depart(p);
+    if (!grid_barrier(p, &s_ok))
         return;
-    }
 
     rank_prepare(p, m, warp_sums);
     // With one tile per CTA the count phase left that tile's classification in smem.
     const bool one_tile = static_cast<int>(G) >= p.nt;
     for (int tile = blockIdx.x; tile < p.nt; tile += G)
         rank_tile(p, m, tile, one_tile);
-    grid_depart(p);
 }
 
 PlanK make_params(const int32_t *topk_idx, int32_t N, int32_t k, int32_t E, int32_t R,
