@@ -468,11 +468,12 @@ __device__ __forceinline__ void st_release_gpu(uint32_t *a, uint32_t v)
 // others wait on, so the words are ready for the next barrier (and the next launch) with no
 // extra step.  A wait gives up after kWaitLimitNs, sets MOE_ERR_TIMEOUT and returns false.
 // All threads must call.
-__device__ bool grid_barrier(const PlanK &p, int *s_ok)
+// `gen` is the generation read (by thread 0) before this CTA's phase began: it cannot
+// advance until this CTA arrives, and reading it early takes a round trip off the barrier.
+__device__ bool grid_barrier(const PlanK &p, uint32_t gen, int *s_ok)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
-        const uint32_t gen = ld_acquire_gpu(&p.sync[1]);
         bool ok = true;
         if (atom_add_acq_rel_gpu(&p.sync[0], 1u) == gridDim.x - 1u) {
             p.sync[0] = 0u;                // no CTA reads the count until the next barrier
@@ -505,11 +506,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
     const uint32_t G = gridDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
+    uint32_t gen = threadIdx.x == 0 ? ld_acquire_gpu(&p.sync[1]) : 0u;
     init_rank_of(p, m);
     for (int tile = blockIdx.x; tile < p.nt; tile += G)
         count_tile(p, m, tile, &s_err);
-    if (!grid_barrier(p, &s_ok))
+    if (!grid_barrier(p, gen, &s_ok))
         return;
+    gen += 1u;  // the generation the next barrier starts from
 
     // Scan phase: one warp per expert row / rank row, in coalesced rounds of 32 tiles;
     // each group of up to 16 rounds is loaded before any of it is scanned.
@@ -560,7 +563,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
         if (lane == 0)
             *p.err = f;
     }
-    if (!grid_barrier(p, &s_ok))
+    if (!grid_barrier(p, gen, &s_ok))
         return;
 
     rank_prepare(p, m, warp_sums);
