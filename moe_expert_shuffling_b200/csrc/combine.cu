@@ -153,15 +153,45 @@ struct CombineBulkParams {
     uint32_t ring_bytes;    // bytes of the stage ring (the rank tables follow it)
 };
 
+constexpr int32_t kNoRank = 0x7fffffff;
+
+// Rank of receive row s: the r with roff[r] <= s < roff[r + 1] (rows are grouped by rank).
+__device__ __forceinline__ int32_t rank_of_row(const int32_t *roff, int R, int32_t s)
+{
+    int lo = 0, hi = R;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (roff[mid] <= s)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+// Position of this lane's column in the token's (rank, column) order, lanes j < k holding
+// column j with rank rj (kNoRank for a dropped column, which sorts after every kept one).
+__device__ __forceinline__ int rank_order_pos(int32_t rj, int k, int lane)
+{
+    int pos = 0;
+    for (int q = 0; q < k; ++q) {
+        const int32_t rq = __shfl_sync(0xffffffffu, rj, q);
+        pos += (rq < rj || (rq == rj && q < lane)) ? 1 : 0;
+    }
+    return pos;
+}
+
 // RANKED: the rank-grouped order -- per rank (ascending) an fp32 fma chain over the
 // token's columns on that rank (ascending), and the partials added in ascending rank
-// order; otherwise one fma chain over the columns in order.
+// order; otherwise one fma chain over the columns in order.  In the ranked order the
+// producer puts the token's kept rows into the stage already sorted by (rank, column), so
+// the consumers read rows at fixed offsets and carry only the sorted weights and a bitmask
+// of the positions where a new rank starts.
 template <int KMAX, int CW, bool RANKED>
 __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
     combine_bulk_kernel(const CombineBulkParams p)
 {
     constexpr uint32_t kChunk_ = Shape<CW>::kChunk;
-    constexpr int32_t kNoRank = 0x7fffffff;
     extern __shared__ __align__(128) uint8_t smem[];
     const int S = static_cast<int>(p.stages);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
@@ -169,16 +199,29 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
     uint8_t *ring = smem + p.bar_bytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int k = p.k;
-    // rank-grouped order: rank offsets, then per consumer warp the token's columns sorted
-    // by (rank, column) with their weights and ranks
+    // rank-grouped order: the rank offsets, then per consumer warp the token's weights and
+    // ranks in (rank, column) order
     int32_t *roff_s = reinterpret_cast<int32_t *>(ring + p.ring_bytes);
-    int32_t *ord_s = roff_s + (RANKED ? p.R + 1 : 0) + (warp > 0 ? (warp - 1) * 96 : 0);
-    float *wo_s = reinterpret_cast<float *>(ord_s + 32);
-    int32_t *ro_s = ord_s + 64;
+    float *wo_s = reinterpret_cast<float *>(roff_s + (RANKED ? p.R + 1 : 0) +
+                                            (warp > 0 ? (warp - 1) * 64 : 0));
+    int32_t *ro_s = reinterpret_cast<int32_t *>(wo_s + 32);
+
+    const uint32_t b = blockIdx.x * p.per_cta;  // this CTA's first token
+    const int n_tok = b < static_cast<uint32_t>(p.N)
+                          ? static_cast<int>(min(p.per_cta, static_cast<uint32_t>(p.N) - b))
+                          : 0;
+    // the first token's slots (and, for the consumers, weights) are fetched before the
+    // barrier so that their latency overlaps the set-up
+    int32_t s_first = -1;
+    float w_first = 0.f;
+    if (n_tok > 0 && lane < k) {
+        s_first = __ldg(p.slot + static_cast<int64_t>(b) * k + lane);
+        if (warp > 0)
+            w_first = __ldg(p.w + static_cast<int64_t>(b) * k + lane);
+    }
     if (RANKED)
         for (int i = threadIdx.x; i <= p.R; i += blockDim.x)
             roff_s[i] = __ldg(p.rank_off + i);
-
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
@@ -188,14 +231,9 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
     }
     __syncthreads();
 
-    const uint32_t b = blockIdx.x * p.per_cta;  // this CTA's first token
-    const int n_tok = b < static_cast<uint32_t>(p.N)
-                          ? static_cast<int>(min(p.per_cta, static_cast<uint32_t>(p.N) - b))
-                          : 0;
-
     if (warp == 0) {
         // ---------------- producer: lane j < k copies row slot[t, j]
-        int32_t s_cur = (n_tok > 0 && lane < k) ? __ldg(p.slot + static_cast<int64_t>(b) * k + lane) : -1;
+        int32_t s_cur = s_first;
         int i = 0;
         bool ok = true;
         for (int m = 0; m < n_tok && ok; ++m) {
@@ -206,6 +244,11 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
             const bool valid =
                 lane < k && static_cast<uint32_t>(s_cur) < static_cast<uint32_t>(p.n_rows);
             const uint32_t nv = __popc(__ballot_sync(0xffffffffu, valid));
+            uint32_t dst = static_cast<uint32_t>(lane) * kChunk_;
+            if (RANKED)
+                dst = static_cast<uint32_t>(rank_order_pos(
+                          valid ? rank_of_row(roff_s, p.R, s_cur) : kNoRank, k, lane)) *
+                      kChunk_;
             for (uint32_t c = 0; c < p.nchunks; ++c, ++i) {
                 const int st = i % S;
                 const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
@@ -219,7 +262,7 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
                     mbar_arrive_expect_tx(&full[st], nv * len);
                 __syncwarp();
                 if (valid)
-                    bulk_load(ring + static_cast<size_t>(st) * p.stage_bytes + lane * kChunk_,
+                    bulk_load(ring + static_cast<size_t>(st) * p.stage_bytes + dst,
                               p.y + static_cast<int64_t>(s_cur) * p.row_bytes + off, len,
                               &full[st]);
             }
@@ -239,62 +282,39 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
     // A token's valid columns (bitmask) and weights are broadcast once per token and kept
     // in registers; each chunk then costs k shared loads, 8k fmas and one 16-byte store.
     const uint32_t v16 = static_cast<uint32_t>(threadIdx.x - 32) * 16u;
-    int32_t s_nxt = -1;
-    float w_nxt = 0.f;
-    if (n_tok > 0 && lane < k) {
-        s_nxt = __ldg(p.slot + static_cast<int64_t>(b) * k + lane);
-        w_nxt = __ldg(p.w + static_cast<int64_t>(b) * k + lane);
-    }
+    int32_t s_nxt = s_first;
+    float w_nxt = w_first;
     int i = 0;
     for (int m = 0; m < n_tok; ++m) {
         const uint32_t t = b + static_cast<uint32_t>(m);
         const uint32_t vmask = __ballot_sync(
             0xffffffffu,
             lane < k && static_cast<uint32_t>(s_nxt) < static_cast<uint32_t>(p.n_rows));
-        float wv[RANKED ? 1 : KMAX];
-        constexpr int KR = (RANKED && KMAX <= 8) ? KMAX : 1;
-        int32_t ordr[KR], ror[KR];
-        float wor[KR];
+        float wv[KMAX];
+        uint32_t nv = 0, starts = 0;  // ranked: kept columns; positions opening a new rank
         if (!RANKED) {
 #pragma unroll
-            for (int j = 0; j < (RANKED ? 1 : KMAX); ++j)
+            for (int j = 0; j < KMAX; ++j)
                 wv[j] = __shfl_sync(0xffffffffu, w_nxt, j);
         } else {
-            // rank of each column from the plan's rank offsets, then its position in the
-            // (rank, column) order
-            int32_t rj = kNoRank;
-            if ((vmask >> lane) & 1u) {
-                int lo = 0, hi = p.R;  // roff_s[lo] <= slot < roff_s[hi]
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (roff_s[mid] <= s_nxt)
-                        lo = mid;
-                    else
-                        hi = mid;
-                }
-                rj = lo;
-            }
-            int pos = 0;
-            for (int q = 0; q < k; ++q) {
-                const int32_t rq = __shfl_sync(0xffffffffu, rj, q);
-                pos += (rq < rj || (rq == rj && q < lane)) ? 1 : 0;
-            }
+            nv = __popc(vmask);
+            const int32_t rj =
+                ((vmask >> lane) & 1u) ? rank_of_row(roff_s, p.R, s_nxt) : kNoRank;
+            const int pos = rank_order_pos(rj, k, lane);
             __syncwarp();
             if (lane < k) {
-                ord_s[pos] = lane;
                 wo_s[pos] = w_nxt;
                 ro_s[pos] = rj;
             }
             __syncwarp();
-            if (KMAX <= 8) {
-                // small k: keep the token's order in registers for all of its chunks
+            const float w_sorted = lane < k ? wo_s[lane] : 0.f;
+            const int32_t r_sorted = lane < k ? ro_s[lane] : kNoRank;
+            const int32_t r_before = __shfl_up_sync(0xffffffffu, r_sorted, 1);
+            starts = __ballot_sync(0xffffffffu, lane > 0 && static_cast<uint32_t>(lane) < nv &&
+                                                    r_sorted != r_before);
 #pragma unroll
-                for (int pq = 0; pq < (KMAX <= 8 ? KMAX : 1); ++pq) {
-                    ordr[pq] = pq < k ? ord_s[pq] : 0;
-                    wor[pq] = pq < k ? wo_s[pq] : 0.f;
-                    ror[pq] = pq < k ? ro_s[pq] : kNoRank;
-                }
-            }
+            for (int j = 0; j < KMAX; ++j)
+                wv[j] = __shfl_sync(0xffffffffu, w_sorted, j);
         }
         if (m + 1 < n_tok && lane < k) {
             s_nxt = __ldg(p.slot + static_cast<int64_t>(t + 1) * k + lane);
@@ -312,57 +332,12 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
             const uint32_t len = min(kChunk_, p.row_bytes - off);
             const uint8_t *stage = ring + static_cast<size_t>(st) * p.stage_bytes + v16;
             const bool mine = v16 < len;
-            float acc[8];
+            float acc[8], part[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
+            for (int e = 0; e < 8; ++e) {
                 acc[e] = 0.f;
-            if (RANKED) {
-                float part[8];
-                int32_t prev = -1;  // rank of the open partial
-#pragma unroll
-                for (int p0 = 0; p0 < KMAX; p0 += 8) {
-                    if (p0 >= k)
-                        break;  // warp-uniform
-                    uint4 q[8];
-#pragma unroll
-                    for (int pp = 0; pp < 8; ++pp) {
-                        const int pq = p0 + pp;
-                        const int32_t rr = KMAX <= 8 ? ror[pp] : (pq < k ? ro_s[pq] : kNoRank);
-                        const int32_t jr = KMAX <= 8 ? ordr[pp] : ord_s[pq < k ? pq : 0];
-                        q[pp] = (mine && rr != kNoRank) ? lds_v4(stage + jr * kChunk_)
-                                                        : make_uint4(0u, 0u, 0u, 0u);
-                    }
-                    if (p0 + 8 >= k) {
-                        __syncwarp();
-                        if (lane == 0)
-                            mbar_arrive(&empty[st]);
-                    }
-#pragma unroll
-                    for (int pp = 0; pp < 8; ++pp) {
-                        const int pq = p0 + pp;
-                        const int32_t rr = KMAX <= 8 ? ror[pp] : (pq < k ? ro_s[pq] : kNoRank);
-                        if (rr == kNoRank)
-                            continue;
-                        if (rr != prev) {
-                            if (prev >= 0) {
-#pragma unroll
-                                for (int e = 0; e < 8; ++e)
-                                    acc[e] = __fadd_rn(acc[e], part[e]);
-                            }
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                part[e] = 0.f;
-                            prev = rr;
-                        }
-                        fma_bf16x8(part, KMAX <= 8 ? wor[pp] : wo_s[pq], q[pp]);
-                    }
-                }
-                if (prev >= 0) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        acc[e] = __fadd_rn(acc[e], part[e]);
-                }
-            } else {
+                part[e] = 0.f;
+            }
 #pragma unroll
             for (int j0 = 0; j0 < KMAX; j0 += 8) {
                 if (j0 >= k)
@@ -371,8 +346,9 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
                     const int j = j0 + jj;
-                    q[jj] = (mine && ((vmask >> j) & 1u)) ? lds_v4(stage + j * kChunk_)
-                                                          : make_uint4(0u, 0u, 0u, 0u);
+                    const bool kept = RANKED ? static_cast<uint32_t>(j) < nv : ((vmask >> j) & 1u);
+                    q[jj] = (mine && kept) ? lds_v4(stage + j * kChunk_)
+                                           : make_uint4(0u, 0u, 0u, 0u);
                 }
                 if (j0 + 8 >= k) {
                     // every row of this stage is in registers: release it to the producer
@@ -383,10 +359,27 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
                     const int j = j0 + jj;
-                    if ((vmask >> j) & 1u)
-                        fma_bf16x8(acc, wv[RANKED ? 0 : j], q[jj]);
+                    if (RANKED) {
+                        if (static_cast<uint32_t>(j) >= nv)
+                            continue;
+                        if ((starts >> j) & 1u) {
+                            // close the previous rank's chain
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                acc[e] = __fadd_rn(acc[e], part[e]);
+                                part[e] = 0.f;
+                            }
+                        }
+                        fma_bf16x8(part, wv[j], q[jj]);
+                    } else if ((vmask >> j) & 1u) {
+                        fma_bf16x8(acc, wv[j], q[jj]);
+                    }
                 }
             }
+            if (RANKED && nv > 0) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    acc[e] = __fadd_rn(acc[e], part[e]);
             }
             if (mine)
                 st_stream_v4(p.out + static_cast<int64_t>(t) * p.row_bytes + off + v16,
@@ -460,13 +453,14 @@ cudaError_t launch_bulk_shape(const CombineArgs &a, int device, cudaStream_t str
     S = std::min(S, kMaxBulkStages);
     p.rank_off = a.rank_off;
     p.R = a.R;
-    // rank-grouped order: the rank offsets plus 96 words per consumer warp
-    const size_t tables = RANKED ? sizeof(int32_t) * (static_cast<size_t>(a.R) + 1 + 96 * CW) : 0;
+    // rank-grouped order: the rank offsets plus 64 words per consumer warp
+    const size_t tables = RANKED ? sizeof(int32_t) * (static_cast<size_t>(a.R) + 1 + 64 * CW) : 0;
     auto smem_for = [&](int st) {
         return static_cast<size_t>(round_up(2 * st * 8, 128)) +
                static_cast<size_t>(st) * p.stage_bytes + tables;
     };
-    while (S > 2 && smem_for(S) > static_cast<size_t>(budget))
+    // the budget is for the ring; the ranked order's tables come on top of it
+    while (S > 2 && smem_for(S) - tables > static_cast<size_t>(budget))
         --S;
     if (smem_for(S) > static_cast<size_t>(max_optin))
         return cudaErrorInvalidValue;
