@@ -65,6 +65,26 @@ def plan_bytes(cfg: Config, N: int | None = None) -> int:
     return 4 * N * cfg.k * 4 + 8 * N * min(cfg.k, cfg.R)
 
 
+L2_BYTES = 126 * 2**20
+
+
+def l2_note(cfg: Config) -> str:
+    """How the timed steps avoid L2 reuse (no flush kernel runs between steps)."""
+    mb = lambda b: f"{b / 2**20:.0f} MB"
+    bufs = [("x", cfg.N * cfg.row_bytes), ("recv", cfg.N * cfg.k * cfg.row_bytes)]
+    if cfg.y != "identity":
+        bufs.append(("y", cfg.N * cfg.k * cfg.H * 2))
+    bufs.append(("out", cfg.N * cfg.H * 2))
+    sizes = ", ".join(f"{n} {mb(b)}" for n, b in bufs)
+    small = [n for n, b in bufs if b <= L2_BYTES]
+    if not small:
+        return f"no flush: every buffer of the step is larger than the 126 MB L2 ({sizes})"
+    total = sum(b for _, b in bufs)
+    return (f"no flush: {', '.join(small)} fit in the 126 MB L2, but one step touches "
+            f"{mb(total)} ({sizes}), {total / L2_BYTES:.1f}x the L2, so little of it "
+            "survives to the next step")
+
+
 def workload_name(cfg: Config) -> str:
     return (f"{cfg.name}: N={cfg.N} H={cfg.H} E={cfg.E} k={cfg.k} R={cfg.R} "
             f"{cfg.payload} routing={cfg.routing} weights={cfg.weights} experts={cfg.y}")
@@ -387,7 +407,7 @@ def run_ours(args):
                    "model": f"{cfg.name}-shaped MoE layer shuffle",
                    "global_batch": cfg.N * world, "seq_len": cfg.N, "parallelism": f"replicas{world}",
                    "ep_ranks_logical": cfg.R,
-                   "l2": "no flush: every input (x, y) and output is larger than the 126 MB L2",
+                   "l2": l2_note(cfg),
                    "launch": "CUDA graph of one step, replayed" if args.graph else "stream"},
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_roofline": {"of_nominal_8000": round(100 * value / world / NOMINAL_HBM_GBS, 2),
