@@ -123,6 +123,42 @@ def kernel_traffic(kernel: str, cfg: Config):
     return rec["bytes_per_unit"] * units
 
 
+def pct_stats(ms_list):
+    """median / p10 / p90 of event times given in ms, reported in us."""
+    v = sorted(1e3 * t for t in ms_list)
+    q = lambda f: v[min(len(v) - 1, int(round(f * (len(v) - 1))))]
+    return {"median": round(statistics.median(v), 2), "p10": round(q(0.1), 2),
+            "p90": round(q(0.9), 2), "n": len(v)}
+
+
+def flushed_kernel_times(step, stream, dev, iters):
+    """Each of plan, dispatch and combine timed alone (CUDA events on the launching stream),
+    each launch preceded by an L2 flush.  The flush READS a buffer of twice the L2 size: that
+    writes back and evicts whatever the previous kernel left dirty and leaves only clean,
+    unrelated lines, so the timed kernel neither hits in L2 nor pays for another's
+    write-back."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    with torch.cuda.stream(stream):
+        scratch = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev)
+        sink = torch.empty((), dtype=torch.float32, device=dev)
+    times = {"plan": [], "dispatch": [], "combine": []}
+    for it in range(iters + 3):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        with torch.cuda.stream(stream):
+            for phase in range(3):
+                torch.sum(scratch, out=sink)
+                ev[2 * phase].record(stream)
+                step(phase_only=phase)
+                ev[2 * phase + 1].record(stream)
+        stream.synchronize()
+        if it >= 3:  # warm-up
+            for phase, name in enumerate(("plan", "dispatch", "combine")):
+                times[name].append(ev[2 * phase].elapsed_time(ev[2 * phase + 1]))
+    out = {name: pct_stats(t) for name, t in times.items()}
+    out["flush"] = f"read of a {2 * l2 >> 20} MB buffer before each launch"
+    return out
+
+
 # ---------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -263,20 +299,24 @@ def run_ours(args):
     identity = y is None
     plan = ms.moe_plan_create(cfg.N, cfg.k, cfg.E, cfg.R, align=args.align)
 
-    def step(ev=None):
+    def step(ev=None, phase_only=None):
+        """One step: plan, dispatch, combine (phase_only = 0, 1 or 2 runs just that one)."""
         if ev is not None:
             ev[0].record(stream)
-        ms.moe_plan(idx, w, cfg.E, cfg.R, plan=plan, stream=stream)
+        if phase_only in (None, 0):
+            ms.moe_plan(idx, w, cfg.E, cfg.R, plan=plan, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        if rs is not None:
-            ms.moe_dispatch(x, plan, recv=recv, x_scale=xs, recv_scale=rs, stream=stream)
-        else:
-            ms.moe_dispatch(x, plan, recv=recv, stream=stream)
+        if phase_only in (None, 1):
+            if rs is not None:
+                ms.moe_dispatch(x, plan, recv=recv, x_scale=xs, recv_scale=rs, stream=stream)
+            else:
+                ms.moe_dispatch(x, plan, recv=recv, stream=stream)
         if ev is not None:
             ev[2].record(stream)
-        ms.moe_combine(recv if identity else y, plan, out=out, stream=stream,
-                       ranked=args.combine == "ranked")
+        if phase_only in (None, 2):
+            ms.moe_combine(recv if identity else y, plan, out=out, stream=stream,
+                           ranked=args.combine == "ranked")
         if ev is not None:
             ev[3].record(stream)
 
@@ -384,6 +424,13 @@ def run_ours(args):
                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(e_ms / args.e2e_steps, 3), "steps": args.e2e_steps}
 
+    # each kernel alone after an L2 flush (outside the timed region)
+    flushed = None
+    if args.flushed_iters > 0:
+        flushed = flushed_kernel_times(step, stream, dev, args.flushed_iters)
+        for name, nbytes in (("dispatch", db), ("combine", cb), ("plan", plan_bytes(cfg))):
+            flushed[name]["gbs_at_median"] = round(nbytes / (flushed[name]["median"] * 1e-6) / 1e9, 1)
+
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
         cpu = cpu_baseline(cfg, idx_h, w_h, x, xs, y, recv, args.cpu_seconds)
@@ -414,6 +461,10 @@ def run_ours(args):
                          f"of_{peak_kind}_{peak:g}": round(100 * value / world / peak, 2)},
         "kernels_us": {"plan": round(plan_us, 2), "dispatch": round(disp_us, 2),
                        "combine": round(comb_us, 2)},
+        "kernels_unflushed_us": {"note": "back-to-back steps on one stream, no flush",
+                                 "plan": pct_stats(t_plan), "dispatch": pct_stats(t_disp),
+                                 "combine": pct_stats(t_comb)},
+        "kernels_flushed_us": flushed,
         "kernels_gbs": {"dispatch": round(db / (disp_us * 1e-6) / 1e9, 1),
                         "combine": round(cb / (comb_us * 1e-6) / 1e9, 1),
                         "plan": round(plan_bytes(cfg) / (plan_us * 1e-6) / 1e9, 1)},
@@ -565,7 +616,33 @@ def cpu_baseline(cfg, idx_h, w_h, x, xs, y, recv, seconds):
     gbs = (dispatch_bytes(cfg, n) + combine_bytes(cfg, n)) * reps / total_t / 1e9
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"first {n} of {cfg.N} tokens (same routing and payload), {reps} "
-                      f"plan+dispatch+combine passes, {total_t:.1f} s, single-threaded C"}
+                      f"plan+dispatch+combine passes, {total_t:.1f} s, single-threaded C",
+            "all_cores": cpu_baseline_omp(cfg, idx_h, w_h, xb, xsb, yb, n_max, seconds / 2)}
+
+
+def cpu_baseline_omp(cfg, idx_h, w_h, xb, xsb, yb, n_max, seconds):
+    """The same oracle source built with -fopenmp (dispatch and combine token loops on all
+    host cores; the plan stays sequential), on the same kind of sample."""
+    import oracle
+    from oracle import build as oracle_build
+    cores = len(os.sched_getaffinity(0))
+    with oracle.using_library(oracle_build.build_omp()):
+        n = min(256, n_max)
+        t0 = time.perf_counter()
+        oracle_sample_step(cfg, idx_h, w_h, xb, xsb, yb, n)
+        dt = time.perf_counter() - t0
+        n = int(max(16, min(n_max, n * (seconds / 3) / max(dt, 1e-6))))
+        reps, total_t = 0, 0.0
+        while total_t < seconds * 0.66 and reps < 50:
+            t0 = time.perf_counter()
+            oracle_sample_step(cfg, idx_h, w_h, xb, xsb, yb, n)
+            total_t += time.perf_counter() - t0
+            reps += 1
+    gbs = (dispatch_bytes(cfg, n) + combine_bytes(cfg, n)) * reps / total_t / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle built with -fopenmp",
+            "sample": f"first {n} of {cfg.N} tokens, {reps} passes, {total_t:.1f} s, "
+                      f"OMP_NUM_THREADS={os.environ.get('OMP_NUM_THREADS', 'unset (all cores)')}"}
 
 
 def run_reference(args):
@@ -636,6 +713,8 @@ def main(argv=None):
                     help="with micro-batches: dispatch of one overlaps combine of the previous")
     ap.add_argument("--combine", default="chain", choices=["chain", "ranked"],
                     help="combine order: one fma chain per token, or grouped by rank first")
+    ap.add_argument("--flushed-iters", type=int, default=50,
+                    help="iterations of each kernel timed alone after an L2 flush (0: skip)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -35,6 +35,12 @@
  * error); other ids are distinct within a token and in [0, E) -- anything else is
  * rejected with ORACLE_EINVAL.  Build: gcc -O2 -ffp-contract=off (no contraction, so
  * every fma below is the only fused operation).
+ *
+ * The token loops of dispatch and combine carry an OpenMP pragma.  The oracle build
+ * ignores it (no -fopenmp); a second build with -fopenmp (liboracle_omp.so) exists only
+ * so the benchmark can also report the oracle's time on all host cores.  Each iteration
+ * writes rows no other iteration writes (slots are distinct; out row t belongs to token
+ * t), so both builds give identical bytes.
  */
 #include <math.h>
 #include <stdint.h>
@@ -203,6 +209,7 @@ void oracle_dispatch(const uint8_t *x, const uint8_t *x_scale, const int32_t *sl
                      int64_t N, int32_t k, int64_t row_bytes, int64_t scale_bytes,
                      uint8_t *recv, uint8_t *recv_scale)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < N; ++t)
         for (int32_t j = 0; j < k; ++j) {
             int64_t s = slot[t * k + j];
@@ -239,6 +246,7 @@ static uint16_t f32_to_bf16_rne(float f)
 void oracle_combine(const uint16_t *y, const int32_t *slot, const float *w, int64_t N,
                     int32_t k, int64_t H, uint16_t *out)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < N; ++t)
         for (int64_t c = 0; c < H; ++c) {
             float acc = 0.0f;

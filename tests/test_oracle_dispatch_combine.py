@@ -386,3 +386,23 @@ def test_dispatch_and_combine_skip_dropped_entries():
     ref_two = oracle.combine(yb, np.ascontiguousarray(sl2[:, :2]), np.ascontiguousarray(w2[:, :2]))
     assert np.array_equal(out[keep], ref_full[keep])
     assert np.array_equal(out[~keep], ref_two[~keep])
+
+
+def test_openmp_build_gives_the_same_bytes():
+    """The -fopenmp build (used only for the multi-core CPU baseline) must compute exactly
+    what the oracle computes: its parallel token loops write disjoint rows."""
+    from oracle import build as oracle_build
+    cfg = CONFIGS["dsv3"].with_tokens(96)
+    idx, w = make_routing(cfg, 3)
+    x, _ = make_payload_x(cfg, 3, "cpu")
+    y = make_payload_y(cfg, 3, "cpu")
+    xb = x.contiguous().view(torch.int16).numpy().view(np.uint8).reshape(cfg.N, -1)
+    yb = y.contiguous().view(torch.int16).numpy().view(np.uint16)
+    p = oracle.plan(idx, cfg.E, cfg.R)
+    recv = oracle.dispatch(xb, p.slot)
+    out = oracle.combine(yb, p.slot, w)
+    with oracle.using_library(oracle_build.build_omp()):
+        recv_omp = oracle.dispatch(xb, p.slot)
+        out_omp = oracle.combine(yb, p.slot, w)
+    assert np.array_equal(recv, recv_omp)
+    assert np.array_equal(out, out_omp)
