@@ -137,7 +137,7 @@ def flushed_kernel_times(step, stream, dev, iters):
     writes back and evicts whatever the previous kernel left dirty and leaves only clean,
     unrelated lines, so the timed kernel neither hits in L2 nor pays for another's
     write-back."""
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or L2_BYTES
     with torch.cuda.stream(stream):
         scratch = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev)
         sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -146,7 +146,7 @@ def flushed_kernel_times(step, stream, dev, iters):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
         with torch.cuda.stream(stream):
             for phase in range(3):
-                torch.sum(scratch, out=sink)
+                torch.sum(scratch, dim=0, out=sink)
                 ev[2 * phase].record(stream)
                 step(phase_only=phase)
                 ev[2 * phase + 1].record(stream)
