@@ -100,10 +100,12 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_traffic(kernel: str, cfg: Config):
+def kernel_traffic(kernel: str, cfg: Config, dropped: bool = False):
     """DRAM bytes per launch from the committed ncu summary: the captured bytes per token
-    scaled to this launch's tokens, if the capture was of this row shape and the kernel's
-    sources are unchanged since; else None."""
+    scaled to this launch's tokens, if the capture was of this row shape, with every entry
+    routed, and the kernel's sources are unchanged since; else None."""
+    if dropped:
+        return None
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
@@ -471,7 +473,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": kernel_traffic(dom, cfg)},
+                     "traffic": kernel_traffic(dom, cfg, dropped=args.drop > 0)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "e2e": e2e,
