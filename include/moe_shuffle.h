@@ -209,6 +209,32 @@ MOE_API moe_status moe_plan_noalloc(const int32_t *topk_idx, int32_t N, int32_t 
 MOE_API moe_status moe_combine_ranked(const void *y, int32_t H, moe_plan_t plan, void *out,
                                       void *stream);
 
+/*
+ * moe_dispatch_combine -- one dispatch and one combine in a single persistent launch, the
+ * single-GPU form of DySHARP's token-centric kernel fusion (DySHARP blog, section 6:
+ * Dispatch and Combine of different tokens run at the same time inside one kernel, each
+ * token's work starting as soon as its inputs are ready).  The results are exactly those of
+ *   moe_dispatch(x, dtype, x_scale, H_x, dispatch_plan, recv, recv_scale) and
+ *   moe_combine(y, H_y, combine_plan, out)   (moe_combine_ranked when ranked != 0).
+ * The two plans may differ (e.g. dispatch of micro-batch m+1 while micro-batch m combines).
+ *
+ * If y == recv (same plan, bf16, H_x == H_y), the combine reads the rows this call
+ * dispatches: token t is combined only after its own rows have been written (per-token
+ * ready flags in the plan; no other synchronisation is needed).  Otherwise y and recv must
+ * not overlap (MOE_EINVAL).
+ *
+ * Arguments are those of moe_dispatch and moe_combine.  fp8 rows need H_x % 512 == 0 (scale
+ * rows of a multiple of 16 bytes).  The launch is cooperative; calls that use the same
+ * dispatch_plan must be ordered on the GPU (one stream, or events): the plan holds the
+ * launch's work counters and flags.  A device wait that runs out (MOE_ERR_TIMEOUT in the
+ * plans' error words) leaves the outputs incomplete; moe_plan_check then rearms the plan.
+ */
+MOE_API moe_status moe_dispatch_combine(const void *x, moe_dtype dtype, const float *x_scale,
+                                        int32_t H_x, moe_plan_t dispatch_plan, void *recv,
+                                        float *recv_scale, const void *y, int32_t H_y,
+                                        moe_plan_t combine_plan, void *out, int32_t ranked,
+                                        void *stream);
+
 /* moe_plan_query -- fill *view with the plan's shape and device pointers. */
 MOE_API moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *view);
 
@@ -243,7 +269,12 @@ typedef enum {
     MOE_TUNE_COMBINE_SMEM_KB = 8,        /* bulk combine: shared-memory budget per CTA (KB) */
     MOE_TUNE_DISPATCH_UNITS_PER_WARP = 9, /* (token, chunk) units per dispatch warp */
     MOE_TUNE_COMBINE_TOKENS_PER_CTA = 10, /* tokens per bulk-combine CTA */
-    MOE_TUNE_PLAN_ENGINE = 11            /* 0 or 1: one cooperative plan kernel, 2: three kernels */
+    MOE_TUNE_PLAN_ENGINE = 11,           /* 0 or 1: one cooperative plan kernel, 2: three kernels */
+    MOE_TUNE_FUSED_CTAS_PER_SM = 12,     /* moe_dispatch_combine: resident CTAs per SM */
+    MOE_TUNE_FUSED_DISPATCH_SHARE = 13,  /* moe_dispatch_combine: % of CTAs that start on dispatch */
+    MOE_TUNE_FUSED_DISPATCH_RUN = 14,    /* moe_dispatch_combine: tokens per dispatch work item (1..32) */
+    MOE_TUNE_FUSED_COMBINE_RUN = 15,     /* moe_dispatch_combine: tokens per combine work item */
+    MOE_TUNE_FUSED_SMEM_KB = 16          /* moe_dispatch_combine: shared memory per CTA (KB) */
 } moe_knob;
 
 MOE_API moe_status moe_tune(moe_knob knob, int32_t value);

@@ -20,6 +20,7 @@ import torch
 
 __all__ = [
     "MoeError", "Plan", "moe_plan", "moe_plan_create", "moe_dispatch", "moe_combine",
+    "moe_dispatch_combine",
     "moe_tune", "lib_path", "version", "ERR_ID_RANGE", "ERR_ID_DUP", "ERR_BOUNDS",
     "ERR_TIMEOUT", "KNOBS",
 ]
@@ -35,6 +36,8 @@ KNOBS = {
     "dispatch_warps_per_cta": 3, "combine_vec_per_lane": 4, "combine_ctas_per_sm": 5,
     "combine_stages": 6, "combine_engine": 7, "combine_smem_kb": 8,
     "dispatch_units_per_warp": 9, "combine_tokens_per_cta": 10, "plan_engine": 11,
+    "fused_ctas_per_sm": 12, "fused_dispatch_share": 13, "fused_dispatch_run": 14,
+    "fused_combine_run": 15, "fused_smem_kb": 16,
 }
 
 _i32 = ctypes.c_int32
@@ -70,6 +73,9 @@ def _load():
     lib.moe_combine.argtypes = [_vp, _i32, _vp, _vp, _vp]
     lib.moe_combine_ranked.restype = st
     lib.moe_combine_ranked.argtypes = [_vp, _i32, _vp, _vp, _vp]
+    lib.moe_dispatch_combine.restype = st
+    lib.moe_dispatch_combine.argtypes = [_vp, ctypes.c_int, _vp, _i32, _vp, _vp, _vp, _vp, _i32,
+                                         _vp, _vp, _i32, _vp]
     lib.moe_plan_query.restype = st
     lib.moe_plan_query.argtypes = [_vp, ctypes.POINTER(_PlanView)]
     lib.moe_plan_check.restype = st
@@ -316,3 +322,50 @@ def moe_combine(y: torch.Tensor, plan: Plan, out: torch.Tensor | None = None, st
     fn = _lib.moe_combine_ranked if ranked else _lib.moe_combine
     _check(fn(_vp(y.data_ptr()), H, plan._h, _vp(out.data_ptr()), _vp(_stream_ptr(stream))))
     return out
+
+
+def moe_dispatch_combine(x: torch.Tensor, dispatch_plan: Plan, recv: torch.Tensor,
+                         y: torch.Tensor, combine_plan: Plan, out: torch.Tensor | None = None,
+                         x_scale: torch.Tensor | None = None,
+                         recv_scale: torch.Tensor | None = None, ranked: bool = False,
+                         stream=None):
+    """moe_dispatch(x, dispatch_plan, recv) and moe_combine(y, combine_plan, out) in one
+    launch.  Pass y=recv (with one plan) to combine the rows this call dispatches.
+    Returns out (and recv_scale for fp8 rows)."""
+    _need_cuda(x, "x", (torch.bfloat16, torch.uint8, torch.float8_e4m3fn), 2)
+    _need_cuda(y, "y", (torch.bfloat16,), 2)
+    N, H = x.shape
+    if N != dispatch_plan.shape[0]:
+        raise ValueError(f"x has {N} rows but the dispatch plan has {dispatch_plan.shape[0]} tokens")
+    fp8 = x.dtype != torch.bfloat16
+    _need_cuda(recv, "recv", (x.dtype,), 2)
+    if tuple(recv.shape) != (dispatch_plan.rows, H):
+        raise ValueError(f"recv must have shape {(dispatch_plan.rows, H)}")
+    xs_ptr = rs_ptr = 0
+    if fp8:
+        if x_scale is None:
+            raise ValueError("fp8 dispatch needs x_scale [N, H/128]")
+        _need_cuda(x_scale, "x_scale", (torch.float32,), 2)
+        if tuple(x_scale.shape) != (N, H // 128):
+            raise ValueError(f"x_scale must have shape {(N, H // 128)}")
+        if recv_scale is None:
+            recv_scale = torch.empty((dispatch_plan.rows, H // 128), dtype=torch.float32,
+                                     device=x.device)
+        _need_cuda(recv_scale, "recv_scale", (torch.float32,), 2)
+        if tuple(recv_scale.shape) != (dispatch_plan.rows, H // 128):
+            raise ValueError(f"recv_scale must have shape {(dispatch_plan.rows, H // 128)}")
+        xs_ptr, rs_ptr = x_scale.data_ptr(), recv_scale.data_ptr()
+    Nc = combine_plan.shape[0]
+    rows, Hy = y.shape
+    if rows != combine_plan.rows:
+        raise ValueError(f"y must have {combine_plan.rows} rows (got {rows})")
+    if out is None:
+        out = torch.empty((Nc, Hy), dtype=torch.bfloat16, device=y.device)
+    _need_cuda(out, "out", (torch.bfloat16,), 2)
+    if tuple(out.shape) != (Nc, Hy):
+        raise ValueError(f"out must have shape {(Nc, Hy)}")
+    _check(_lib.moe_dispatch_combine(
+        _vp(x.data_ptr()), MOE_FP8E4M3 if fp8 else MOE_BF16, _vp(xs_ptr), H, dispatch_plan._h,
+        _vp(recv.data_ptr()), _vp(rs_ptr), _vp(y.data_ptr()), Hy, combine_plan._h,
+        _vp(out.data_ptr()), 1 if ranked else 0, _vp(_stream_ptr(stream))))
+    return (out, recv_scale) if fp8 else out

@@ -206,6 +206,11 @@ moe_status moe_tune(moe_knob knob, int32_t value)
     case MOE_TUNE_DISPATCH_UNITS_PER_WARP: t.dispatch_units_per_warp = value; break;
     case MOE_TUNE_COMBINE_TOKENS_PER_CTA: t.combine_tokens_per_cta = value; break;
     case MOE_TUNE_PLAN_ENGINE: t.plan_engine = value; break;
+    case MOE_TUNE_FUSED_CTAS_PER_SM: t.fused_ctas_per_sm = value; break;
+    case MOE_TUNE_FUSED_DISPATCH_SHARE: t.fused_dispatch_share = value; break;
+    case MOE_TUNE_FUSED_DISPATCH_RUN: t.fused_dispatch_run = value; break;
+    case MOE_TUNE_FUSED_COMBINE_RUN: t.fused_combine_run = value; break;
+    case MOE_TUNE_FUSED_SMEM_KB: t.fused_smem_kb = value; break;
     default: return fail(MOE_EINVAL, "unknown tuning knob %d", static_cast<int>(knob));
     }
     return ok();
@@ -270,6 +275,8 @@ moe_status moe_plan_create_aligned(int32_t max_tokens, int32_t k, int32_t E, int
         {reinterpret_cast<void **>(&p->tile_cnt), sizeof(int32_t) * E * nt},
         {reinterpret_cast<void **>(&p->tile_rcnt), sizeof(int32_t) * R * nt},
         {reinterpret_cast<void **>(&p->tile_err), sizeof(uint32_t) * nt},
+        {reinterpret_cast<void **>(&p->work), 4 * sizeof(uint32_t)},
+        {reinterpret_cast<void **>(&p->ready), sizeof(uint32_t) * (max_tokens > 0 ? max_tokens : 1)},
     };
     size_t total = 0;
     for (const Part &part : parts)
@@ -337,8 +344,10 @@ moe_status moe_plan(const int32_t *topk_idx, const float *topk_w, int32_t N, int
     return ok();
 }
 
-moe_status moe_dispatch(const void *x, moe_dtype dtype, const float *x_scale, int32_t H,
-                        moe_plan_t plan, void *recv, float *recv_scale, void *stream)
+// Checks a dispatch call and fills its kernel arguments.
+static moe_status dispatch_args(const void *x, moe_dtype dtype, const float *x_scale, int32_t H,
+                                moe_plan_t plan, void *recv, float *recv_scale,
+                                moe::DispatchArgs *a)
 {
     if (!plan)
         return fail(MOE_EINVAL, "plan must not be NULL");
@@ -372,26 +381,36 @@ moe_status moe_dispatch(const void *x, moe_dtype dtype, const float *x_scale, in
     moe_status st = check_plan_device(p);
     if (st != MOE_OK)
         return st;
+    a->x = static_cast<const uint8_t *>(x);
+    a->xs = reinterpret_cast<const uint8_t *>(x_scale);
+    a->recv = static_cast<uint8_t *>(recv);
+    a->rs = reinterpret_cast<uint8_t *>(recv_scale);
+    a->slot = p->slot;
+    a->err = p->err;
+    a->N = p->N;
+    a->k = p->k;
+    a->n_rows = static_cast<int32_t>(moe::recv_rows(p->N, p->k, p->E, p->align));
+    a->row_bytes = static_cast<uint32_t>(H) * elem;
+    a->srow_bytes = srow;
+    return MOE_OK;
+}
+
+moe_status moe_dispatch(const void *x, moe_dtype dtype, const float *x_scale, int32_t H,
+                        moe_plan_t plan, void *recv, float *recv_scale, void *stream)
+{
     moe::DispatchArgs a;
-    a.x = static_cast<const uint8_t *>(x);
-    a.xs = reinterpret_cast<const uint8_t *>(x_scale);
-    a.recv = static_cast<uint8_t *>(recv);
-    a.rs = reinterpret_cast<uint8_t *>(recv_scale);
-    a.slot = p->slot;
-    a.err = p->err;
-    a.N = p->N;
-    a.k = p->k;
-    a.n_rows = static_cast<int32_t>(moe::recv_rows(p->N, p->k, p->E, p->align));
-    a.row_bytes = static_cast<uint32_t>(H) * elem;
-    a.srow_bytes = srow;
-    cudaError_t e = moe::launch_dispatch(a, p->device, static_cast<cudaStream_t>(stream));
+    moe_status st = dispatch_args(x, dtype, x_scale, H, plan, recv, recv_scale, &a);
+    if (st != MOE_OK)
+        return st;
+    cudaError_t e = moe::launch_dispatch(a, plan->device, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return cuda_fail(e, "dispatch kernel");
     return ok();
 }
 
-static moe_status combine_impl(const void *y, int32_t H, moe_plan_t plan, void *out, void *stream,
-                               bool ranked)
+// Checks a combine call and fills its kernel arguments.
+static moe_status combine_args(const void *y, int32_t H, moe_plan_t plan, void *out, bool ranked,
+                               moe::CombineArgs *a)
 {
     if (!plan)
         return fail(MOE_EINVAL, "plan must not be NULL");
@@ -405,22 +424,73 @@ static moe_status combine_impl(const void *y, int32_t H, moe_plan_t plan, void *
     moe_status st = check_plan_device(p);
     if (st != MOE_OK)
         return st;
+    a->y = static_cast<const uint16_t *>(y);
+    a->slot = p->slot;
+    a->w = p->topk_w;
+    a->out = static_cast<uint16_t *>(out);
+    a->err = p->err;
+    a->N = p->N;
+    a->k = p->k;
+    a->n_rows = static_cast<int32_t>(moe::recv_rows(p->N, p->k, p->E, p->align));
+    a->H = H;
+    a->rank_off = p->rank_off;
+    a->R = p->R;
+    a->ranked = ranked;
+    return MOE_OK;
+}
+
+static moe_status combine_impl(const void *y, int32_t H, moe_plan_t plan, void *out, void *stream,
+                               bool ranked)
+{
     moe::CombineArgs a;
-    a.y = static_cast<const uint16_t *>(y);
-    a.slot = p->slot;
-    a.w = p->topk_w;
-    a.out = static_cast<uint16_t *>(out);
-    a.err = p->err;
-    a.N = p->N;
-    a.k = p->k;
-    a.n_rows = static_cast<int32_t>(moe::recv_rows(p->N, p->k, p->E, p->align));
-    a.H = H;
-    a.rank_off = p->rank_off;
-    a.R = p->R;
-    a.ranked = ranked;
-    cudaError_t e = moe::launch_combine(a, p->device, static_cast<cudaStream_t>(stream));
+    moe_status st = combine_args(y, H, plan, out, ranked, &a);
+    if (st != MOE_OK)
+        return st;
+    cudaError_t e = moe::launch_combine(a, plan->device, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess)
         return cuda_fail(e, "combine kernel");
+    return ok();
+}
+
+moe_status moe_dispatch_combine(const void *x, moe_dtype dtype, const float *x_scale,
+                                int32_t H_x, moe_plan_t dispatch_plan, void *recv,
+                                float *recv_scale, const void *y, int32_t H_y,
+                                moe_plan_t combine_plan, void *out, int32_t ranked, void *stream)
+{
+    moe::FusedArgs f;
+    moe_status st =
+        dispatch_args(x, dtype, x_scale, H_x, dispatch_plan, recv, recv_scale, &f.d);
+    if (st != MOE_OK)
+        return st;
+    st = combine_args(y, H_y, combine_plan, out, ranked != 0, &f.c);
+    if (st != MOE_OK)
+        return st;
+    if (dispatch_plan->device != combine_plan->device)
+        return fail(MOE_EINVAL, "both plans must be on the same device");
+    if (f.d.srow_bytes % 16 != 0)
+        return fail(MOE_EINVAL,
+                    "fused dispatch needs fp8 scale rows of a multiple of 16 bytes "
+                    "(H %% 512 == 0; got H=%d)",
+                    H_x);
+    // The combine may read the rows this call dispatches only as a whole: the same buffer
+    // laid out by the same plan, in which case each token waits for its own dispatch.
+    const uintptr_t r0 = reinterpret_cast<uintptr_t>(recv);
+    const uintptr_t r1 = r0 + static_cast<uintptr_t>(f.d.n_rows) * f.d.row_bytes;
+    const uintptr_t y0 = reinterpret_cast<uintptr_t>(y);
+    const uintptr_t y1 = y0 + static_cast<uintptr_t>(f.c.n_rows) * static_cast<uintptr_t>(f.c.H) * 2u;
+    const bool depends = y0 == r0 && f.d.N > 0 && f.c.N > 0;
+    if (depends && (combine_plan != dispatch_plan || dtype != MOE_BF16 || H_x != H_y))
+        return fail(MOE_EINVAL, "y == recv needs one plan, bf16 rows and H_x == H_y");
+    if (!depends && f.d.N > 0 && f.c.N > 0 && y0 < r1 && r0 < y1)
+        return fail(MOE_EINVAL, "y and recv overlap without being the same buffer");
+    f.work = dispatch_plan->work;
+    f.ready = dispatch_plan->ready;
+    f.ready_len = static_cast<uint32_t>(dispatch_plan->cap);
+    f.use_flags = depends;
+    cudaError_t e =
+        moe::launch_fused(f, dispatch_plan->device, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "fused dispatch/combine kernel");
     return ok();
 }
 
@@ -478,6 +548,12 @@ moe_status moe_plan_check(moe_plan_t plan, void *stream, uint32_t *flags)
         e = cudaMemset(plan->sync, 0, 2 * sizeof(uint32_t));
         if (e != cudaSuccess)
             return cuda_fail(e, "cudaMemset(sync)");
+        // and the fused kernel's work words, with its flags (the epoch starts again)
+        e = cudaMemset(plan->work, 0, 4 * sizeof(uint32_t));
+        if (e == cudaSuccess)
+            e = cudaMemset(plan->ready, 0, sizeof(uint32_t) * (plan->cap > 0 ? plan->cap : 1));
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaMemset(work, ready)");
     }
     return ok();
 }

@@ -15,8 +15,7 @@
 // units; each lane issues its KB x VPL 16-byte loads before the first fma.
 #include <algorithm>
 
-#include <cuda_bf16.h>
-
+#include "combine_cta.cuh"
 #include "common.cuh"
 #include "internal.cuh"
 
@@ -35,29 +34,6 @@ struct CombineParams {
     int32_t N, k, n_rows, H, nvec;
     uint32_t nchunks;
 };
-
-__device__ __forceinline__ void fma_bf16x8(float *acc, float wj, const uint4 &v)
-{
-    const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float lo = __uint_as_float(words[q] << 16);
-        const float hi = __uint_as_float(words[q] & 0xffff0000u);
-        acc[2 * q] = __fmaf_rn(wj, lo, acc[2 * q]);
-        acc[2 * q + 1] = __fmaf_rn(wj, hi, acc[2 * q + 1]);
-    }
-}
-
-__device__ __forceinline__ uint4 pack_bf16x8(const float *acc)
-{
-    uint32_t words[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
-        words[q] = *reinterpret_cast<const uint32_t *>(&h);
-    }
-    return make_uint4(words[0], words[1], words[2], words[3]);
-}
 
 template <int KB, int VPL>
 __global__ void __launch_bounds__(kCombineThreads) combine_lsu_kernel(const CombineParams p)
@@ -123,15 +99,6 @@ __global__ void __launch_bounds__(kCombineThreads) combine_lsu_kernel(const Comb
 
 
 // ------------------------------------------------------------------ bulk engine
-// A unit covers CW * 512 bytes of each of the token's k rows: one 16-byte vector per
-// consumer thread, CW consumer warps.  Wider k gets narrower chunks so that a stage
-// (k x chunk) stays at 16 KB: CW = 4 for k <= 8, 2 for k <= 16, 1 for k <= 32.
-template <int CW>
-struct Shape {
-    static constexpr uint32_t kChunk = 512u * CW;
-    static constexpr int kThreads = 32 * (1 + CW);
-};
-constexpr int kMaxBulkStages = 16;
 // Measured on B200 (dsv3 and long shapes): a ring of 32-36 KB per CTA, 3 CTAs per SM and
 // short runs of 4 tokens per CTA (the block scheduler evens out the tail) are fastest;
 // deeper rings, more CTAs per SM and persistent CTAs are slower.
@@ -139,72 +106,14 @@ constexpr int kDefaultSmemBudget = 36 * 1024 + 128;
 constexpr int kDefaultCtasPerSm = 3;
 constexpr int kDefaultTokensPerCta = 4;
 
-struct CombineBulkParams {
-    const uint8_t *y;
-    const int32_t *slot;
-    const float *w;
-    uint8_t *out;
-    uint32_t *err;
-    int32_t N, k, n_rows;
-    uint32_t row_bytes, nchunks, stages, stage_bytes, bar_bytes;
-    uint32_t per_cta;       // tokens of each CTA: [cta * per_cta, +per_cta)
-    const int32_t *rank_off;  // [R+1] first receive row of each rank (rank-grouped order)
-    int32_t R;
-    uint32_t ring_bytes;    // bytes of the stage ring (the rank tables follow it)
-};
-
-constexpr int32_t kNoRank = 0x7fffffff;
-
-// Rank of receive row s: the r with roff[r] <= s < roff[r + 1] (rows are grouped by rank).
-__device__ __forceinline__ int32_t rank_of_row(const int32_t *roff, int R, int32_t s)
-{
-    int lo = 0, hi = R;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (roff[mid] <= s)
-            lo = mid;
-        else
-            hi = mid;
-    }
-    return lo;
-}
-
-// Position of this lane's column in the token's (rank, column) order, lanes j < k holding
-// column j with rank rj (kNoRank for a dropped column, which sorts after every kept one).
-__device__ __forceinline__ int rank_order_pos(int32_t rj, int k, int lane)
-{
-    int pos = 0;
-    for (int q = 0; q < k; ++q) {
-        const int32_t rq = __shfl_sync(0xffffffffu, rj, q);
-        pos += (rq < rj || (rq == rj && q < lane)) ? 1 : 0;
-    }
-    return pos;
-}
-
-// RANKED: the rank-grouped order -- per rank (ascending) an fp32 fma chain over the
-// token's columns on that rank (ascending), and the partials added in ascending rank
-// order; otherwise one fma chain over the columns in order.  In the ranked order the
-// producer puts the token's kept rows into the stage already sorted by (rank, column), so
-// the consumers read rows at fixed offsets and carry only the sorted weights and a bitmask
-// of the positions where a new rank starts.
 template <int KMAX, int CW, bool RANKED>
 __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
     combine_bulk_kernel(const CombineBulkParams p)
 {
-    constexpr uint32_t kChunk_ = Shape<CW>::kChunk;
     extern __shared__ __align__(128) uint8_t smem[];
-    const int S = static_cast<int>(p.stages);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-    uint64_t *empty = full + S;
-    uint8_t *ring = smem + p.bar_bytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int k = p.k;
-    // rank-grouped order: the rank offsets, then per consumer warp the token's weights and
-    // ranks in (rank, column) order
-    int32_t *roff_s = reinterpret_cast<int32_t *>(ring + p.ring_bytes);
-    float *wo_s = reinterpret_cast<float *>(roff_s + (RANKED ? p.R + 1 : 0) +
-                                            (warp > 0 ? (warp - 1) * 64 : 0));
-    int32_t *ro_s = reinterpret_cast<int32_t *>(wo_s + 32);
+    CombineRing r;
+    r.carve<RANKED>(p, smem, warp);
 
     const uint32_t b = blockIdx.x * p.per_cta;  // this CTA's first token
     const int n_tok = b < static_cast<uint32_t>(p.N)
@@ -214,183 +123,23 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
     // barrier so that their latency overlaps the set-up
     int32_t s_first = -1;
     float w_first = 0.f;
-    if (n_tok > 0 && lane < k) {
-        s_first = __ldg(p.slot + static_cast<int64_t>(b) * k + lane);
+    if (n_tok > 0 && lane < p.k) {
+        s_first = __ldg(p.slot + static_cast<int64_t>(b) * p.k + lane);
         if (warp > 0)
-            w_first = __ldg(p.w + static_cast<int64_t>(b) * k + lane);
+            w_first = __ldg(p.w + static_cast<int64_t>(b) * p.k + lane);
     }
     if (RANKED)
-        for (int i = threadIdx.x; i <= p.R; i += blockDim.x)
-            roff_s[i] = __ldg(p.rank_off + i);
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], CW);
-        }
-        mbar_init_fence();
-    }
+        for (int q = threadIdx.x; q <= p.R; q += blockDim.x)
+            r.roff_s[q] = __ldg(p.rank_off + q);
+    if (threadIdx.x == 0)
+        r.init<CW>();
     __syncthreads();
 
-    if (warp == 0) {
-        // ---------------- producer: lane j < k copies row slot[t, j]
-        int32_t s_cur = s_first;
-        int i = 0;
-        bool ok = true;
-        for (int m = 0; m < n_tok && ok; ++m) {
-            const uint32_t t = b + static_cast<uint32_t>(m);
-            int32_t s_nxt = -1;
-            if (m + 1 < n_tok && lane < k)
-                s_nxt = __ldg(p.slot + static_cast<int64_t>(t + 1) * k + lane);
-            const bool valid =
-                lane < k && static_cast<uint32_t>(s_cur) < static_cast<uint32_t>(p.n_rows);
-            const uint32_t nv = __popc(__ballot_sync(0xffffffffu, valid));
-            uint32_t dst = static_cast<uint32_t>(lane) * kChunk_;
-            if (RANKED)
-                dst = static_cast<uint32_t>(rank_order_pos(
-                          valid ? rank_of_row(roff_s, p.R, s_cur) : kNoRank, k, lane)) *
-                      kChunk_;
-            for (uint32_t c = 0; c < p.nchunks; ++c, ++i) {
-                const int st = i % S;
-                const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
-                if (!__all_sync(0xffffffffu, mbar_wait_bounded(&empty[st], ph ^ 1u))) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t off = c * kChunk_;
-                const uint32_t len = min(kChunk_, p.row_bytes - off);
-                if (lane == 0)
-                    mbar_arrive_expect_tx(&full[st], nv * len);
-                __syncwarp();
-                if (valid)
-                    bulk_load(ring + static_cast<size_t>(st) * p.stage_bytes + dst,
-                              p.y + static_cast<int64_t>(s_cur) * p.row_bytes + off, len,
-                              &full[st]);
-            }
-            s_cur = s_nxt;
-        }
-        if (!ok) {
-            if (lane == 0)
-                atomicOr(p.err, MOE_ERR_TIMEOUT);
-            // let the copies of the last stages land before the CTA's memory is released
-            for (int q = (i > S ? i - S : 0); q < i; ++q)
-                (void)mbar_wait_bounded(&full[q % S], static_cast<uint32_t>((q / S) & 1));
-        }
-        return;
-    }
-
-    // ---------------- consumers: thread v owns bytes [16v, 16v + 16) of every chunk.
-    // A token's valid columns (bitmask) and weights are broadcast once per token and kept
-    // in registers; each chunk then costs k shared loads, 8k fmas and one 16-byte store.
-    const uint32_t v16 = static_cast<uint32_t>(threadIdx.x - 32) * 16u;
-    int32_t s_nxt = s_first;
-    float w_nxt = w_first;
     int i = 0;
-    for (int m = 0; m < n_tok; ++m) {
-        const uint32_t t = b + static_cast<uint32_t>(m);
-        const uint32_t vmask = __ballot_sync(
-            0xffffffffu,
-            lane < k && static_cast<uint32_t>(s_nxt) < static_cast<uint32_t>(p.n_rows));
-        float wv[KMAX];
-        uint32_t nv = 0, starts = 0;  // ranked: kept columns; positions opening a new rank
-        if (!RANKED) {
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j)
-                wv[j] = __shfl_sync(0xffffffffu, w_nxt, j);
-        } else {
-            nv = __popc(vmask);
-            const int32_t rj =
-                ((vmask >> lane) & 1u) ? rank_of_row(roff_s, p.R, s_nxt) : kNoRank;
-            const int pos = rank_order_pos(rj, k, lane);
-            __syncwarp();
-            if (lane < k) {
-                wo_s[pos] = w_nxt;
-                ro_s[pos] = rj;
-            }
-            __syncwarp();
-            const float w_sorted = lane < k ? wo_s[lane] : 0.f;
-            const int32_t r_sorted = lane < k ? ro_s[lane] : kNoRank;
-            const int32_t r_before = __shfl_up_sync(0xffffffffu, r_sorted, 1);
-            starts = __ballot_sync(0xffffffffu, lane > 0 && static_cast<uint32_t>(lane) < nv &&
-                                                    r_sorted != r_before);
-#pragma unroll
-            for (int j = 0; j < KMAX; ++j)
-                wv[j] = __shfl_sync(0xffffffffu, w_sorted, j);
-        }
-        if (m + 1 < n_tok && lane < k) {
-            s_nxt = __ldg(p.slot + static_cast<int64_t>(t + 1) * k + lane);
-            w_nxt = __ldg(p.w + static_cast<int64_t>(t + 1) * k + lane);
-        }
-        bool ok = true;
-        for (uint32_t c = 0; c < p.nchunks; ++c, ++i) {
-            const int st = i % S;
-            const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
-            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[st], ph))) {
-                ok = false;
-                break;
-            }
-            const uint32_t off = c * kChunk_;
-            const uint32_t len = min(kChunk_, p.row_bytes - off);
-            const uint8_t *stage = ring + static_cast<size_t>(st) * p.stage_bytes + v16;
-            const bool mine = v16 < len;
-            float acc[8], part[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                acc[e] = 0.f;
-                part[e] = 0.f;
-            }
-#pragma unroll
-            for (int j0 = 0; j0 < KMAX; j0 += 8) {
-                if (j0 >= k)
-                    break;  // warp-uniform
-                uint4 q[8];
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const int j = j0 + jj;
-                    const bool kept = RANKED ? static_cast<uint32_t>(j) < nv : ((vmask >> j) & 1u);
-                    q[jj] = (mine && kept) ? lds_v4(stage + j * kChunk_)
-                                           : make_uint4(0u, 0u, 0u, 0u);
-                }
-                if (j0 + 8 >= k) {
-                    // every row of this stage is in registers: release it to the producer
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(&empty[st]);
-                }
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const int j = j0 + jj;
-                    if (RANKED) {
-                        if (static_cast<uint32_t>(j) >= nv)
-                            continue;
-                        if ((starts >> j) & 1u) {
-                            // close the previous rank's chain
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                acc[e] = __fadd_rn(acc[e], part[e]);
-                                part[e] = 0.f;
-                            }
-                        }
-                        fma_bf16x8(part, wv[j], q[jj]);
-                    } else if ((vmask >> j) & 1u) {
-                        fma_bf16x8(acc, wv[j], q[jj]);
-                    }
-                }
-            }
-            if (RANKED && nv > 0) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    acc[e] = __fadd_rn(acc[e], part[e]);
-            }
-            if (mine)
-                st_stream_v4(p.out + static_cast<int64_t>(t) * p.row_bytes + off + v16,
-                             pack_bf16x8(acc));
-        }
-        if (!ok) {
-            if (lane == 0)
-                atomicOr(p.err, MOE_ERR_TIMEOUT);
-            return;
-        }
-    }
+    if (warp == 0)
+        (void)combine_produce<KMAX, CW, RANKED>(p, r, b, n_tok, s_first, i, nullptr, 0u);
+    else
+        (void)combine_consume<KMAX, CW, RANKED>(p, r, b, n_tok, s_first, w_first, i);
 }
 
 template <int KB, int VPL>

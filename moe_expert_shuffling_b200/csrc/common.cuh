@@ -167,6 +167,43 @@ __device__ __forceinline__ uint4 lds_v4(const void *p)
     return v;
 }
 
+// gpu-scope acquire / release accesses for flags and counters shared between CTAs.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *a)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t *a, uint32_t v)
+{
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(a), "r"(v)
+                 : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t *a, uint32_t v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+
+// Order this thread's async-proxy (bulk copy) accesses to global memory against its
+// generic-proxy accesses: after bulk stores have completed and before a flag is released;
+// after a flag has been acquired and before bulk loads read what it guards.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Relaxed read of a word that other CTAs may set (an error flag polled inside a wait).
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t *a)
+{
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+    return v;
+}
+
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 

@@ -2,45 +2,25 @@
 // produced by the copy itself (FUSCO, arXiv 2512.22036, abstract; FUSCO summary, Group 3:
 // data is placed at its destination with no staging buffer and no later rearrangement).
 //
-// Engine: warps each running their own pipeline over a contiguous run of work units
-// (token, row chunk).  Lane 0 stages a chunk of x[t] into shared memory with one bulk
-// async copy (cp.async.bulk, completion on an mbarrier); once it has landed, lane j
-// issues the bulk store of that chunk to receive row slot[t, j].  So every token row
-// is read from HBM once and written k times -- the "read once, fan out locally" form of
-// FUSCO's dedup (one move per token, which is at most one per destination rank).  A
-// stage is refilled only after the stores reading it have drained (wait_group.read).
-// fp8 rows carry their fp32 scale block along when its size is a multiple of 16 bytes;
-// otherwise a small second kernel moves the scales.
+// Engine: warps each running their own bulk-copy pipeline (dispatch_warp.cuh) over a
+// contiguous run of work units (token, row chunk), so every token row is read from HBM
+// once and written k times -- the "read once, fan out locally" form of FUSCO's dedup (one
+// move per token, which is at most one per destination rank).  fp8 rows carry their fp32
+// scale block along when its size is a multiple of 16 bytes; otherwise a small second
+// kernel moves the scales.
 #include <algorithm>
 
 #include "common.cuh"
+#include "dispatch_warp.cuh"
 #include "internal.cuh"
 
 namespace moe {
 namespace {
 
-constexpr uint32_t kMaxChunkBytes = 32768;
-constexpr int kMaxStages = 8;
 // Measured on B200 (dsv3 and long shapes): short runs of 2 units per warp on a grid that
 // covers all units beat persistent warps by ~12% (the block scheduler evens out the
 // tail); 4 stages with 2 store groups in flight per warp.
 constexpr int kDefaultUnitsPerWarp = 2;
-
-struct DispatchParams {
-    const uint8_t *x;
-    const uint8_t *xs;
-    uint8_t *recv;
-    uint8_t *rs;
-    const int32_t *slot;
-    uint32_t *err;
-    uint32_t units;         // N * nchunks (< 2^31)
-    uint32_t per_warp;      // units of each warp: [warp * per_warp, +per_warp)
-    int32_t k, n_rows;
-    uint32_t nchunks;
-    int32_t stages, lag;
-    uint32_t row_bytes, srow_bytes, chunk_bytes, stage_bytes, scale_off, bar_bytes;
-    bool bulk_scales;
-};
 
 __global__ void __launch_bounds__(128) dispatch_bulk_kernel(const DispatchParams p)
 {
@@ -60,83 +40,7 @@ __global__ void __launch_bounds__(128) dispatch_bulk_kernel(const DispatchParams
         mbar_init_fence();
     }
     __syncwarp();
-
-    // Issue the load of this warp's i-th unit into stage i % S (lane 0 only).
-    auto issue_load = [&](int i) {
-        const uint32_t u = u0 + static_cast<uint32_t>(i);
-        const uint32_t t = u / p.nchunks;
-        const uint32_t c = u - t * p.nchunks;
-        const uint32_t off = c * p.chunk_bytes;
-        const uint32_t len = min(p.chunk_bytes, p.row_bytes - off);
-        const int s = static_cast<int>(i % S);
-        uint8_t *st = stage0 + static_cast<size_t>(s) * p.stage_bytes;
-        const bool sc = p.bulk_scales && c == 0;
-        mbar_arrive_expect_tx(&bars[s], len + (sc ? p.srow_bytes : 0u));
-        bulk_load(st, p.x + static_cast<int64_t>(t) * p.row_bytes + off, len, &bars[s]);
-        if (sc)
-            bulk_load(st + p.scale_off, p.xs + static_cast<int64_t>(t) * p.srow_bytes,
-                      p.srow_bytes, &bars[s]);
-    };
-
-    int next_load = S < n_my ? S : n_my;  // units [0, next_load) have been issued
-    if (lane == 0)
-        for (int i = 0; i < next_load; ++i)
-            issue_load(i);
-
-    int32_t cur = -1;
-    if (n_my > 0 && lane < p.k)
-        cur = __ldg(p.slot + (u0 / p.nchunks) * p.k + lane);
-
-    bool ok = true;
-    int i = 0;
-    for (; i < n_my; ++i) {
-        const int s = i % S;
-        const uint32_t parity = static_cast<uint32_t>((i / S) & 1);
-        const uint32_t u = u0 + static_cast<uint32_t>(i);
-        const uint32_t t = u / p.nchunks;
-        const uint32_t c = u - t * p.nchunks;
-        const uint32_t off = c * p.chunk_bytes;
-        const uint32_t len = min(p.chunk_bytes, p.row_bytes - off);
-
-        // Slots of the next unit, fetched while this unit's row is in flight.
-        int32_t nxt = -1;
-        if (i + 1 < n_my && lane < p.k)
-            nxt = __ldg(p.slot + ((u + 1) / p.nchunks) * p.k + lane);
-
-        const bool landed = mbar_wait_bounded(&bars[s], parity);
-        if (!__all_sync(0xffffffffu, landed)) {
-            ok = false;
-            break;
-        }
-        fence_proxy_async_smem();
-        const uint8_t *st = stage0 + static_cast<size_t>(s) * p.stage_bytes;
-        if (lane < p.k && static_cast<uint32_t>(cur) < static_cast<uint32_t>(p.n_rows)) {
-            bulk_store(p.recv + static_cast<int64_t>(cur) * p.row_bytes + off, st, len);
-            if (p.bulk_scales && c == 0)
-                bulk_store(p.rs + static_cast<int64_t>(cur) * p.srow_bytes, st + p.scale_off,
-                           p.srow_bytes);
-        }
-        bulk_commit();
-
-        // Refill the stage of unit i - lag once its stores have read shared memory.
-        const int r = i - p.lag;
-        if (r >= 0 && r + S < n_my) {
-            bulk_wait_read_dyn(p.lag);
-            __syncwarp();
-            if (lane == 0)
-                issue_load(r + S);
-            next_load = r + S + 1;
-        }
-        cur = nxt;
-    }
-    bulk_wait_all();
-    if (!ok) {
-        if (lane == 0)
-            atomicOr(p.err, MOE_ERR_TIMEOUT);
-        // Let loads still in flight land before this warp's shared memory is released.
-        for (int m = i; m < next_load; ++m)
-            (void)mbar_wait_bounded(&bars[m % S], static_cast<uint32_t>((m / S) & 1));
-    }
+    (void)dispatch_warp_run(p, bars, stage0, u0, n_my, 0u, true);
 }
 
 // Scale rows whose size is not a multiple of 16 bytes: one thread per fp32 scale.
@@ -163,20 +67,16 @@ cudaError_t launch_dispatch(const DispatchArgs &a, int device, cudaStream_t stre
         return cudaSuccess;
     const Tuning &tu = tuning();
     int stages = tu.dispatch_stages > 0 ? tu.dispatch_stages : 4;
-    stages = std::min(std::max(stages, 2), kMaxStages);
+    stages = std::min(std::max(stages, 2), kDispatchMaxStages);
     int lag = tu.dispatch_lag > 0 ? tu.dispatch_lag : 2;
     lag = std::min(std::max(lag, 1), std::min(stages - 1, 7));
     int wpc = tu.dispatch_warps_per_cta > 0 ? tu.dispatch_warps_per_cta : 1;
     wpc = std::min(std::max(wpc, 1), 4);
 
-    const uint32_t nchunks =
-        static_cast<uint32_t>(ceil_div(a.row_bytes, kMaxChunkBytes));
-    const uint32_t chunk =
-        static_cast<uint32_t>(round_up(ceil_div(a.row_bytes, nchunks), 16));
-    const bool bulk_scales = a.srow_bytes > 0 && a.srow_bytes % 16 == 0;
-    const uint32_t scale_off = static_cast<uint32_t>(round_up(chunk, 128));
-    const uint32_t stage_bytes =
-        static_cast<uint32_t>(round_up(scale_off + (bulk_scales ? a.srow_bytes : 0u), 128));
+    const DispatchGeometry g = dispatch_geometry(a.row_bytes, a.srow_bytes);
+    const uint32_t nchunks = g.nchunks, chunk = g.chunk, scale_off = g.scale_off,
+                   stage_bytes = g.stage_bytes;
+    const bool bulk_scales = g.bulk_scales;
 
     const int max_optin = max_smem_optin(device);
     cudaError_t e = cudaSuccess;

@@ -29,6 +29,11 @@ struct moe_plan_s {
     uint32_t *tile_err = nullptr;
     const float *topk_w = nullptr;
     int32_t plan_kernels = 0;  // kernels the last launch_plan enqueued
+    // moe_dispatch_combine: work words [next dispatch item, next combine item, CTAs done,
+    // epoch of the last launch] (the launch's last CTA resets the counters and advances the
+    // epoch) and per-token ready flags [cap] holding the epoch of the launch that last
+    // dispatched the token
+    uint32_t *work = nullptr, *ready = nullptr;
 };
 
 namespace moe {
@@ -60,6 +65,11 @@ struct Tuning {
     int dispatch_units_per_warp = 0;
     int combine_tokens_per_cta = 0;
     int plan_engine = 0;       // 0/1: one cooperative kernel when it fits, 2: three kernels
+    int fused_ctas_per_sm = 0;
+    int fused_dispatch_share = 0;  // percent of CTAs that start on dispatch work
+    int fused_dispatch_run = 0;    // tokens per dispatch work item
+    int fused_combine_run = 0;     // tokens per combine work item
+    int fused_smem_kb = 0;
 };
 Tuning &tuning();
 
@@ -116,5 +126,16 @@ struct CombineArgs {
     bool ranked = false;   // rank-grouped summation order instead of one chain
 };
 cudaError_t launch_combine(const CombineArgs &a, int device, cudaStream_t stream);
+
+// One persistent launch doing a dispatch and a combine at once (moe_dispatch_combine).
+struct FusedArgs {
+    DispatchArgs d;
+    CombineArgs c;
+    uint32_t *work;          // [4] the dispatch plan's work counters and epoch
+    uint32_t *ready;         // [ready_len] the dispatch plan's per-token flags
+    uint32_t ready_len;
+    bool use_flags;          // c reads the rows d writes (y == recv, one plan)
+};
+cudaError_t launch_fused(const FusedArgs &a, int device, cudaStream_t stream);
 
 }  // namespace moe

@@ -443,26 +443,6 @@ __global__ void __launch_bounds__(kPlanThreads) plan_rank_kernel(const PlanK p)
 }
 
 // ----------------------------------------------------------- fused (cooperative)
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *a)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t *a, uint32_t v)
-{
-    uint32_t old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(a), "r"(v)
-                 : "memory");
-    return old;
-}
-
-__device__ __forceinline__ void st_release_gpu(uint32_t *a, uint32_t v)
-{
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
-}
-
 // Sense-reversing grid barrier for a co-resident grid.  sync[0] counts arrivals; the last
 // CTA to arrive sets it back to 0 and advances the generation word sync[1], which the
 // others wait on, so the words are ready for the next barrier (and the next launch) with no
