@@ -133,9 +133,23 @@ def pct_stats(ms_list):
             "p90": round(q(0.9), 2), "n": len(v)}
 
 
-def flushed_kernel_times(step, stream, dev, iters):
-    """Each of plan, dispatch and combine timed alone (CUDA events on the launching stream),
-    each launch preceded by an L2 flush.  The flush READS a buffer of twice the L2 size: that
+def kernel_split(d: dict, fused: bool) -> dict:
+    """Per-kernel entries of the line: with --fused the dispatch slot holds the one launch
+    that does dispatch and combine."""
+    d = dict(d)
+    if fused:
+        if "dispatch_combine" not in d:
+            d["dispatch_combine"] = d["dispatch"]
+        d.pop("dispatch", None)
+        d.pop("combine", None)
+    else:
+        d.pop("dispatch_combine", None)
+    return d
+
+
+def flushed_kernel_times(step, stream, dev, iters, names=("plan", "dispatch", "combine")):
+    """Each kernel of the step (plan, dispatch, combine) timed alone (CUDA events on the
+    launching stream), each launch preceded by an L2 flush.  The flush READS a buffer of twice the L2 size: that
     writes back and evicts whatever the previous kernel left dirty and leaves only clean,
     unrelated lines, so the timed kernel neither hits in L2 nor pays for another's
     write-back."""
@@ -143,18 +157,18 @@ def flushed_kernel_times(step, stream, dev, iters):
     with torch.cuda.stream(stream):
         scratch = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev)
         sink = torch.empty((), dtype=torch.float32, device=dev)
-    times = {"plan": [], "dispatch": [], "combine": []}
+    times = {name: [] for name in names}
     for it in range(iters + 3):
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]
         with torch.cuda.stream(stream):
-            for phase in range(3):
+            for phase in range(len(names)):
                 torch.sum(scratch, dim=0, out=sink)
                 ev[2 * phase].record(stream)
                 step(phase_only=phase)
                 ev[2 * phase + 1].record(stream)
         stream.synchronize()
         if it >= 3:  # warm-up
-            for phase, name in enumerate(("plan", "dispatch", "combine")):
+            for phase, name in enumerate(names):
                 times[name].append(ev[2 * phase].elapsed_time(ev[2 * phase + 1]))
     out = {name: pct_stats(t) for name, t in times.items()}
     out["flush"] = f"read of a {2 * l2 >> 20} MB buffer before each launch"
@@ -302,13 +316,23 @@ def run_ours(args):
     plan = ms.moe_plan_create(cfg.N, cfg.k, cfg.E, cfg.R, align=args.align)
 
     def step(ev=None, phase_only=None):
-        """One step: plan, dispatch, combine (phase_only = 0, 1 or 2 runs just that one)."""
+        """One step: plan, dispatch, combine (phase_only = 0, 1 or 2 runs just that one).
+        With --fused: plan, then dispatch and combine in one launch (phase 1)."""
         if ev is not None:
             ev[0].record(stream)
         if phase_only in (None, 0):
             ms.moe_plan(idx, w, cfg.E, cfg.R, plan=plan, stream=stream)
         if ev is not None:
             ev[1].record(stream)
+        if args.fused:
+            if phase_only in (None, 1):
+                ms.moe_dispatch_combine(x, plan, recv, recv if identity else y, plan, out=out,
+                                        x_scale=xs, recv_scale=rs,
+                                        ranked=args.combine == "ranked", stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
+                ev[3].record(stream)
+            return
         if phase_only in (None, 1):
             if rs is not None:
                 ms.moe_dispatch(x, plan, recv=recv, x_scale=xs, recv_scale=rs, stream=stream)
@@ -377,14 +401,16 @@ def run_ours(args):
     disp_us = 1e3 * statistics.mean(t_disp)
     comb_us = 1e3 * statistics.mean(t_comb)
     plan_us = 1e3 * statistics.mean(t_plan)
-    if disp_us >= comb_us:
+    if args.fused:
+        dom, dom_bytes, dom_us = "fused_dispatch_combine_kernel", db + cb, disp_us
+    elif disp_us >= comb_us:
         dom, dom_bytes, dom_us = "dispatch_bulk_kernel", db, disp_us
     else:
         dom, dom_bytes, dom_us = "combine_bulk_kernel", cb, comb_us
     achieved = dom_bytes / (dom_us * 1e-6) / 1e9
     # plan (1 cooperative kernel or 3) + dispatch (+ the scale kernel for fp8 scale rows
     # that are not a multiple of 16 bytes) + combine
-    launches_per_step = (plan.plan_kernels + 1 + 1 +
+    launches_per_step = (plan.plan_kernels + 1 + (0 if args.fused else 1) +
                          (1 if cfg.payload == "fp8" and (4 * (cfg.H // 128)) % 16 else 0))
 
     # end to end: pinned host inputs -> device, step, result -> pinned host
@@ -429,8 +455,14 @@ def run_ours(args):
     # each kernel alone after an L2 flush (outside the timed region)
     flushed = None
     if args.flushed_iters > 0:
-        flushed = flushed_kernel_times(step, stream, dev, args.flushed_iters)
-        for name, nbytes in (("dispatch", db), ("combine", cb), ("plan", plan_bytes(cfg))):
+        if args.fused:
+            flushed = flushed_kernel_times(step, stream, dev, args.flushed_iters,
+                                           names=("plan", "dispatch_combine"))
+            sizes = (("dispatch_combine", db + cb), ("plan", plan_bytes(cfg)))
+        else:
+            flushed = flushed_kernel_times(step, stream, dev, args.flushed_iters)
+            sizes = (("dispatch", db), ("combine", cb), ("plan", plan_bytes(cfg)))
+        for name, nbytes in sizes:
             flushed[name]["gbs_at_median"] = round(nbytes / (flushed[name]["median"] * 1e-6) / 1e9, 1)
 
     cpu = None
@@ -452,7 +484,8 @@ def run_ours(args):
         "config": {"workload": workload_name(cfg)
                    + ("" if args.combine == "chain" else ", combine grouped by rank")
                    + (f", segments aligned to {args.align} rows" if args.align > 1 else "")
-                   + (f", {args.drop:.0%} of entries dropped" if args.drop > 0 else ""),
+                   + (f", {args.drop:.0%} of entries dropped" if args.drop > 0 else "")
+                   + (", dispatch and combine in one launch" if args.fused else ""),
                    "model": f"{cfg.name}-shaped MoE layer shuffle",
                    "global_batch": cfg.N * world, "seq_len": cfg.N, "parallelism": f"replicas{world}",
                    "ep_ranks_logical": cfg.R,
@@ -461,15 +494,17 @@ def run_ours(args):
         "tokens_per_s": round(tokens_per_s, 1),
         "pct_roofline": {"of_nominal_8000": round(100 * value / world / NOMINAL_HBM_GBS, 2),
                          f"of_{peak_kind}_{peak:g}": round(100 * value / world / peak, 2)},
-        "kernels_us": {"plan": round(plan_us, 2), "dispatch": round(disp_us, 2),
-                       "combine": round(comb_us, 2)},
-        "kernels_unflushed_us": {"note": "back-to-back steps on one stream, no flush",
-                                 "plan": pct_stats(t_plan), "dispatch": pct_stats(t_disp),
-                                 "combine": pct_stats(t_comb)},
+        "kernels_us": kernel_split({"plan": round(plan_us, 2), "dispatch": round(disp_us, 2),
+                                    "combine": round(comb_us, 2)}, args.fused),
+        "kernels_unflushed_us": kernel_split(
+            {"note": "back-to-back steps on one stream, no flush", "plan": pct_stats(t_plan),
+             "dispatch": pct_stats(t_disp), "combine": pct_stats(t_comb)}, args.fused),
         "kernels_flushed_us": flushed,
-        "kernels_gbs": {"dispatch": round(db / (disp_us * 1e-6) / 1e9, 1),
-                        "combine": round(cb / (comb_us * 1e-6) / 1e9, 1),
-                        "plan": round(plan_bytes(cfg) / (plan_us * 1e-6) / 1e9, 1)},
+        "kernels_gbs": kernel_split(
+            {"dispatch": round(db / (disp_us * 1e-6) / 1e9, 1),
+             "combine": round(cb / (max(comb_us, 1e-3) * 1e-6) / 1e9, 1),
+             "dispatch_combine": round((db + cb) / (disp_us * 1e-6) / 1e9, 1),
+             "plan": round(plan_bytes(cfg) / (plan_us * 1e-6) / 1e9, 1)}, args.fused),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
@@ -485,7 +520,8 @@ def run_ours(args):
 def run_micro_batches(args):
     """The batch split into M micro-batches.  Without --overlap they run one after the
     other; with it, dispatch of micro-batch m runs on a second stream while micro-batch
-    m-1 combines (concurrent dispatch and combine, ordered by events)."""
+    m-1 combines (concurrent dispatch and combine, ordered by events); with --fused the
+    two run in one moe_dispatch_combine launch."""
     import moe_expert_shuffling_b200 as ms
     from moe_expert_shuffling_b200 import build as lib_build
 
@@ -523,6 +559,12 @@ def run_micro_batches(args):
             ms.moe_plan(mb["idx"], mb["w"], cfg.E, cfg.R, plan=mb["plan"], stream=sa)
         ms.moe_dispatch(mbs[0]["x"], mbs[0]["plan"], recv=mbs[0]["recv"], stream=sa)
         for m in range(1, M):
+            if args.fused:
+                # dispatch of micro-batch m and combine of m-1 in one launch
+                ms.moe_dispatch_combine(mbs[m]["x"], mbs[m]["plan"], mbs[m]["recv"],
+                                        mbs[m - 1]["y"], mbs[m - 1]["plan"],
+                                        out=mbs[m - 1]["out"], stream=sa)
+                continue
             if args.overlap:
                 ready = torch.cuda.Event()
                 ready.record(sa)
@@ -567,10 +609,12 @@ def run_micro_batches(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": workload_name(cfg) + f", {M} micro-batches"
-                   + (", dispatch of each overlapping the previous combine" if args.overlap
+                   + (", dispatch of each fused with the previous combine in one launch"
+                      if args.fused else
+                      ", dispatch of each overlapping the previous combine" if args.overlap
                       else ", one after the other")},
         "pct_roofline": {"of_nominal_8000": round(100 * value / world / NOMINAL_HBM_GBS, 2)},
-        "gpu_launches": (3 * M) * args.steps,
+        "gpu_launches": ((2 * M + 1) if args.fused else (3 * M)) * args.steps,
     }), flush=True)
 
 
@@ -713,6 +757,8 @@ def main(argv=None):
                     help="split each step's batch into this many micro-batches")
     ap.add_argument("--overlap", action="store_true",
                     help="with micro-batches: dispatch of one overlaps combine of the previous")
+    ap.add_argument("--fused", action="store_true",
+                    help="dispatch and combine in one launch (moe_dispatch_combine)")
     ap.add_argument("--combine", default="chain", choices=["chain", "ranked"],
                     help="combine order: one fma chain per token, or grouped by rank first")
     ap.add_argument("--flushed-iters", type=int, default=50,

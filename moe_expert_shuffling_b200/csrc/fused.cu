@@ -32,11 +32,23 @@
 namespace moe {
 namespace {
 
-constexpr int kDefaultCtasPerSm = 3;
-constexpr int kDefaultSmemKb = 64;
-constexpr uint32_t kDefaultDispatchRun = 2;       // tokens per dispatch item
-constexpr uint32_t kDefaultDispatchRunFlags = 4;  // ... when each item ends in a flag release
-constexpr uint32_t kDefaultCombineRun = 8;        // tokens per combine item
+// Defaults, measured on B200 over the dsv3, skew, long, Mixtral, top-16 and top-32 shapes
+// (independent expert outputs), and dsv3 and Mixtral with y = recv:
+//  * 4 CTAs of 48 KB per SM for CW = 4 consumer warps; narrower chunks (CW = 2, 1) get
+//    proportionally more, smaller CTAs, as the combine kernel does;
+//  * dispatch items of about 256 KB of traffic (2 tokens of the dsv3 shape, 8 of Mixtral);
+//  * combine items of about 512 KB of traffic, at most 4 tokens (half of both when they
+//    wait on flags);
+//  * 10% of the CTAs starting on dispatch (30% when the combine waits on flags: with fewer,
+//    most CTAs would wait for the few that dispatch).
+// With these the fused step takes 0.95-0.98x the time of the two separate kernels.
+constexpr int kDefaultCtasPerSm = 4;
+constexpr int kDefaultSmemKb = 48;
+constexpr int kDefaultDispatchSharePct = 10;
+constexpr int kDefaultDispatchSharePctFlags = 30;
+constexpr double kDispatchItemBytes = 256.0 * 1024;
+constexpr double kCombineItemBytes = 512.0 * 1024;
+constexpr uint32_t kMaxCombineRun = 4;
 constexpr int kDispatchStages = 4;
 
 struct FusedParams {
@@ -249,7 +261,8 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
     // with fewer stages if even one does not fit), and a combine ring using the larger of
     // the budget and the dispatch rings' area.
     const size_t budget = static_cast<size_t>(
-        std::min((tu.fused_smem_kb > 0 ? tu.fused_smem_kb : kDefaultSmemKb) * 1024, max_optin));
+        std::min((tu.fused_smem_kb > 0 ? tu.fused_smem_kb : kDefaultSmemKb * CW / 4) * 1024,
+                 max_optin));
     int d_stages = kDispatchStages;
     while (d_stages > 2 && static_cast<size_t>(d_stages) * g.stage_bytes > budget)
         --d_stages;
@@ -282,37 +295,42 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
         return e;
     if (per_sm < 1)
         return cudaErrorInvalidConfiguration;
-    per_sm = std::min(per_sm, tu.fused_ctas_per_sm > 0 ? tu.fused_ctas_per_sm : kDefaultCtasPerSm);
+    per_sm = std::min(per_sm, tu.fused_ctas_per_sm > 0 ? tu.fused_ctas_per_sm
+                                                       : kDefaultCtasPerSm * 4 / CW);
     const int64_t grid = static_cast<int64_t>(sm_count(device)) * per_sm;
 
     // work items
+    const double d_token_bytes = static_cast<double>(a.d.row_bytes + a.d.srow_bytes) * (1 + a.d.k);
     uint32_t d_run = tu.fused_dispatch_run > 0
                          ? static_cast<uint32_t>(tu.fused_dispatch_run)
-                         : (a.use_flags ? kDefaultDispatchRunFlags : kDefaultDispatchRun);
+                         : static_cast<uint32_t>(kDispatchItemBytes / d_token_bytes + 0.5);
     d_run = std::min<uint32_t>(std::max<uint32_t>(d_run, 1), 32);  // one flag per lane
-    const uint32_t c_run = tu.fused_combine_run > 0 ? static_cast<uint32_t>(tu.fused_combine_run)
-                                                    : kDefaultCombineRun;
+    uint32_t c_run = static_cast<uint32_t>(tu.fused_combine_run);
+    if (c_run == 0) {
+        const double c_token_bytes = static_cast<double>(c.row_bytes) * (1 + a.c.k);
+        const double div = a.use_flags ? 2.0 : 1.0;
+        c_run = static_cast<uint32_t>(kCombineItemBytes / div / c_token_bytes + 0.5);
+        c_run = std::min<uint32_t>(std::max<uint32_t>(c_run, 1),
+                                   static_cast<uint32_t>(kMaxCombineRun / div));
+    }
     fp.d_run_tokens = d_run;
     fp.c_run_tokens = c_run;
     fp.d_items = static_cast<uint32_t>(ceil_div(a.d.N, d_run));
     fp.c_items = static_cast<uint32_t>(ceil_div(a.c.N, c_run));
 
-    // CTAs that start on dispatch: the dispatch side's share of the bytes (or the knob),
-    // at least one when there is dispatch work (the ready flags rely on it) and at least
-    // one starting on combine when there is combine work.
+    // CTAs that start on dispatch: a share of the grid, at least one when there is
+    // dispatch work (the ready flags rely on it) and at least one starting on combine when
+    // there is combine work.
     int64_t d_first;
     if (fp.d_items == 0) {
         d_first = 0;
     } else if (fp.c_items == 0) {
         d_first = grid;
     } else {
-        if (tu.fused_dispatch_share > 0) {
-            d_first = grid * std::min(tu.fused_dispatch_share, 100) / 100;
-        } else {
-            const double db = static_cast<double>(a.d.N) * a.d.row_bytes * (1 + a.d.k);
-            const double cb = static_cast<double>(a.c.N) * c.row_bytes * (1 + a.c.k);
-            d_first = static_cast<int64_t>(grid * db / (db + cb) + 0.5);
-        }
+        const int share = tu.fused_dispatch_share > 0 ? std::min(tu.fused_dispatch_share, 100)
+                          : a.use_flags ? kDefaultDispatchSharePctFlags
+                                        : kDefaultDispatchSharePct;
+        d_first = grid * share / 100;
         d_first = grid < 2 ? grid : std::min<int64_t>(std::max<int64_t>(d_first, 1), grid - 1);
     }
     fp.d_first_ctas = static_cast<uint32_t>(d_first);
