@@ -14,7 +14,7 @@
  *     Arrays are dense and row-major.  A plan is used on the device it was created on.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
  *     Calls only enqueue work on it; none of them synchronises the host or copies
- *     device data to the host, except moe_plan_check.
+ *     device data to the host, except moe_plan_check and moe_wait_selftest.
  *   - Arguments are checked on the host before anything is enqueued; a bad argument
  *     returns MOE_EINVAL and enqueues nothing.  A CUDA failure returns MOE_ECUDA.
  *     moe_last_error() then describes the failure (per host thread).
@@ -56,7 +56,7 @@ typedef enum {
 #define MOE_ERR_ID_RANGE 1u   /* a routing id outside [0, E) */
 #define MOE_ERR_ID_DUP 2u     /* a token listed the same expert twice */
 #define MOE_ERR_BOUNDS 4u     /* an internal index fell outside its array (entry skipped) */
-#define MOE_ERR_TIMEOUT 8u    /* a device wait gave up after its iteration limit */
+#define MOE_ERR_TIMEOUT 8u    /* a device wait gave up after its limit (about 1 s) */
 
 /* Opaque plan: device arrays owned by the library, reusable across calls. */
 typedef struct moe_plan_s *moe_plan_t;
@@ -234,6 +234,20 @@ MOE_API moe_status moe_dispatch_combine(const void *x, moe_dtype dtype, const fl
                                         float *recv_scale, const void *y, int32_t H_y,
                                         moe_plan_t combine_plan, void *out, int32_t ranked,
                                         void *stream);
+
+/*
+ * moe_wait_selftest -- a diagnostic with no counterpart in the reference pages.  Runs one of
+ * the library's bounded device waits on something that never completes and returns, in
+ * *flags, the error word it leaves:
+ *   which = 0  the per-token ready-flag wait of moe_dispatch_combine, on a flag nothing sets;
+ *   which = 1  the mbarrier wait of the bulk-copy pipelines, on a barrier that expects two
+ *              arrivals and gets one (no copy in flight).
+ * Either wait gives up after about one second; *flags is then MOE_ERR_TIMEOUT and the CUDA
+ * context stays usable.  Synchronous: allocates two device words, launches one 32-thread
+ * block on `stream`, waits for it and frees the words.  MOE_EINVAL for another `which` or
+ * a NULL `flags`; MOE_ECUDA if a CUDA call fails.
+ */
+MOE_API moe_status moe_wait_selftest(int32_t which, void *stream, uint32_t *flags);
 
 /* moe_plan_query -- fill *view with the plan's shape and device pointers. */
 MOE_API moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *view);

@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "MoeError", "Plan", "moe_plan", "moe_plan_create", "moe_dispatch", "moe_combine",
-    "moe_dispatch_combine",
+    "moe_dispatch_combine", "moe_wait_selftest",
     "moe_tune", "lib_path", "version", "ERR_ID_RANGE", "ERR_ID_DUP", "ERR_BOUNDS",
     "ERR_TIMEOUT", "KNOBS",
 ]
@@ -88,6 +88,8 @@ def _load():
     lib.moe_version.argtypes = []
     lib.moe_tune.restype = st
     lib.moe_tune.argtypes = [ctypes.c_int, _i32]
+    lib.moe_wait_selftest.restype = st
+    lib.moe_wait_selftest.argtypes = [_i32, _vp, ctypes.POINTER(ctypes.c_uint32)]
     return lib
 
 
@@ -369,3 +371,12 @@ def moe_dispatch_combine(x: torch.Tensor, dispatch_plan: Plan, recv: torch.Tenso
         _vp(recv.data_ptr()), _vp(rs_ptr), _vp(y.data_ptr()), Hy, combine_plan._h,
         _vp(out.data_ptr()), 1 if ranked else 0, _vp(_stream_ptr(stream))))
     return (out, recv_scale) if fp8 else out
+
+
+def moe_wait_selftest(which: int, stream=None) -> int:
+    """Run one bounded device wait on something that never completes (0: ready flag,
+    1: mbarrier) and return the error word it leaves (ERR_TIMEOUT when the wait gave up).
+    Blocks for about a second."""
+    flags = ctypes.c_uint32(0)
+    _check(_lib.moe_wait_selftest(which, _vp(_stream_ptr(stream)), ctypes.byref(flags)))
+    return flags.value

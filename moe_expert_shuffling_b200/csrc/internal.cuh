@@ -138,4 +138,8 @@ struct FusedArgs {
 };
 cudaError_t launch_fused(const FusedArgs &a, int device, cudaStream_t stream);
 
+// moe_wait_selftest: one bounded device wait on something that never completes; *flags gets
+// the error word (synchronous).
+cudaError_t run_wait_selftest(int which, cudaStream_t stream, uint32_t *flags);
+
 }  // namespace moe
