@@ -241,11 +241,13 @@ MOE_API moe_status moe_dispatch_combine(const void *x, moe_dtype dtype, const fl
  * *flags, the error word it leaves:
  *   which = 0  the per-token ready-flag wait of moe_dispatch_combine, on a flag nothing sets;
  *   which = 1  the mbarrier wait of the bulk-copy pipelines, on a barrier that expects two
- *              arrivals and gets one (no copy in flight).
- * Either wait gives up after about one second; *flags is then MOE_ERR_TIMEOUT and the CUDA
- * context stays usable.  Synchronous: allocates two device words, launches one 32-thread
- * block on `stream`, waits for it and frees the words.  MOE_EINVAL for another `which` or
- * a NULL `flags`; MOE_ECUDA if a CUDA call fails.
+ *              arrivals and gets one (no copy in flight);
+ *   which = 2  the grid barrier of the plan kernel, in a grid of two blocks of which only
+ *              one arrives.
+ * Each wait gives up after about one second; *flags is then MOE_ERR_TIMEOUT and the CUDA
+ * context stays usable.  Synchronous: allocates three device words, launches two 32-thread
+ * blocks on `stream`, waits for them and frees the words.  MOE_EINVAL for another `which`
+ * or a NULL `flags`; MOE_ECUDA if a CUDA call fails.
  */
 MOE_API moe_status moe_wait_selftest(int32_t which, void *stream, uint32_t *flags);
 

@@ -375,8 +375,8 @@ def moe_dispatch_combine(x: torch.Tensor, dispatch_plan: Plan, recv: torch.Tenso
 
 def moe_wait_selftest(which: int, stream=None) -> int:
     """Run one bounded device wait on something that never completes (0: ready flag,
-    1: mbarrier) and return the error word it leaves (ERR_TIMEOUT when the wait gave up).
-    Blocks for about a second."""
+    1: mbarrier, 2: grid barrier) and return the error word it leaves (ERR_TIMEOUT when the
+    wait gave up).  Blocks for about a second."""
     flags = ctypes.c_uint32(0)
     _check(_lib.moe_wait_selftest(which, _vp(_stream_ptr(stream)), ctypes.byref(flags)))
     return flags.value

@@ -562,8 +562,10 @@ moe_status moe_wait_selftest(int32_t which, void *stream, uint32_t *flags)
 {
     if (!flags)
         return fail(MOE_EINVAL, "flags must not be NULL");
-    if (which != 0 && which != 1)
-        return fail(MOE_EINVAL, "which must be 0 (flag wait) or 1 (mbarrier wait), got %d", which);
+    if (which < 0 || which > 2)
+        return fail(MOE_EINVAL,
+                    "which must be 0 (flag wait), 1 (mbarrier wait) or 2 (grid barrier), got %d",
+                    which);
     cudaError_t e = moe::run_wait_selftest(which, static_cast<cudaStream_t>(stream), flags);
     if (e != cudaSuccess)
         return cuda_fail(e, "wait self-test");

@@ -204,6 +204,39 @@ __device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t *a)
     return v;
 }
 
+// Sense-reversing grid barrier for a co-resident grid.  sync[0] counts arrivals; the last
+// CTA to arrive sets it back to 0 and advances the generation word sync[1], which the
+// others wait on, so the words are ready for the next barrier (and the next launch) with no
+// extra step.  A wait gives up after kWaitLimitNs, sets MOE_ERR_TIMEOUT and returns false.
+// All threads must call.
+// `gen` is the generation read (by thread 0) before this CTA's phase began: it cannot
+// advance until this CTA arrives, and reading it early takes a round trip off the barrier.
+__device__ __forceinline__ bool grid_barrier(uint32_t *sync, uint32_t *err, uint32_t gen, int *s_ok)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        bool ok = true;
+        if (atom_add_acq_rel_gpu(&sync[0], 1u) == gridDim.x - 1u) {
+            sync[0] = 0u;                // no CTA reads the count until the next barrier
+            st_release_gpu(&sync[1], gen + 1u);
+        } else {
+            const uint64_t t0 = global_timer_ns();
+            for (uint32_t it = 0; ld_acquire_gpu(&sync[1]) == gen; ++it) {
+                if ((it & 15u) == 15u &&
+                    (global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30))) {
+                    atomicOr(err, MOE_ERR_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+                __nanosleep(32);
+            }
+        }
+        *s_ok = ok;
+    }
+    __syncthreads();
+    return *s_ok != 0;
+}
+
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 

@@ -443,38 +443,6 @@ __global__ void __launch_bounds__(kPlanThreads) plan_rank_kernel(const PlanK p)
 }
 
 // ----------------------------------------------------------- fused (cooperative)
-// Sense-reversing grid barrier for a co-resident grid.  sync[0] counts arrivals; the last
-// CTA to arrive sets it back to 0 and advances the generation word sync[1], which the
-// others wait on, so the words are ready for the next barrier (and the next launch) with no
-// extra step.  A wait gives up after kWaitLimitNs, sets MOE_ERR_TIMEOUT and returns false.
-// All threads must call.
-// `gen` is the generation read (by thread 0) before this CTA's phase began: it cannot
-// advance until this CTA arrives, and reading it early takes a round trip off the barrier.
-__device__ bool grid_barrier(const PlanK &p, uint32_t gen, int *s_ok)
-{
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        bool ok = true;
-        if (atom_add_acq_rel_gpu(&p.sync[0], 1u) == gridDim.x - 1u) {
-            p.sync[0] = 0u;                // no CTA reads the count until the next barrier
-            st_release_gpu(&p.sync[1], gen + 1u);
-        } else {
-            const uint64_t t0 = global_timer_ns();
-            for (uint32_t it = 0; ld_acquire_gpu(&p.sync[1]) == gen; ++it) {
-                if ((it & 15u) == 15u &&
-                    (global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30))) {
-                    atomicOr(p.err, MOE_ERR_TIMEOUT);
-                    ok = false;
-                    break;
-                }
-                __nanosleep(32);
-            }
-        }
-        *s_ok = ok;
-    }
-    __syncthreads();
-    return *s_ok != 0;
-}
 
 __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
 {
@@ -490,7 +458,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
     init_rank_of(p, m);
     for (int tile = blockIdx.x; tile < p.nt; tile += G)
         count_tile(p, m, tile, &s_err);
-    if (!grid_barrier(p, gen, &s_ok))
+    if (!grid_barrier(p.sync, p.err, gen, &s_ok))
         return;
     gen += 1u;  // the generation the next barrier starts from
 
@@ -543,7 +511,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
         if (lane == 0)
             *p.err = f;
     }
-    if (!grid_barrier(p, gen, &s_ok))
+    if (!grid_barrier(p.sync, p.err, gen, &s_ok))
         return;
 
     rank_prepare(p, m, warp_sums);

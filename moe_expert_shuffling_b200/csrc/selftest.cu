@@ -13,9 +13,19 @@ namespace {
 // which = 0: the ready-flag wait of the fused kernel, on a flag nothing sets.
 // which = 1: the mbarrier wait of the copy pipelines, on a barrier that expects two
 //            arrivals and gets one (no copy is in flight).
-__global__ void wait_selftest_kernel(const uint32_t *never_set, uint32_t *err, int which)
+// which = 2: the plan's grid barrier, in a grid of two CTAs of which only CTA 0 arrives.
+__global__ void wait_selftest_kernel(uint32_t *words, uint32_t *err, int which)
 {
     __shared__ uint64_t bar;
+    __shared__ int s_ok;
+    const uint32_t *never_set = words;
+    if (which == 2) {
+        if (blockIdx.x == 0)
+            (void)grid_barrier(words, err, 0u, &s_ok);  // words[0..1]: count, generation
+        return;
+    }
+    if (blockIdx.x != 0)
+        return;
     if (which == 0) {
         if (threadIdx.x == 0 && !wait_flag(never_set, 1u, err))
             atomicOr(err, MOE_ERR_TIMEOUT);
@@ -37,17 +47,18 @@ __global__ void wait_selftest_kernel(const uint32_t *never_set, uint32_t *err, i
 
 cudaError_t run_wait_selftest(int which, cudaStream_t stream, uint32_t *flags)
 {
-    uint32_t *words = nullptr;  // [0]: the flag nothing sets, [1]: the error word
-    cudaError_t e = cudaMalloc(&words, 2 * sizeof(uint32_t));
+    // [0..1]: the flag nothing sets / the barrier's count and generation, [2]: error word
+    uint32_t *words = nullptr;
+    cudaError_t e = cudaMalloc(&words, 3 * sizeof(uint32_t));
     if (e != cudaSuccess)
         return e;
-    e = cudaMemsetAsync(words, 0, 2 * sizeof(uint32_t), stream);
+    e = cudaMemsetAsync(words, 0, 3 * sizeof(uint32_t), stream);
     if (e == cudaSuccess) {
-        wait_selftest_kernel<<<1, 32, 0, stream>>>(words, words + 1, which);
+        wait_selftest_kernel<<<2, 32, 0, stream>>>(words, words + 2, which);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess)
-        e = cudaMemcpyAsync(flags, words + 1, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream);
+        e = cudaMemcpyAsync(flags, words + 2, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess)
         e = cudaStreamSynchronize(stream);
     const cudaError_t f = cudaFree(words);

@@ -16,7 +16,7 @@ from workloads import CONFIGS
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("which", [0, 1], ids=["ready_flag", "mbarrier"])
+@pytest.mark.parametrize("which", [0, 1, 2], ids=["ready_flag", "mbarrier", "grid_barrier"])
 def test_wait_gives_up_and_reports_timeout(which):
     import moe_expert_shuffling_b200 as ms
     torch.cuda.synchronize()
