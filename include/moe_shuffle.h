@@ -223,6 +223,10 @@ MOE_API moe_status moe_combine_ranked(const void *y, int32_t H, moe_plan_t plan,
  * ready flags in the plan; no other synchronisation is needed).  Otherwise y and recv must
  * not overlap (MOE_EINVAL).
  *
+ * Calls moving less than MOE_TUNE_FUSED_MIN_KB of payload (320 MB by default; below it the
+ * one-launch kernel's start-up outweighs the overlap) run the dispatch and combine kernels
+ * one after the other on `stream` instead, with the same results.
+ *
  * Arguments are those of moe_dispatch and moe_combine.  fp8 rows need H_x % 512 == 0 (scale
  * rows of a multiple of 16 bytes).  The launch is cooperative; calls that use the same
  * dispatch_plan must be ordered on the GPU (one stream, or events): the plan holds the
@@ -290,7 +294,10 @@ typedef enum {
     MOE_TUNE_FUSED_DISPATCH_SHARE = 13,  /* moe_dispatch_combine: % of CTAs that start on dispatch */
     MOE_TUNE_FUSED_DISPATCH_RUN = 14,    /* moe_dispatch_combine: tokens per dispatch work item (1..32) */
     MOE_TUNE_FUSED_COMBINE_RUN = 15,     /* moe_dispatch_combine: tokens per combine work item */
-    MOE_TUNE_FUSED_SMEM_KB = 16          /* moe_dispatch_combine: shared memory per CTA (KB) */
+    MOE_TUNE_FUSED_SMEM_KB = 16,         /* moe_dispatch_combine: shared memory per CTA (KB) */
+    MOE_TUNE_FUSED_MIN_KB = 17           /* moe_dispatch_combine: least traffic (KB) for the
+                                            one-launch kernel; smaller calls run the two
+                                            kernels back to back (default 327680 = 320 MB) */
 } moe_knob;
 
 MOE_API moe_status moe_tune(moe_knob knob, int32_t value);

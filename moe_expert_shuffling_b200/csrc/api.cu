@@ -211,6 +211,7 @@ moe_status moe_tune(moe_knob knob, int32_t value)
     case MOE_TUNE_FUSED_DISPATCH_RUN: t.fused_dispatch_run = value; break;
     case MOE_TUNE_FUSED_COMBINE_RUN: t.fused_combine_run = value; break;
     case MOE_TUNE_FUSED_SMEM_KB: t.fused_smem_kb = value; break;
+    case MOE_TUNE_FUSED_MIN_KB: t.fused_min_kb = value; break;
     default: return fail(MOE_EINVAL, "unknown tuning knob %d", static_cast<int>(knob));
     }
     return ok();
@@ -483,12 +484,27 @@ moe_status moe_dispatch_combine(const void *x, moe_dtype dtype, const float *x_s
         return fail(MOE_EINVAL, "y == recv needs one plan, bf16 rows and H_x == H_y");
     if (!depends && f.d.N > 0 && f.c.N > 0 && y0 < r1 && r0 < y1)
         return fail(MOE_EINVAL, "y and recv overlap without being the same buffer");
+    // Small calls: the two kernels back to back (stream order also covers y == recv).
+    // Measured on B200: the one-launch kernel starts to win between 250 and 500 MB.
+    const double traffic_kb =
+        (static_cast<double>(f.d.N) * (f.d.row_bytes + f.d.srow_bytes) * (1 + f.d.k) +
+         static_cast<double>(f.c.N) * f.c.H * 2.0 * (1 + f.c.k)) / 1024.0;
+    const int min_kb = moe::tuning().fused_min_kb > 0 ? moe::tuning().fused_min_kb : 320 * 1024;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (traffic_kb < min_kb) {
+        cudaError_t e = moe::launch_dispatch(f.d, dispatch_plan->device, s);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "dispatch kernel");
+        e = moe::launch_combine(f.c, combine_plan->device, s);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "combine kernel");
+        return ok();
+    }
     f.work = dispatch_plan->work;
     f.ready = dispatch_plan->ready;
     f.ready_len = static_cast<uint32_t>(dispatch_plan->cap);
     f.use_flags = depends;
-    cudaError_t e =
-        moe::launch_fused(f, dispatch_plan->device, static_cast<cudaStream_t>(stream));
+    cudaError_t e = moe::launch_fused(f, dispatch_plan->device, s);
     if (e != cudaSuccess)
         return cuda_fail(e, "fused dispatch/combine kernel");
     return ok();

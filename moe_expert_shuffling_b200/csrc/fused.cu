@@ -19,7 +19,8 @@
 // memory (work[3] + 1, advanced by each launch's last CTA), so a launch replayed from a
 // CUDA graph never sees the flags of an earlier replay as its own.  Dispatch work never
 // waits on combine work and the grid is co-resident (cooperative launch), so every flag a
-// combine waits on is set by a CTA that is running: no wait can deadlock.  Each wait still
+// combine waits on is set by a CTA that is running: no wait can deadlock.  Without flags no
+// CTA waits on another, and the launch is an ordinary one.  Each wait still
 // gives up after the wait limit, or as soon as another CTA reports a timeout, and the
 // error word then carries MOE_ERR_TIMEOUT.
 #include <algorithm>
@@ -297,7 +298,6 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
         return cudaErrorInvalidConfiguration;
     per_sm = std::min(per_sm, tu.fused_ctas_per_sm > 0 ? tu.fused_ctas_per_sm
                                                        : kDefaultCtasPerSm * 4 / CW);
-    const int64_t grid = static_cast<int64_t>(sm_count(device)) * per_sm;
 
     // work items
     const double d_token_bytes = static_cast<double>(a.d.row_bytes + a.d.srow_bytes) * (1 + a.d.k);
@@ -318,6 +318,12 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
     fp.d_items = static_cast<uint32_t>(ceil_div(a.d.N, d_run));
     fp.c_items = static_cast<uint32_t>(ceil_div(a.c.N, c_run));
 
+    // Every CTA the device holds at once, but no more than there are items to take (a
+    // small batch would otherwise pay for hundreds of idle CTAs and their counter traffic).
+    const int64_t items = ceil_div(fp.d_items, d_warps) + static_cast<int64_t>(fp.c_items);
+    const int64_t grid = std::max<int64_t>(
+        2, std::min<int64_t>(static_cast<int64_t>(sm_count(device)) * per_sm, items));
+
     // CTAs that start on dispatch: a share of the grid, at least one when there is
     // dispatch work (the ready flags rely on it) and at least one starting on combine when
     // there is combine work.
@@ -335,6 +341,12 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
     }
     fp.d_first_ctas = static_cast<uint32_t>(d_first);
 
+    // Only the ready-flag waits need every CTA resident at once (cooperative launch); with
+    // no flags no CTA waits on another and an ordinary launch, cheaper to start, is enough.
+    if (!a.use_flags) {
+        kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(fp);
+        return cudaGetLastError();
+    }
     void *args[] = {&fp};
     e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern),
                                     dim3(static_cast<unsigned>(grid)), dim3(threads), args, smem,

@@ -70,6 +70,7 @@ struct Tuning {
     int fused_dispatch_run = 0;    // tokens per dispatch work item
     int fused_combine_run = 0;     // tokens per combine work item
     int fused_smem_kb = 0;
+    int fused_min_kb = 0;          // least traffic for the one-launch kernel
 };
 Tuning &tuning();
 

@@ -15,7 +15,8 @@
 //          token t selects the expert), so no step is sequential.
 // By default the phases run in one cooperative kernel (plan_fused_kernel) whose CTAs
 // meet at two sense-reversing grid barriers; a wait gives up after 1 s and reports
-// MOE_ERR_TIMEOUT.
+// MOE_ERR_TIMEOUT.  A routing of at most one tile (N <= 128, e.g. a decode step) runs
+// all phases in one CTA (plan_one_tile_kernel).
 // When the grid cannot be co-resident the phases run as three kernels instead.
 //
 // Inside a tile a warp looks at several tokens at once: lane = (token, column) with the
@@ -284,6 +285,10 @@ __device__ void count_tile(const PlanK &p, const PlanSmem &m, int tile, uint32_t
 // Segment sizes are the counts rounded up to the alignment.  Also marks every receive
 // row that no entry maps to (segment padding and rows after the last segment) with -1
 // in src_tok/src_j, spread over all CTAs of the grid.
+// Segment offsets from m.ebase (segment sizes) and m.rbase (rank counts), which the caller
+// has filled; the rest as rank_prepare.
+__device__ void prepare_offsets(const PlanK &p, const PlanSmem &m, int32_t *warp_sums);
+
 __device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_sums)
 {
     for (int i = threadIdx.x; i < p.E + p.R; i += blockDim.x) {
@@ -294,6 +299,11 @@ __device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_su
             m.rbase[i - p.E] = __ldcg(p.rcnt + (i - p.E));
         }
     }
+    prepare_offsets(p, m, warp_sums);
+}
+
+__device__ void prepare_offsets(const PlanK &p, const PlanSmem &m, int32_t *warp_sums)
+{
     __syncthreads();
     scan_into(m.ebase, p.E, m.eoff, warp_sums);
     scan_into(m.rbase, p.R, m.roff, warp_sums);
@@ -322,16 +332,16 @@ __device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_su
     }
 }
 
+__device__ void rank_entries(const PlanK &p, const PlanSmem &m, int tile, int ntok);
+
 // Rank phase for one tile.  All threads must call; rank_prepare must have run.  With
 // tile_ready the tile's classification (count_tile of this tile) is still in shared
 // memory; otherwise it is rebuilt.
 __device__ void rank_tile(const PlanK &p, const PlanSmem &m, int tile, bool tile_ready)
 {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int ntok = tile_tokens(p, tile);
     if (ntok == 0)
         return;  // block-uniform
-    const int k = p.k;
     if (!tile_ready)
         (void)classify_tile(p, m, tile, ntok);  // flags were reported by the count phase
     // This tile's first receive row per expert and first dedup entry per rank.
@@ -340,8 +350,15 @@ __device__ void rank_tile(const PlanK &p, const PlanSmem &m, int tile, bool tile
     for (int r = threadIdx.x; r < p.R; r += blockDim.x)
         m.rbase[r] = m.roff[r] + __ldcg(p.tile_rcnt + static_cast<int64_t>(r) * p.nt + tile);
     __syncthreads();
+    rank_entries(p, m, tile, ntok);
+}
 
-    // Stable rank = tile base + earlier tokens of the tile on the same expert.
+// Stable rank of every entry of a classified tile whose bases m.ebase / m.rbase are set:
+// tile base + earlier tokens of the tile on the same expert.  All threads must call.
+__device__ void rank_entries(const PlanK &p, const PlanSmem &m, int tile, int ntok)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int k = p.k;
     const LaneMap lm = lane_map(k);
     const int j = lane & ((1 << lm.wbits) - 1);
     const int sub = lane >> lm.wbits;
@@ -440,6 +457,48 @@ __global__ void __launch_bounds__(kPlanThreads) plan_rank_kernel(const PlanK p)
     init_rank_of(p, m);
     rank_prepare(p, m, warp_sums);
     rank_tile(p, m, blockIdx.x, false);
+}
+
+// ------------------------------------------------------------- one tile (N <= 128)
+// Every phase in one CTA: the counts are the popcounts of the single tile's masks, so no
+// scratch, no grid barrier and no cooperative launch is needed.
+__global__ void __launch_bounds__(kPlanThreads) plan_one_tile_kernel(const PlanK p)
+{
+    extern __shared__ int32_t smem[];
+    __shared__ uint32_t s_err;
+    __shared__ int32_t warp_sums[kPlanThreads / 32];
+    const PlanSmem m = carve(smem, p.E, p.R, p.k);
+    if (threadIdx.x == 0)
+        s_err = 0;
+    init_rank_of(p, m);
+    const int ntok = tile_tokens(p, 0);
+    const uint32_t flags = classify_tile(p, m, 0, ntok);  // synchronises first
+    if (flags)
+        atomicOr(&s_err, flags);
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+        const uint32_t *mk = &m.emask[4 * e];
+        const int32_t c = __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+        p.cnt[e] = c;
+        m.ebase[e] = (c + p.align - 1) / p.align * p.align;
+    }
+    for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
+        const uint32_t *mk = &m.rmask[4 * r];
+        const int32_t c = __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+        p.rcnt[r] = c;
+        m.rbase[r] = c;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        *p.err = s_err;  // before any MOE_ERR_BOUNDS of the rank step is or-ed in
+    prepare_offsets(p, m, warp_sums);
+    // the tile's bases are the segment starts themselves
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
+        m.ebase[e] = m.eoff[e];
+    for (int r = threadIdx.x; r < p.R; r += blockDim.x)
+        m.rbase[r] = m.roff[r];
+    __syncthreads();
+    if (ntok > 0)  // block-uniform
+        rank_entries(p, m, 0, ntok);
 }
 
 // ----------------------------------------------------------- fused (cooperative)
@@ -552,6 +611,8 @@ bool ensure_attrs(int dev)
         cudaFuncSetAttribute(plan_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              bytes) != cudaSuccess ||
         cudaFuncSetAttribute(plan_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(plan_one_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              bytes) != cudaSuccess)
         return false;
     done[dev] = true;
@@ -591,6 +652,13 @@ cudaError_t launch_plan(moe_plan_s *pl, const int32_t *topk_idx, cudaStream_t st
     p.err = pl->err;
     p.sync = pl->sync;
 
+    if (tuning().plan_engine != 2 && p.nt <= 1) {
+        // A single tile: one ordinary launch of one CTA.
+        const size_t smem = sizeof(int32_t) * plan_smem_words(p.E, p.R, p.k);
+        pl->plan_kernels = 1;
+        plan_one_tile_kernel<<<1, kPlanThreads, smem, stream>>>(p);
+        return cudaGetLastError();
+    }
     if (tuning().plan_engine != 2) {
         // One cooperative launch when the grid fits on the device at once.
         static int coop[64] = {0};
@@ -606,8 +674,12 @@ cudaError_t launch_plan(moe_plan_s *pl, const int32_t *topk_idx, cudaStream_t st
             kernel_fit(reinterpret_cast<const void *>(plan_fused_kernel), pl->device,
                        kPlanThreads, smem, &per_sm) == cudaSuccess &&
             per_sm > 0) {
+            // One CTA per tile, and at least enough CTAs for one warp per expert / rank row
+            // in the scan phase (a few tiles of a wide expert set would otherwise leave each
+            // warp dozens of rows, each one dependent round trip to L2).
             const int64_t fit = static_cast<int64_t>(sm_count(pl->device)) * per_sm;
-            const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(p.nt, fit)));
+            const int64_t want = std::max<int64_t>(p.nt, ceil_div(p.E + p.R, kPlanWarps));
+            const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, fit)));
             void *args[] = {&p};
             pl->plan_kernels = 1;
             return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(plan_fused_kernel),

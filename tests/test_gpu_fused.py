@@ -18,6 +18,16 @@ from workloads import CONFIGS
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True)
+def always_one_launch():
+    """These tests exercise the one-launch kernel at every size (by default calls below
+    320 MB run the two kernels back to back)."""
+    import moe_expert_shuffling_b200 as ms
+    ms.moe_tune("fused_min_kb", 1)
+    yield
+    ms.moe_tune("fused_min_kb", 0)
+
+
 def oracle_recv(cfg, x, xs, ref):
     if cfg.payload == "fp8":
         return oracle.dispatch(x.cpu().numpy(), ref.slot, xs.cpu().numpy(), rows=ref.rows)
@@ -229,3 +239,11 @@ def test_fused_inside_a_cuda_graph():
         torch.cuda.synchronize()
         assert p.check() == 0
         assert np.array_equal(bits16(out), want_out)
+
+
+@pytest.mark.parametrize("identity", [False, True], ids=["y", "recv"])
+def test_small_calls_run_the_two_kernels_with_the_same_results(identity):
+    import moe_expert_shuffling_b200 as ms
+    ms.moe_tune("fused_min_kb", 0)  # the default threshold: this call is below it
+    fused_case(CONFIGS["mixtral"].with_tokens(300), 19, identity=identity, ranked=False)
+    fused_case(CONFIGS["dsv3"].with_tokens(200), 20, identity=identity, ranked=True)

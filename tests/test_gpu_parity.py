@@ -326,3 +326,39 @@ def test_drops_alone_raise_no_error():
     assert not bits16(out).any()              # nothing routed: out is +0
     a = plan_to_host(p)
     assert np.all(a["slot"] == -1) and np.all(a["src_tok"] == -1) and a["cnt"].sum() == 0
+
+
+@pytest.mark.parametrize("cfg,frac,align", [
+    (CONFIGS["dsv3"].with_tokens(128), 0.0, 1),
+    (CONFIGS["dsv3"].with_tokens(16), 0.25, 64),
+    (CONFIGS["dsv3"].replace(N=100, H=64, E=1024, k=8, R=1024), 0.0, 1),
+    (CONFIGS["dsv3"].replace(N=50, H=64, E=64, k=32, R=8), 0.1, 8),
+    (CONFIGS["mixtral"].with_tokens(1), 0.0, 1),
+], ids=lambda v: f"{v.name}-N{v.N}-E{v.E}-k{v.k}" if hasattr(v, "name") else str(v))
+def test_single_tile_plans(cfg, frac, align):
+    """Routings of at most one tile (N <= 128) take the one-CTA plan kernel; its plan,
+    dispatch and combine match the oracle bit for bit."""
+    import moe_expert_shuffling_b200 as ms
+    idx, w, x, _, _ = make_inputs(cfg, 17, y=False)
+    if frac > 0:
+        idx = drop_some(idx, frac, 3)
+    ref = oracle.plan(idx, cfg.E, cfg.R, align=align)
+    p = ms.moe_plan_create(cfg.N, cfg.k, cfg.E, cfg.R, align=align)
+    p, ti, tw = gpu_plan(idx, w, cfg.E, cfg.R, plan=p)
+    assert p.plan_kernels == 1
+    got = plan_to_host(p)
+    for name in ("cnt", "expert_off", "rcnt", "rank_off", "rtok_off", "slot", "src_tok",
+                 "src_j", "rtok"):
+        assert np.array_equal(got[name], getattr(ref, name)), name
+    assert np.array_equal(got["fanout"], ref.fanout)
+    assert int(got["err"][0]) == 0
+    recv = ms.moe_dispatch(x, p)
+    out = ms.moe_combine(recv, p)
+    assert p.check() == 0
+    used = ref.src_tok >= 0
+    want_recv = oracle.dispatch(bits16(x).view(np.uint8).reshape(cfg.N, -1), ref.slot, rows=ref.rows)
+    got_recv = bits16(recv).view(np.uint8).reshape(ref.rows, -1)
+    assert np.array_equal(got_recv[used], want_recv[used])
+    y_bits = want_recv.view(np.uint16).reshape(ref.rows, cfg.H).copy()
+    y_bits[~used] = 0
+    assert np.array_equal(bits16(out), oracle.combine(y_bits, ref.slot, w))
