@@ -618,6 +618,76 @@ def run_micro_batches(args):
     }), flush=True)
 
 
+def run_latency(args):
+    """Latency of one step at small token counts (decode-sized batches): each of plan,
+    dispatch, combine, dispatch+combine in one call, and the whole step, captured in a CUDA
+    graph and replayed (CUDA events around the replays, mean per replay).  One JSON line per
+    token count; not the bench line."""
+    import moe_expert_shuffling_b200 as ms
+    from moe_expert_shuffling_b200 import build as lib_build
+
+    lib_build.build()
+    dev = torch.device("cuda", 0)
+    s = torch.cuda.Stream(device=dev)
+
+    def replay_us(fn, iters):
+        with torch.cuda.stream(s):
+            for _ in range(args.warmup):
+                fn()
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            g.replay()
+            a.record(s)
+            for _ in range(iters):
+                g.replay()
+            b.record(s)
+        b.synchronize()
+        return round(1e3 * a.elapsed_time(b) / iters, 2)
+
+    for N in (int(v) for v in args.latency.split(",")):
+        cfg = CONFIGS[args.config].with_tokens(N)
+        idx_h, w_h = make_routing(cfg, args.seed)
+        with torch.cuda.stream(s):
+            x, xs = make_payload_x(cfg, args.seed, dev)
+            y = make_payload_y(cfg.replace(y="normal"), args.seed, dev)
+            idx = torch.from_numpy(idx_h).to(dev)
+            w = torch.from_numpy(w_h).to(dev)
+            plan = ms.moe_plan_create(N, cfg.k, cfg.E, cfg.R)
+            ms.moe_plan(idx, w, cfg.E, cfg.R, plan=plan, stream=s)
+            recv = torch.empty((plan.rows, cfg.H), dtype=x.dtype, device=dev)
+            rs = (torch.empty((plan.rows, cfg.H // 128), dtype=torch.float32, device=dev)
+                  if cfg.payload == "fp8" else None)
+            out = torch.empty((N, cfg.H), dtype=torch.bfloat16, device=dev)
+        s.synchronize()
+        kw = dict(x_scale=xs, recv_scale=rs) if cfg.payload == "fp8" else {}
+
+        def pl():
+            ms.moe_plan(idx, w, cfg.E, cfg.R, plan=plan, stream=s)
+
+        def dp():
+            ms.moe_dispatch(x, plan, recv=recv, stream=s, **kw)
+
+        def cb():
+            ms.moe_combine(y, plan, out=out, stream=s)
+
+        def dc():
+            ms.moe_dispatch_combine(x, plan, recv, y, plan, out=out, stream=s, **kw)
+
+        res = {"workload": workload_name(cfg), "tokens": N, "unit": "us",
+               "plan": replay_us(pl, args.steps), "dispatch": replay_us(dp, args.steps),
+               "combine": replay_us(cb, args.steps), "dispatch_combine": replay_us(dc, args.steps),
+               "step": replay_us(lambda: (pl(), dp(), cb()), args.steps),
+               "plan_kernels": plan.plan_kernels}
+        if plan.check(s) != 0:
+            raise SystemExit("device reported invalid routing or a timeout")
+        plan.close()
+        print(json.dumps(res), flush=True)
+
+
 # ------------------------------------------------------------------------ CPU oracle
 def oracle_sample_step(cfg: Config, idx_h, w_h, x_bytes, xs_bytes, y_bits, n):
     """One oracle plan + dispatch + combine over the first n tokens of the workload."""
@@ -767,11 +837,16 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0)
+    ap.add_argument("--latency", default="",
+                    help="comma-separated token counts: print per-step latencies of the "
+                         "workload's shape at each (small batches) instead of the bench line")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.latency:
+        run_latency(args)
     elif args.micro_batches > 1:
         run_micro_batches(args)
     else:

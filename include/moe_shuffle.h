@@ -295,9 +295,11 @@ typedef enum {
     MOE_TUNE_FUSED_DISPATCH_RUN = 14,    /* moe_dispatch_combine: tokens per dispatch work item (1..32) */
     MOE_TUNE_FUSED_COMBINE_RUN = 15,     /* moe_dispatch_combine: tokens per combine work item */
     MOE_TUNE_FUSED_SMEM_KB = 16,         /* moe_dispatch_combine: shared memory per CTA (KB) */
-    MOE_TUNE_FUSED_MIN_KB = 17           /* moe_dispatch_combine: least traffic (KB) for the
+    MOE_TUNE_FUSED_MIN_KB = 17,          /* moe_dispatch_combine: least traffic (KB) for the
                                             one-launch kernel; smaller calls run the two
                                             kernels back to back (default 327680 = 320 MB) */
+    MOE_TUNE_COMBINE_MAX_CW = 18         /* bulk combine: most consumer warps per CTA (4 or 8;
+                                            default 8: k <= 4 uses 8, wider k uses 4 or fewer) */
 } moe_knob;
 
 MOE_API moe_status moe_tune(moe_knob knob, int32_t value);

@@ -37,7 +37,7 @@ KNOBS = {
     "combine_stages": 6, "combine_engine": 7, "combine_smem_kb": 8,
     "dispatch_units_per_warp": 9, "combine_tokens_per_cta": 10, "plan_engine": 11,
     "fused_ctas_per_sm": 12, "fused_dispatch_share": 13, "fused_dispatch_run": 14,
-    "fused_combine_run": 15, "fused_smem_kb": 16, "fused_min_kb": 17,
+    "fused_combine_run": 15, "fused_smem_kb": 16, "fused_min_kb": 17, "combine_max_cw": 18,
 }
 
 _i32 = ctypes.c_int32

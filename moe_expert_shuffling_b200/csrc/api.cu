@@ -212,6 +212,7 @@ moe_status moe_tune(moe_knob knob, int32_t value)
     case MOE_TUNE_FUSED_COMBINE_RUN: t.fused_combine_run = value; break;
     case MOE_TUNE_FUSED_SMEM_KB: t.fused_smem_kb = value; break;
     case MOE_TUNE_FUSED_MIN_KB: t.fused_min_kb = value; break;
+    case MOE_TUNE_COMBINE_MAX_CW: t.combine_max_cw = value; break;
     default: return fail(MOE_EINVAL, "unknown tuning knob %d", static_cast<int>(knob));
     }
     return ok();

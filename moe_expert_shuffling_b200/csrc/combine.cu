@@ -101,13 +101,14 @@ __global__ void __launch_bounds__(kCombineThreads) combine_lsu_kernel(const Comb
 // ------------------------------------------------------------------ bulk engine
 // Measured on B200 (dsv3 and long shapes): a ring of 32-36 KB per CTA, 3 CTAs per SM and
 // short runs of 4 tokens per CTA (the block scheduler evens out the tail) are fastest;
-// deeper rings, more CTAs per SM and persistent CTAs are slower.
+// deeper rings, more CTAs per SM and persistent CTAs are slower.  The wide shape for
+// k <= 4 (Mixtral) is fastest with runs of 8 tokens.
 constexpr int kDefaultSmemBudget = 36 * 1024 + 128;
 constexpr int kDefaultCtasPerSm = 3;
 constexpr int kDefaultTokensPerCta = 4;
 
 template <int KMAX, int CW, bool RANKED>
-__global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
+__global__ void __launch_bounds__(Shape<CW>::kThreads, CW >= 8 ? 2 : 1)
     combine_bulk_kernel(const CombineBulkParams p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -226,12 +227,12 @@ cudaError_t launch_bulk_shape(const CombineArgs &a, int device, cudaStream_t str
         return cudaErrorInvalidConfiguration;
     // the default keeps about 12 consumer warps per SM whatever the chunk width
     per_sm = std::min(per_sm, tu.combine_ctas_per_sm > 0 ? tu.combine_ctas_per_sm
-                                                          : kDefaultCtasPerSm * 4 / CW);
+                                                          : std::max(1, kDefaultCtasPerSm * 4 / CW));
     // Contiguous runs of tokens per CTA; the grid covers all tokens so that CTAs that
     // finish early are replaced by the block scheduler.
     const int64_t resident = static_cast<int64_t>(sm_count(device)) * per_sm;
     int64_t per_cta = tu.combine_tokens_per_cta > 0 ? tu.combine_tokens_per_cta
-                                                    : kDefaultTokensPerCta;
+                                                    : (CW >= 8 ? 2 : 1) * kDefaultTokensPerCta;
     if (ceil_div(a.N, per_cta) < resident)
         per_cta = std::max<int64_t>(1, ceil_div(a.N, resident));
     p.per_cta = static_cast<uint32_t>(per_cta);
@@ -243,6 +244,13 @@ cudaError_t launch_bulk_shape(const CombineArgs &a, int device, cudaStream_t str
 template <bool RANKED>
 cudaError_t launch_combine_bulk(const CombineArgs &a, int device, cudaStream_t stream)
 {
+    // Chunks widen for k <= 4 (8 consumer warps, 4 KB per row) so that a stage is not a
+    // couple of 2 KB rows with a barrier round each.  Measured on B200 at the Mixtral
+    // shape (k = 2): 35.6 us against 49.7 us with 4 consumer warps; 16 consumer warps
+    // (8 KB per row) were slower than 8.
+    const int max_cw = tuning().combine_max_cw > 0 ? tuning().combine_max_cw : 8;
+    if (a.k <= 4 && max_cw >= 8)
+        return launch_bulk_shape<4, 8, RANKED>(a, device, stream);
     if (a.k <= 8)
         return launch_bulk_shape<8, 4, RANKED>(a, device, stream);
     if (a.k <= 16)

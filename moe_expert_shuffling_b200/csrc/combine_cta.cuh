@@ -46,8 +46,9 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float *acc)
 }
 
 // A unit covers CW * 512 bytes of each of the token's k rows: one 16-byte vector per
-// consumer thread, CW consumer warps.  Wider k gets narrower chunks so that a stage
-// (k x chunk) stays at 16 KB: CW = 4 for k <= 8, 2 for k <= 16, 1 for k <= 32.
+// consumer thread, CW consumer warps.  The chunk narrows as k grows so that a stage
+// (k x chunk) stays at 16 KB or less: CW = 8 for k <= 4, 4 for k <= 8, 2 for k <= 16,
+// 1 for k <= 32.
 template <int CW>
 struct Shape {
     static constexpr uint32_t kChunk = 512u * CW;
@@ -229,6 +230,7 @@ __device__ __forceinline__ bool combine_consume(const CombineBulkParams &p, cons
                                                 float w_nxt, int &i)
 {
     constexpr uint32_t kChunk_ = Shape<CW>::kChunk;
+    constexpr int kJ = KMAX < 8 ? KMAX : 8;  // rows held in registers at once
     const int lane = threadIdx.x & 31;
     const int k = p.k;
     const int S = r.S;
@@ -287,25 +289,25 @@ __device__ __forceinline__ bool combine_consume(const CombineBulkParams &p, cons
                 part[e] = 0.f;
             }
 #pragma unroll
-            for (int j0 = 0; j0 < KMAX; j0 += 8) {
+            for (int j0 = 0; j0 < KMAX; j0 += kJ) {
                 if (j0 >= k)
                     break;  // warp-uniform
-                uint4 q[8];
+                uint4 q[kJ];
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
+                for (int jj = 0; jj < kJ; ++jj) {
                     const int j = j0 + jj;
                     const bool kept = RANKED ? static_cast<uint32_t>(j) < nv : ((vmask >> j) & 1u);
                     q[jj] = (mine && kept) ? lds_v4(stage + j * kChunk_)
                                            : make_uint4(0u, 0u, 0u, 0u);
                 }
-                if (j0 + 8 >= k) {
+                if (j0 + kJ >= k) {
                     // every row of this stage is in registers: release it to the producer
                     __syncwarp();
                     if (lane == 0)
                         mbar_arrive(&r.empty[st]);
                 }
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
+                for (int jj = 0; jj < kJ; ++jj) {
                     const int j = j0 + jj;
                     if (RANKED) {
                         if (static_cast<uint32_t>(j) >= nv)

@@ -71,6 +71,7 @@ struct Tuning {
     int fused_combine_run = 0;     // tokens per combine work item
     int fused_smem_kb = 0;
     int fused_min_kb = 0;          // least traffic for the one-launch kernel
+    int combine_max_cw = 0;        // cap on consumer warps per combine CTA (4, 8 or 16)
 };
 Tuning &tuning();
 

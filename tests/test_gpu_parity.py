@@ -362,3 +362,31 @@ def test_single_tile_plans(cfg, frac, align):
     y_bits = want_recv.view(np.uint16).reshape(ref.rows, cfg.H).copy()
     y_bits[~used] = 0
     assert np.array_equal(bits16(out), oracle.combine(y_bits, ref.slot, w))
+
+
+@pytest.mark.parametrize("knobs", [{"combine_max_cw": 4}, {"combine_max_cw": 8},
+                                   {"combine_tokens_per_cta": 1}],
+                         ids=["4-warps", "8-warps", "1-token-runs"])
+@pytest.mark.parametrize("cfg", [CONFIGS["mixtral"].with_tokens(1500),
+                                 CONFIGS["long"].replace(N=900, H=512, k=4, E=16, R=16),
+                                 CONFIGS["tiny"].replace(k=3, N=333)],
+                         ids=lambda c: f"{c.name}-k{c.k}")
+def test_small_k_combine_shapes(cfg, knobs):
+    """k <= 4 combines with 8 consumer warps (4 KB per row) by default; both chunk widths
+    and both orders match the oracle bit for bit."""
+    import moe_expert_shuffling_b200 as ms
+    idx, w, x, xs, y = make_inputs(cfg, 23)
+    ref = oracle.plan(idx, cfg.E, cfg.R)
+    try:
+        for k, v in knobs.items():
+            ms.moe_tune(k, v)
+        p, ti, tw = gpu_plan(idx, w, cfg.E, cfg.R)
+        out = ms.moe_combine(y, p)
+        out_r = ms.moe_combine(y, p, ranked=True)
+        assert p.check() == 0
+    finally:
+        for k in knobs:
+            ms.moe_tune(k, 0)
+    yb = bits16(y)
+    assert np.array_equal(bits16(out), oracle.combine(yb, ref.slot, w))
+    assert np.array_equal(bits16(out_r), oracle.combine_ranked(yb, ref.slot, w, idx, cfg.E, cfg.R))
