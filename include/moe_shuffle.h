@@ -132,8 +132,9 @@ MOE_API moe_status moe_plan_create_aligned(int32_t max_tokens, int32_t k, int32_
  *   rtok/fanout = the tokens of rank r in ascending order with the mask of their
  *   columns on r -- one move per (token, rank) pair.
  * Deterministic (no result depends on thread timing).  Enqueues one kernel: a single
- * block for N <= 128 (one tile), else one cooperative kernel (three kernels where its grid
- * cannot be co-resident).
+ * block for N <= 128 (one tile), one thread-block cluster of one block per 128 tokens for
+ * N <= 2048, else one cooperative kernel (three kernels where its grid cannot be
+ * co-resident).
  */
 MOE_API moe_status moe_plan(const int32_t *topk_idx, const float *topk_w, int32_t N, int32_t k,
                     int32_t E, int32_t R, void *stream, moe_plan_t *plan);

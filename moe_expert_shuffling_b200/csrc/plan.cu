@@ -16,13 +16,17 @@
 // By default the phases run in one cooperative kernel (plan_fused_kernel) whose CTAs
 // meet at two sense-reversing grid barriers; a wait gives up after 1 s and reports
 // MOE_ERR_TIMEOUT.  A routing of at most one tile (N <= 128, e.g. a decode step) runs
-// all phases in one CTA (plan_one_tile_kernel).
+// all phases in one CTA (plan_one_tile_kernel), and one of 2..16 tiles on one thread-block
+// cluster with the tile counts shared through distributed shared memory
+// (plan_cluster_kernel).
 // When the grid cannot be co-resident the phases run as three kernels instead.
 //
 // Inside a tile a warp looks at several tokens at once: lane = (token, column) with the
 // columns of one token in a segment of W = next power of two >= k lanes, so a token's
 // k ids are compared with width-W shuffles.
 #include <algorithm>
+
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 #include "internal.cuh"
@@ -501,6 +505,85 @@ __global__ void __launch_bounds__(kPlanThreads) plan_one_tile_kernel(const PlanK
         rank_entries(p, m, 0, ntok);
 }
 
+// ------------------------------------------- a few tiles on one thread-block cluster
+// Routings of 2..kClusterTiles tiles: one CTA per tile in one cluster.  Each CTA counts its
+// tile; after the cluster barrier every CTA reads all tiles' counts from the other CTAs'
+// shared memory (distributed shared memory) to get its tile base and the totals.  The
+// cluster's hardware barrier replaces the grid barriers, and no global scratch is used.
+// Every CTA takes the same two barriers whatever its data.  Up to 16 tiles: clusters of
+// more than 8 CTAs are opted into (non-portable size, which sm_100 supports); the launch
+// falls back to the cooperative kernel when such a cluster cannot be resident.
+constexpr int kClusterTiles = 16;
+
+__host__ __device__ constexpr size_t plan_cluster_smem_words(int E, int R, int k)
+{
+    return plan_smem_words(E, R, k) + 2 * static_cast<size_t>(E + R);
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_cluster_kernel(const PlanK p)
+{
+    namespace cg = cooperative_groups;
+    extern __shared__ int32_t smem[];
+    __shared__ uint32_t s_err;
+    __shared__ int32_t warp_sums[kPlanThreads / 32];
+    cg::cluster_group cluster = cg::this_cluster();
+    const PlanSmem m = carve(smem, p.E, p.R, p.k);
+    int32_t *tc = reinterpret_cast<int32_t *>(m.lead + kPlanTile * p.k);  // [E+R] tile counts
+    int32_t *tb = tc + (p.E + p.R);                                       // [E+R] tile bases
+    const int tile = static_cast<int>(cluster.block_rank());  // the grid is one cluster
+    const int C = static_cast<int>(cluster.num_blocks());
+    const int ntok = tile_tokens(p, tile);
+    if (threadIdx.x == 0)
+        s_err = 0;
+    init_rank_of(p, m);
+    const uint32_t flags = classify_tile(p, m, tile, ntok);  // synchronises first
+    if (flags)
+        atomicOr(&s_err, flags);
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+        const uint32_t *mk = &m.emask[4 * e];
+        tc[e] = __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+    }
+    for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
+        const uint32_t *mk = &m.rmask[4 * r];
+        tc[p.E + r] = __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+    }
+    cluster.sync();  // every tile's counts and flags are visible to the cluster
+
+    // this tile's base (earlier tiles) and the total of every expert / rank row
+    for (int row = threadIdx.x; row < p.E + p.R; row += blockDim.x) {
+        int32_t before = 0, total = 0;
+        for (int c = 0; c < C; ++c) {
+            const int32_t v = cluster.map_shared_rank(tc, c)[row];
+            before += c < tile ? v : 0;
+            total += v;
+        }
+        tb[row] = before;
+        // every CTA writes the same totals, so each reads back its own writes below
+        if (row < p.E) {
+            p.cnt[row] = total;
+            m.ebase[row] = (total + p.align - 1) / p.align * p.align;
+        } else {
+            p.rcnt[row - p.E] = total;
+            m.rbase[row - p.E] = total;
+        }
+    }
+    if (tile == 0 && threadIdx.x == 0) {
+        uint32_t f = 0;
+        for (int c = 0; c < C; ++c)
+            f |= *cluster.map_shared_rank(&s_err, c);
+        *p.err = f;  // before any MOE_ERR_BOUNDS of the rank step is or-ed in
+    }
+    cluster.sync();  // no shared memory is read across the cluster after this point
+
+    prepare_offsets(p, m, warp_sums);
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
+        m.ebase[e] = m.eoff[e] + tb[e];
+    for (int r = threadIdx.x; r < p.R; r += blockDim.x)
+        m.rbase[r] = m.roff[r] + tb[p.E + r];
+    __syncthreads();
+    rank_entries(p, m, tile, ntok);
+}
+
 // ----------------------------------------------------------- fused (cooperative)
 
 __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
@@ -631,6 +714,32 @@ cudaError_t launch_three(const PlanK &p, cudaStream_t stream)
 
 }  // namespace
 
+// Whether a cluster of `nt` plan CTAs with `smem` bytes each can be resident (cached: the
+// answer depends only on these and the device).
+bool cluster_fits(int nt, size_t smem, int device, const cudaLaunchConfig_t *cfg, int *clusters)
+{
+    struct Fit {
+        int nt, device;
+        size_t smem;
+        int clusters;
+    };
+    static Fit cache[64];
+    static int n_cache = 0;
+    for (int i = 0; i < n_cache; ++i)
+        if (cache[i].nt == nt && cache[i].device == device && cache[i].smem == smem) {
+            *clusters = cache[i].clusters;
+            return true;
+        }
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, reinterpret_cast<const void *>(plan_cluster_kernel),
+                                       cfg) != cudaSuccess)
+        return false;
+    if (n_cache < 64)
+        cache[n_cache++] = {nt, device, smem, c};
+    *clusters = c;
+    return true;
+}
+
 cudaError_t launch_plan(moe_plan_s *pl, const int32_t *topk_idx, cudaStream_t stream)
 {
     if (!ensure_attrs(pl->device))
@@ -658,6 +767,41 @@ cudaError_t launch_plan(moe_plan_s *pl, const int32_t *topk_idx, cudaStream_t st
         pl->plan_kernels = 1;
         plan_one_tile_kernel<<<1, kPlanThreads, smem, stream>>>(p);
         return cudaGetLastError();
+    }
+    if (tuning().plan_engine != 2 && p.nt <= kClusterTiles) {
+        // A few tiles: one cluster of one CTA per tile, when such a cluster can be resident.
+        const size_t smem = sizeof(int32_t) * plan_cluster_smem_words(p.E, p.R, p.k);
+        int per_sm = 0;
+        static int non_portable[64] = {0};
+        const int dv = pl->device >= 0 && pl->device < 64 ? pl->device : 0;
+        if (non_portable[dv] == 0)
+            non_portable[dv] = cudaFuncSetAttribute(plan_cluster_kernel,
+                                                    cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                                    1) == cudaSuccess ? 1 : -1;
+        if ((p.nt <= 8 || non_portable[dv] > 0) &&
+            smem <= static_cast<size_t>(max_smem_optin(pl->device)) &&
+            kernel_fit(reinterpret_cast<const void *>(plan_cluster_kernel), pl->device,
+                       kPlanThreads, smem, &per_sm) == cudaSuccess &&
+            per_sm > 0) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(static_cast<unsigned>(p.nt));
+            cfg.blockDim = dim3(kPlanThreads);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = static_cast<unsigned>(p.nt);
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            if (cluster_fits(p.nt, smem, pl->device, &cfg, &clusters) && clusters > 0) {
+                pl->plan_kernels = 1;
+                return cudaLaunchKernelEx(&cfg, plan_cluster_kernel, p);
+            }
+        }
+        (void)cudaGetLastError();
     }
     if (tuning().plan_engine != 2) {
         // One cooperative launch when the grid fits on the device at once.

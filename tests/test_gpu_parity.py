@@ -334,7 +334,9 @@ def test_drops_alone_raise_no_error():
     (CONFIGS["dsv3"].replace(N=100, H=64, E=1024, k=8, R=1024), 0.0, 1),
     (CONFIGS["dsv3"].replace(N=50, H=64, E=64, k=32, R=8), 0.1, 8),
     (CONFIGS["mixtral"].with_tokens(1), 0.0, 1),
-    # a few tiles: the cooperative kernel with its grid floor of one warp per row
+    # 2..16 tiles: one thread-block cluster, tile counts through distributed shared memory
+    (CONFIGS["dsv3"].with_tokens(2048), 0.1, 8),
+    (CONFIGS["dsv3"].with_tokens(1100), 0.0, 1),
     (CONFIGS["dsv3"].with_tokens(129), 0.0, 1),
     (CONFIGS["dsv3"].with_tokens(1024), 0.0, 1),
     (CONFIGS["dsv3"].with_tokens(700), 0.2, 16),
@@ -344,9 +346,9 @@ def test_drops_alone_raise_no_error():
     (CONFIGS["tiny"].replace(k=1, N=1000), 0.0, 1),
 ], ids=lambda v: f"{v.name}-N{v.N}-E{v.E}-k{v.k}" if hasattr(v, "name") else str(v))
 def test_single_tile_plans(cfg, frac, align):
-    """Routings of at most one tile (N <= 128) take the one-CTA plan kernel, a few tiles the
-    cooperative kernel on its minimum grid; their plan, dispatch and combine match the
-    oracle bit for bit."""
+    """Routings of at most one tile (N <= 128) take the one-CTA plan kernel, and those of
+    2..16 tiles the one-cluster kernel; their plan, dispatch and combine match the oracle bit
+    for bit."""
     import moe_expert_shuffling_b200 as ms
     idx, w, x, _, _ = make_inputs(cfg, 17, y=False)
     if frac > 0:
