@@ -117,3 +117,21 @@ def test_product_has_no_oracle_dependency():
     out = subprocess.run(["ldd", os.path.join(pkg, "libmoeshuffle.so")], capture_output=True,
                          text=True).stdout
     assert "oracle" not in out
+
+
+def test_python_knobs_match_the_header(lib):
+    """Every MOE_TUNE_* value in the header is a knob of the binding under the same name and
+    number, and the library accepts each of them."""
+    import moe_expert_shuffling_b200 as ms
+    text = open(os.path.join(ROOT, "include", "moe_shuffle.h")).read()
+    header = {m.group(1).lower(): int(m.group(2))
+              for m in re.finditer(r"MOE_TUNE_([A-Z0-9_]+)\s*=\s*(\d+)", text)}
+    assert header == ms.KNOBS
+    for value in header.values():
+        assert lib.moe_tune(value, 0) == 0
+
+
+def test_wait_selftest_rejects_unknown_wait_on_host(lib):
+    flags = ctypes.c_uint32(0)
+    assert lib.moe_wait_selftest(7, None, ctypes.byref(flags)) == 1
+    assert lib.moe_wait_selftest(0, None, None) == 1
