@@ -413,6 +413,14 @@ def run_ours(args):
     launches_per_step = (plan.plan_kernels + 1 + (0 if args.fused else 1) +
                          (1 if cfg.payload == "fp8" and (4 * (cfg.H // 128)) % 16 else 0))
 
+    # dedup counters (informational, read after the timed region): the plan lists one move
+    # per (token, destination rank); entries beyond that are fanned out locally
+    moves = int(plan.arrays()["rcnt"].sum().item())
+    dedup = {"entries": entries, "moves": moves,
+             "moves_per_token": round(moves / cfg.N, 4),
+             "redundant_fraction": round(1.0 - moves / max(entries, 1), 4),
+             "wire_bytes": moves * cfg.row_bytes}
+
     # end to end: pinned host inputs -> device, step, result -> pinned host
     e2e = None
     if args.e2e_steps > 0:
@@ -510,6 +518,7 @@ def run_ours(args):
                      "frac": round(achieved / peak, 4),
                      "traffic": kernel_traffic(dom, cfg, dropped=args.drop > 0)},
         "gpu_launches": launches_per_step * args.steps,
+        "dedup": dedup,
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,
