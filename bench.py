@@ -14,6 +14,12 @@ of all ranks' bytes over the slowest rank's time.
 
 --impl reference times the CPU oracle (single thread, the machine's host core) on a bounded
 token sample of the same workload and prints the same metric.
+
+Variants of the step (each prints the same kind of line): --fused (dispatch and combine in
+one moe_dispatch_combine launch), --combine ranked (rank-grouped combine order), --align A
+and --drop F (aligned segments, dropped entries), --micro-batches M [--overlap | --fused]
+(pipelined micro-batches), --no-graph (host launches instead of graph replay).
+--latency N1,N2,... prints per-call latencies at small token counts instead.
 """
 
 from __future__ import annotations
