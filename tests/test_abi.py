@@ -135,3 +135,9 @@ def test_wait_selftest_rejects_unknown_wait_on_host(lib):
     flags = ctypes.c_uint32(0)
     assert lib.moe_wait_selftest(7, None, ctypes.byref(flags)) == 1
     assert lib.moe_wait_selftest(0, None, None) == 1
+
+
+def test_fused_call_rejects_null_plans_on_host(lib):
+    args = [None, 0, None, 64, None, None, None, None, 64, None, None, 0, None]
+    assert lib.moe_dispatch_combine(*args) == 1
+    assert b"plan" in lib.moe_last_error()
