@@ -106,10 +106,24 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def code_digest(paths) -> str:
+    """SHA-256 of C/C++/CUDA sources with comments and whitespace removed: it changes when
+    the code changes, not when a comment does."""
+    import re
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)   # block comments
+        text = re.sub(r"//[^\n]*", " ", text)                # line comments
+        h.update("".join(text.split()).encode())
+    return h.hexdigest()
+
+
 def kernel_traffic(kernel: str, cfg: Config, dropped: bool = False):
     """DRAM bytes per launch from the committed ncu summary: the captured bytes per token
     scaled to this launch's tokens, if the capture was of this row shape, with every entry
-    routed, and the kernel's sources are unchanged since; else None."""
+    routed, and the kernel's code is unchanged since (comments aside); else None."""
     if dropped:
         return None
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
@@ -122,11 +136,7 @@ def kernel_traffic(kernel: str, cfg: Config, dropped: bool = False):
     if (shape.get("H"), shape.get("k"), shape.get("payload")) != (cfg.H, cfg.k, cfg.payload):
         return None
     units = cfg.N
-    h = hashlib.sha256()
-    for rel in rec["sources"]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
-    if h.hexdigest() != rec["sources_sha256"]:
+    if code_digest(rec["sources"]) != rec.get("sources_code_sha256"):
         return None
     return rec["bytes_per_unit"] * units
 

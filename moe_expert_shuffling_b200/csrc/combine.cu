@@ -3,13 +3,14 @@
 // sections 1-2).  The chain runs in top-k column order, so every launch configuration
 // and both engines give the same bits.
 //
-// Bulk engine (default): persistent CTAs, one producer warp and four consumer warps.
-// Work unit = (token, 2 KB column chunk of every row).  The producer issues one bulk
-// async copy per routed row chunk (lane j copies row slot[t, j]) into a ring of stages
-// in shared memory, each completing on a "full" mbarrier; consumers take a stage, each
-// thread reduces 8 columns over the k rows from shared memory and writes 16 bytes of
-// out, then release the stage on its "empty" mbarrier.  Bytes in flight are bounded by
-// shared memory (up to ~190 KB per SM) rather than by registers.
+// Bulk engine (default, combine_cta.cuh): CTAs of one producer warp and CW consumer
+// warps (8, 4, 2 or 1 as k grows), each CTA taking a short run of tokens on a grid that
+// covers them all.  Work unit = (token, CW * 512-byte column chunk of every row).  The
+// producer issues one bulk async copy per routed row chunk (lane j copies row slot[t, j])
+// into a ring of stages in shared memory, each completing on a "full" mbarrier; consumers
+// take a stage, each thread reduces 8 columns over the k rows from shared memory and
+// writes 16 bytes of out, then release the stage on its "empty" mbarrier.  Bytes in flight
+// are bounded by shared memory rather than by registers.
 //
 // LSU engine (for comparison): a persistent grid of warps over (token, 32*VPL vector)
 // units; each lane issues its KB x VPL 16-byte loads before the first fma.

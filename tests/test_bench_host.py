@@ -1,7 +1,6 @@
 """Host-side logic of bench.py (no GPU): the algorithmic byte counts behind the metric,
 the per-kernel statistics, the L2 statement, and the DRAM-traffic lookup."""
 
-import hashlib
 import json
 import os
 
@@ -70,20 +69,22 @@ def test_l2_note_states_sizes():
 
 def test_kernel_traffic_lookup(tmp_path, monkeypatch):
     src = tmp_path / "k.cu"
-    src.write_text("kernel source")
-    sha = hashlib.sha256(b"kernel source").hexdigest()
+    src.write_text("int f() { return 1; }  // a kernel\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     (tmp_path / "profiles").mkdir()
     rec = {"dispatch_bulk_kernel": {"bytes_per_unit": 100.0, "unit": "token",
                                     "shape": {"H": 7168, "k": 8, "payload": "bf16"},
-                                    "sources": ["k.cu"], "sources_sha256": sha}}
+                                    "sources": ["k.cu"],
+                                    "sources_code_sha256": bench.code_digest(["k.cu"])}}
     (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps(rec))
-    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     cfg = CONFIGS["dsv3"]
     assert bench.kernel_traffic("dispatch_bulk_kernel", cfg) == 100.0 * cfg.N
     assert bench.kernel_traffic("dispatch_bulk_kernel", cfg, dropped=True) is None
     assert bench.kernel_traffic("dispatch_bulk_kernel", CONFIGS["long"]) is None   # other shape
     assert bench.kernel_traffic("combine_bulk_kernel", cfg) is None                # not captured
-    src.write_text("kernel source, edited")
+    src.write_text("/* reworded */ int f()\n{\n    return 1;  // the same code\n}\n")
+    assert bench.kernel_traffic("dispatch_bulk_kernel", cfg) == 100.0 * cfg.N    # comments only
+    src.write_text("int f() { return 2; }\n")
     assert bench.kernel_traffic("dispatch_bulk_kernel", cfg) is None               # stale
 
 
