@@ -186,10 +186,15 @@ MOE_API moe_status moe_combine(const void *y, int32_t H, moe_plan_t plan, void *
  * process exits; a call needing more than (E + R + 1) * ceil(N / 128) <= 262144 scratch
  * words returns MOE_EINVAL.  The first call on each device does a one-time set-up (it
  * looks up that array's device address); make that first call before any stream capture
- * begins.  All
- * calls share the array, so calls whose kernels could overlap on the GPU race and must
- * be ordered (one stream, or events).  topk_w is not taken: moe_combine needs a plan
- * from moe_plan.
+ * begins.  All calls share the array, so calls whose kernels could overlap on the GPU race
+ * and must be ordered (one stream, or events).  topk_w is not taken: moe_combine needs a
+ * plan from moe_plan.
+ *
+ * The call runs on the current device (ordinals 0..63; another ordinal returns MOE_EINVAL),
+ * not on the device that owns the arrays: topk_idx and every output must be device memory
+ * of the current device (or managed memory), else MOE_EINVAL before anything is enqueued.
+ * The array's device address is looked up once per device and kept, so cudaDeviceReset
+ * between calls is not supported.
  */
 MOE_API moe_status moe_plan_noalloc(const int32_t *topk_idx, int32_t N, int32_t k, int32_t E,
                                     int32_t R, int32_t *cnt, int32_t *expert_off, int32_t *rcnt,
@@ -284,10 +289,10 @@ typedef enum {
     MOE_TUNE_DISPATCH_LAG = 1,           /* store groups a warp keeps in flight (1..stages-1) */
     MOE_TUNE_DISPATCH_CTAS_PER_SM = 2,   /* cap on resident dispatch CTAs per SM */
     MOE_TUNE_DISPATCH_WARPS_PER_CTA = 3, /* dispatch warps per CTA (1..4) */
-    MOE_TUNE_COMBINE_VEC_PER_LANE = 4,   /* LSU combine: 16-byte vectors per lane (1, 2, 4) */
+                                         /* 4: retired (an engine that was slower) */
     MOE_TUNE_COMBINE_CTAS_PER_SM = 5,    /* cap on resident combine CTAs per SM */
     MOE_TUNE_COMBINE_STAGES = 6,         /* bulk combine: shared-memory stages (2..16) */
-    MOE_TUNE_COMBINE_ENGINE = 7,         /* 0 or 1: bulk-copy engine, 2: LSU engine */
+                                         /* 7: retired */
     MOE_TUNE_COMBINE_SMEM_KB = 8,        /* bulk combine: shared-memory budget per CTA (KB) */
     MOE_TUNE_DISPATCH_UNITS_PER_WARP = 9, /* (token, chunk) units per dispatch warp */
     MOE_TUNE_COMBINE_TOKENS_PER_CTA = 10, /* tokens per bulk-combine CTA */

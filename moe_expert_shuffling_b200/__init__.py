@@ -33,8 +33,8 @@ MOE_BF16, MOE_FP8E4M3 = 0, 1
 ERR_ID_RANGE, ERR_ID_DUP, ERR_BOUNDS, ERR_TIMEOUT = 1, 2, 4, 8
 KNOBS = {
     "dispatch_stages": 0, "dispatch_lag": 1, "dispatch_ctas_per_sm": 2,
-    "dispatch_warps_per_cta": 3, "combine_vec_per_lane": 4, "combine_ctas_per_sm": 5,
-    "combine_stages": 6, "combine_engine": 7, "combine_smem_kb": 8,
+    "dispatch_warps_per_cta": 3, "combine_ctas_per_sm": 5,
+    "combine_stages": 6, "combine_smem_kb": 8,
     "dispatch_units_per_warp": 9, "combine_tokens_per_cta": 10, "plan_engine": 11,
     "fused_ctas_per_sm": 12, "fused_dispatch_share": 13, "fused_dispatch_run": 14,
     "fused_combine_run": 15, "fused_smem_kb": 16, "fused_min_kb": 17, "combine_max_cw": 18,

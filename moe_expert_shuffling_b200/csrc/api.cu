@@ -198,10 +198,8 @@ moe_status moe_tune(moe_knob knob, int32_t value)
     case MOE_TUNE_DISPATCH_LAG: t.dispatch_lag = value; break;
     case MOE_TUNE_DISPATCH_CTAS_PER_SM: t.dispatch_ctas_per_sm = value; break;
     case MOE_TUNE_DISPATCH_WARPS_PER_CTA: t.dispatch_warps_per_cta = value; break;
-    case MOE_TUNE_COMBINE_VEC_PER_LANE: t.combine_vec_per_lane = value; break;
     case MOE_TUNE_COMBINE_CTAS_PER_SM: t.combine_ctas_per_sm = value; break;
     case MOE_TUNE_COMBINE_STAGES: t.combine_stages = value; break;
-    case MOE_TUNE_COMBINE_ENGINE: t.combine_mode = value; break;
     case MOE_TUNE_COMBINE_SMEM_KB: t.combine_smem_kb = value; break;
     case MOE_TUNE_DISPATCH_UNITS_PER_WARP: t.dispatch_units_per_warp = value; break;
     case MOE_TUNE_COMBINE_TOKENS_PER_CTA: t.combine_tokens_per_cta = value; break;

@@ -57,10 +57,8 @@ struct Tuning {
     int dispatch_lag = 0;
     int dispatch_ctas_per_sm = 0;
     int dispatch_warps_per_cta = 0;
-    int combine_vec_per_lane = 0;
     int combine_ctas_per_sm = 0;
     int combine_stages = 0;
-    int combine_mode = 0;      // 0/1: bulk engine, 2: LSU engine
     int combine_smem_kb = 0;
     int dispatch_units_per_warp = 0;
     int combine_tokens_per_cta = 0;

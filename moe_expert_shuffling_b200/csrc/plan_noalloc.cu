@@ -12,6 +12,10 @@
 // has to start at zero, because each call writes every scratch word it later reads.
 // Calls whose kernels overlap on the GPU (for example on two streams without an
 // ordering between them) race on the array and must not be issued.
+//
+// The array's device address is looked up once per device ordinal (below 64) and kept, so
+// the library does not support cudaDeviceReset between calls: a new context would be given
+// the old context's address.
 #include <mutex>
 
 #include "common.cuh"
@@ -51,6 +55,29 @@ moe_status scratch_address(int dev, int32_t **out)
 }
 
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// The caller owns every array, so a host pointer or another GPU's pointer would reach the
+// kernels unchecked; reject anything but device memory of `dev` (or managed memory) here.
+moe_status check_device_array(const void *p, int dev, const char *name)
+{
+    cudaPointerAttributes a{};
+    const cudaError_t e = cudaPointerGetAttributes(&a, p);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return moe::record_error(MOE_EINVAL, "moe_plan_noalloc: %s is not device memory (%s)",
+                                 name, cudaGetErrorString(e));
+    }
+    if (a.type == cudaMemoryTypeManaged)
+        return MOE_OK;
+    if (a.type != cudaMemoryTypeDevice)
+        return moe::record_error(MOE_EINVAL,
+                                 "moe_plan_noalloc: %s is host memory, not device memory", name);
+    if (a.device != dev)
+        return moe::record_error(MOE_EINVAL,
+                                 "moe_plan_noalloc: %s lives on device %d but device %d is current",
+                                 name, a.device, dev);
+    return MOE_OK;
+}
 
 }  // namespace
 
@@ -94,6 +121,15 @@ extern "C" moe_status moe_plan_noalloc(const int32_t *topk_idx, int32_t N, int32
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return moe::record_error(MOE_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    const char *names[] = {"topk_idx", "cnt", "expert_off", "rcnt", "rank_off", "rtok_off", "slot",
+                           "src_tok", "src_j", "rtok", "fanout", "err"};
+    for (int i = 0; i < 12; ++i) {
+        if (!ptrs[i])
+            continue;  // only the per-entry arrays may be NULL, and only when N == 0
+        const moe_status pst = check_device_array(ptrs[i], dev, names[i]);
+        if (pst != MOE_OK)
+            return pst;
+    }
     int32_t *scratch = nullptr;
     const moe_status st = scratch_address(dev, &scratch);
     if (st != MOE_OK)

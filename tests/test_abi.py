@@ -95,6 +95,8 @@ def test_destroy_null_is_noop(lib):
 
 def test_tune_rejects_unknown_knob(lib):
     assert lib.moe_tune(99, 1) == 1
+    assert lib.moe_tune(4, 1) == 1   # retired knobs
+    assert lib.moe_tune(7, 1) == 1
     assert lib.moe_tune(0, -1) == 1
     assert lib.moe_tune(0, 0) == 0   # default restored
 
@@ -102,7 +104,7 @@ def test_tune_rejects_unknown_knob(lib):
 def test_python_binding_imports_and_knows_knobs():
     import moe_expert_shuffling_b200 as ms
     assert ms.version().startswith("moeshuffle")
-    assert set(ms.KNOBS) >= {"dispatch_stages", "combine_vec_per_lane"}
+    assert set(ms.KNOBS) >= {"dispatch_stages", "combine_stages"}
     with pytest.raises(TypeError):
         ms.moe_plan("not a tensor", None, 8, 4)
 
@@ -141,3 +143,17 @@ def test_fused_call_rejects_null_plans_on_host(lib):
     args = [None, 0, None, 64, None, None, None, None, 64, None, None, 0, None]
     assert lib.moe_dispatch_combine(*args) == 1
     assert b"plan" in lib.moe_last_error()
+
+
+@pytest.mark.parametrize("N,k,E,R", [
+    (1 << 20, 8, 256, 32),          # far beyond the fixed scratch array
+    (127 * 128 + 1, 8, 1024, 1024),  # one tile past the limit: (2049) * 128 > 262144 words
+    (907 * 128 + 1, 8, 256, 32),     # one tile past the limit: 289 * 908 > 262144 words
+])
+def test_noalloc_rejects_more_tokens_than_its_scratch_holds(lib, N, k, E, R):
+    """The size limit of moe_plan_noalloc is checked on the host before anything else; no
+    array is passed, so even a broken check could not launch a kernel."""
+    lib.moe_plan_noalloc.restype = ctypes.c_int
+    st = lib.moe_plan_noalloc(None, N, k, E, R, *([None] * 11), None)
+    assert st == 1
+    assert b"scratch" in lib.moe_last_error()

@@ -136,14 +136,8 @@ def test_identity_experts_return_x(name):
     CONFIGS["long"].replace(N=50, H=65536),                                # chunked fp8 row
     CONFIGS["long"].replace(N=1000, H=512, k=4, E=16, R=16),
 ], ids=lambda c: f"{c.name}-N{c.N}-H{c.H}-E{c.E}-k{c.k}-R{c.R}-{c.payload}")
-@pytest.mark.parametrize("engine", [0, 2], ids=["bulk", "lsu"])
-def test_edge_shapes(cfg, engine):
-    import moe_expert_shuffling_b200 as ms
-    ms.moe_tune("combine_engine", engine)
-    try:
-        r = run_all(cfg, 0)
-    finally:
-        ms.moe_tune("combine_engine", 0)
+def test_edge_shapes(cfg):
+    r = run_all(cfg, 0)
     assert_plan_equal(r["gp"], r["ref"])
     assert np.array_equal(r["got_recv"], r["ref_recv"])
     if r["ref_rs"] is not None:
@@ -188,53 +182,50 @@ def test_plan_reuse_and_capacity():
 
 
 def test_invalid_routing_is_flagged_and_contained():
-    """Out-of-range and repeated ids set error bits, get slot -1 and are skipped."""
+    """Out-of-range and repeated ids set error bits, get slot -1 and are skipped: plan,
+    dispatch and combine equal, bit for bit, the oracle's on the routing with those entries
+    marked dropped (-1)."""
     import moe_expert_shuffling_b200 as ms
     cfg = CONFIGS["tiny"].with_tokens(300)
     idx, w, x, _, y = make_inputs(cfg, 0)
     bad = idx.copy()
     bad[3, 0] = cfg.E            # out of range
     bad[10, 1] = -5              # negative
-    bad[20, 1] = bad[20, 0]      # repeated in one token
+    bad[20, 1] = bad[20, 0]      # repeated in one token (the first occurrence stays valid)
     bad[299, 0] = 2 ** 31 - 1
     p, ti, tw = gpu_plan(bad, w, cfg.E, cfg.R)
     recv = torch.zeros((cfg.N * cfg.k, cfg.H), dtype=torch.bfloat16, device="cuda")
     ms.moe_dispatch(x, p, recv=recv)
     out = ms.moe_combine(y, p)
+    out_r = ms.moe_combine(y, p, ranked=True)
     flags = p.check()
     assert flags & ms.ERR_ID_RANGE and flags & ms.ERR_ID_DUP
     assert not flags & (ms.ERR_BOUNDS | ms.ERR_TIMEOUT)
+
+    cleaned = bad.copy()
+    for t, j in ((3, 0), (10, 1), (20, 1), (299, 0)):
+        cleaned[t, j] = -1
+    ref = oracle.plan(cleaned, cfg.E, cfg.R)
     g = plan_to_host(p)
-    valid = np.ones_like(bad, dtype=bool)
-    valid[3, 0] = valid[10, 1] = valid[20, 1] = valid[299, 0] = False
-    assert np.all(g["slot"][~valid] == -1)
-    # the valid entries form the plan of the routing with the bad entries removed
-    n_valid = int(valid.sum())
-    assert int(g["cnt"].sum()) == n_valid
-    s = g["slot"][valid]
-    assert np.array_equal(np.sort(s), np.arange(n_valid))
-    xb = bits16(x)
-    rb = bits16(recv)
-    tok = np.nonzero(valid)[0]
-    assert np.array_equal(rb[s], xb[tok])
-    # combine of a token with a skipped entry sums only its valid entries
+    for name in ("cnt", "expert_off", "rcnt", "rank_off", "rtok_off", "slot", "src_tok",
+                 "src_j", "rtok"):
+        assert np.array_equal(g[name], getattr(ref, name)), name
+    assert np.array_equal(g["fanout"], ref.fanout)
+    assert int(g["cnt"].sum()) == int((cleaned >= 0).sum())
+    used = ref.src_tok >= 0
+    want_recv = oracle.dispatch(bits16(x).view(np.uint8).reshape(cfg.N, -1), ref.slot)
+    got_recv = bits16(recv).view(np.uint8).reshape(cfg.N * cfg.k, -1)
+    assert np.array_equal(got_recv[used], want_recv[used])
+    assert not got_recv[~used].any()              # rows no entry maps to stay untouched
     yb = bits16(y)
-    t = 3
-    acc = np.float32(0)
-    for j in range(cfg.k):
-        if valid[t, j]:
-            acc = np.float32(acc + np.float32(w[t, j]) * bits_to_f32(yb[g["slot"][t, j]]))
-    got = bits_to_f32(bits16(out)[t])
-    assert np.allclose(got, acc, rtol=8e-3, atol=1e-2)
+    assert np.array_equal(bits16(out), oracle.combine(yb, ref.slot, w))
+    assert np.array_equal(bits16(out_r), oracle.combine_ranked(yb, ref.slot, w, cleaned, cfg.E, cfg.R))
 
 
 @pytest.mark.parametrize("knobs", [
     {"dispatch_stages": 2, "dispatch_lag": 1},
     {"dispatch_stages": 8, "dispatch_lag": 4, "dispatch_warps_per_cta": 2},
     {"dispatch_ctas_per_sm": 1, "combine_ctas_per_sm": 1},
-    {"combine_engine": 2, "combine_vec_per_lane": 1},
-    {"combine_engine": 2, "combine_vec_per_lane": 2},
-    {"combine_engine": 2, "combine_vec_per_lane": 4},
     {"combine_stages": 2},
     {"plan_engine": 2},
     {"dispatch_units_per_warp": 10000, "combine_tokens_per_cta": 10000},
