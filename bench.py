@@ -141,6 +141,24 @@ def kernel_traffic(kernel: str, cfg: Config, dropped: bool = False):
     return rec["bytes_per_unit"] * units
 
 
+def step_traffic(cfg: Config, fused: bool, algorithmic: int, dropped: bool = False,
+                 aligned: bool = False, ranked: bool = False):
+    """DRAM bytes of one whole step (plan, dispatch, combine -- or plan and the fused
+    launch) from the committed ncu capture of consecutive launches with caches left alone
+    (--cache-control none), so that lines one kernel leaves dirty in L2 are counted when
+    the next one writes them back; scaled per token to this workload when the capture was
+    of this shape and the kernels' code is unchanged.  Against the algorithmic bytes."""
+    if dropped or aligned or ranked:
+        return None
+    key = f"step_{cfg.name}" + ("_fused" if fused else "")
+    bpt = kernel_traffic(key, cfg)
+    if bpt is None:
+        return None
+    return {"dram_bytes": round(bpt), "algorithmic_bytes": algorithmic,
+            "ratio": round(bpt / algorithmic, 4),
+            "source": "profiles/dram_traffic.json: " + key}
+
+
 def pct_stats(ms_list):
     """median / p10 / p90 of event times given in ms, reported in us."""
     v = sorted(1e3 * t for t in ms_list)
@@ -299,11 +317,47 @@ def barrier(world: int):
         dist.barrier()
 
 
+def apply_tuning(args):
+    """--tune KNOB=VALUE: launch parameters of the library (speed only, never results)."""
+    import moe_expert_shuffling_b200 as ms
+    for t in args.tune:
+        knob, value = t.split("=")
+        ms.moe_tune(knob, int(value))
+
+
+def plan_cost_in_step(step, stream, step_ms: float, args) -> dict:
+    """What the plan adds to a graph-replayed step: the same replays of a graph holding only
+    dispatch and combine (on the plan already built), against the timed step.  The per-kernel
+    event timings launch each kernel from the host between two events, so their plan figure
+    is mostly launch latency; this one is measured the way `value` is."""
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step(phase_only=1)
+        if not args.fused:
+            step(phase_only=2)
+    stream.synchronize()
+    n = max(10, min(args.steps, 500))
+    with torch.cuda.stream(stream):
+        graph.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            graph.replay()
+        b.record(stream)
+    b.synchronize()
+    without = a.elapsed_time(b) / n
+    del graph
+    return {"step_us": round(1e3 * step_ms, 2), "step_without_plan_us": round(1e3 * without, 2),
+            "plan_us": round(1e3 * (step_ms - without), 2),
+            "note": "graph replays of the whole step against replays of dispatch + combine alone"}
+
+
 def run_ours(args):
     import moe_expert_shuffling_b200 as ms
     from moe_expert_shuffling_b200 import build as lib_build
 
     lib_build.build()
+    apply_tuning(args)
     world, rank, local = dist_setup(args)
     cfg = CONFIGS[args.config]
     if args.tokens > 0:
@@ -329,7 +383,8 @@ def run_ours(args):
         out = torch.empty((cfg.N, cfg.H), dtype=torch.bfloat16, device=dev)
     stream.synchronize()
     identity = y is None
-    plan = ms.moe_plan_create(cfg.N, cfg.k, cfg.E, cfg.R, align=args.align)
+    plan = ms.moe_plan_create(cfg.N, cfg.k, cfg.E, cfg.R, align=args.align,
+                              dedup_lists=not args.no_dedup_lists)
 
     def step(ev=None, phase_only=None):
         """One step: plan, dispatch, combine (phase_only = 0, 1 or 2 runs just that one).
@@ -404,6 +459,7 @@ def run_ours(args):
         evs = evs[:min(args.steps, 200)]
     else:
         elapsed_ms = evs[0][0].elapsed_time(evs[-1][3])
+    plan_cost = plan_cost_in_step(step, stream, elapsed_ms / args.steps, args) if graph else None
     t_plan = [e[0].elapsed_time(e[1]) for e in evs]
     t_disp = [e[1].elapsed_time(e[2]) for e in evs]
     t_comb = [e[2].elapsed_time(e[3]) for e in evs]
@@ -432,6 +488,7 @@ def run_ours(args):
     # dedup counters (informational, read after the timed region): the plan lists one move
     # per (token, destination rank); entries beyond that are fanned out locally
     moves = int(plan.arrays()["rcnt"].sum().item())
+    plan_kind = plan.plan_kind
     dedup = {"entries": entries, "moves": moves,
              "moves_per_token": round(moves / cfg.N, 4),
              "redundant_fraction": round(1.0 - moves / max(entries, 1), 4),
@@ -509,7 +566,9 @@ def run_ours(args):
                    + ("" if args.combine == "chain" else ", combine grouped by rank")
                    + (f", segments aligned to {args.align} rows" if args.align > 1 else "")
                    + (f", {args.drop:.0%} of entries dropped" if args.drop > 0 else "")
-                   + (", dispatch and combine in one launch" if args.fused else ""),
+                   + (", dispatch and combine in one launch" if args.fused else "")
+                   + (", plan without the per-rank lists" if args.no_dedup_lists else "")
+                   + "".join(f", {t}" for t in args.tune),
                    "model": f"{cfg.name}-shaped MoE layer shuffle",
                    "global_batch": cfg.N * world, "seq_len": cfg.N, "parallelism": f"replicas{world}",
                    "ep_ranks_logical": cfg.R,
@@ -524,6 +583,7 @@ def run_ours(args):
             {"note": "back-to-back steps on one stream, no flush", "plan": pct_stats(t_plan),
              "dispatch": pct_stats(t_disp), "combine": pct_stats(t_comb)}, args.fused),
         "kernels_flushed_us": flushed,
+        "plan_in_step_us": plan_cost,
         "kernels_gbs": kernel_split(
             {"dispatch": round(db / (disp_us * 1e-6) / 1e9, 1),
              "combine": round(cb / (max(comb_us, 1e-3) * 1e-6) / 1e9, 1),
@@ -533,7 +593,11 @@ def run_ours(args):
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "traffic": kernel_traffic(dom, cfg, dropped=args.drop > 0)},
+        "step_traffic": step_traffic(cfg, args.fused, db + cb + plan_bytes(cfg),
+                                     dropped=args.drop > 0, aligned=args.align > 1,
+                                     ranked=args.combine == "ranked"),
         "gpu_launches": launches_per_step * args.steps,
+        "plan_kind": plan_kind,
         "dedup": dedup,
         "clocks": clk,
         "e2e": e2e,
@@ -551,6 +615,7 @@ def run_micro_batches(args):
     from moe_expert_shuffling_b200 import build as lib_build
 
     lib_build.build()
+    apply_tuning(args)
     world, rank, local = dist_setup(args)
     cfg = CONFIGS[args.config]
     if args.tokens > 0:
@@ -652,6 +717,7 @@ def run_latency(args):
     from moe_expert_shuffling_b200 import build as lib_build
 
     lib_build.build()
+    apply_tuning(args)
     dev = torch.device("cuda", 0)
     s = torch.cuda.Stream(device=dev)
 
@@ -706,7 +772,7 @@ def run_latency(args):
                "plan": replay_us(pl, args.steps), "dispatch": replay_us(dp, args.steps),
                "combine": replay_us(cb, args.steps), "dispatch_combine": replay_us(dc, args.steps),
                "step": replay_us(lambda: (pl(), dp(), cb()), args.steps),
-               "plan_kernels": plan.plan_kernels}
+               "plan_kernels": plan.plan_kernels, "plan_kind": plan.plan_kind}
         if plan.check(s) != 0:
             raise SystemExit("device reported invalid routing or a timeout")
         plan.close()
@@ -856,6 +922,10 @@ def main(argv=None):
                     help="dispatch and combine in one launch (moe_dispatch_combine)")
     ap.add_argument("--combine", default="chain", choices=["chain", "ranked"],
                     help="combine order: one fma chain per token, or grouped by rank first")
+    ap.add_argument("--no-dedup-lists", action="store_true",
+                    help="plans skip the per-rank lists rtok / fanout (MOE_PLAN_NO_DEDUP_LISTS)")
+    ap.add_argument("--tune", action="append", default=[], metavar="KNOB=VALUE",
+                    help="set a launch parameter (moe_tune; speed only), repeatable")
     ap.add_argument("--flushed-iters", type=int, default=50,
                     help="iterations of each kernel timed alone after an L2 flush (0: skip)")
     ap.add_argument("--seed", type=int, default=0)
@@ -868,6 +938,7 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+
     if args.impl == "reference":
         run_reference(args)
     elif args.latency:

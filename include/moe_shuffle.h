@@ -82,7 +82,15 @@ typedef struct {
     int32_t plan_kernels;          /* kernels the last moe_plan call enqueued (1 or 3) */
     int32_t align;                 /* expert segments start on multiples of this many rows */
     int32_t recv_rows;             /* rows a receive buffer needs: N*k + E*(align-1) */
+    int32_t plan_kind;             /* MOE_PLAN_KIND_* of the last moe_plan call */
+    int32_t dedup_lists;           /* 1 if moe_plan writes rtok / fanout (the default) */
 } moe_plan_view;
+
+/* Which planner kernel the last moe_plan call ran (moe_plan_view.plan_kind). */
+#define MOE_PLAN_KIND_ONE_TILE 0    /* N <= 128: one block */
+#define MOE_PLAN_KIND_GROUPS 1      /* thread-block clusters of up to 16 tiles of 128 tokens */
+#define MOE_PLAN_KIND_COOPERATIVE 2 /* one cooperative kernel with two grid barriers */
+#define MOE_PLAN_KIND_THREE 3       /* count, scan and rank kernels */
 
 /*
  * moe_plan_create -- allocate a plan for up to `max_tokens` tokens of shape (k, E, R).
@@ -103,6 +111,19 @@ MOE_API moe_status moe_plan_create(int32_t max_tokens, int32_t k, int32_t E, int
  */
 MOE_API moe_status moe_plan_create_aligned(int32_t max_tokens, int32_t k, int32_t E, int32_t R,
                                            int32_t align, moe_plan_t *out);
+
+/* Flags of moe_plan_create_ex. */
+#define MOE_PLAN_NO_DEDUP_LISTS 1u  /* moe_plan skips the per-rank lists rtok / fanout */
+
+/*
+ * moe_plan_create_ex -- as moe_plan_create_aligned, with option flags.  With
+ * MOE_PLAN_NO_DEDUP_LISTS the plan's per-rank dedup lists (rtok, fanout) are not written by
+ * moe_plan (their contents are then undefined); everything else, rcnt and rtok_off
+ * included, is.  Neither dispatch nor combine reads the lists, so callers that do not use
+ * them save the planner their stores.  Unknown flags return MOE_EINVAL.
+ */
+MOE_API moe_status moe_plan_create_ex(int32_t max_tokens, int32_t k, int32_t E, int32_t R,
+                                      int32_t align, uint32_t flags, moe_plan_t *out);
 
 /*
  * moe_plan -- build the logical-segment plan of one routing (FUSCO abstract: the
@@ -132,9 +153,13 @@ MOE_API moe_status moe_plan_create_aligned(int32_t max_tokens, int32_t k, int32_
  *   rtok/fanout = the tokens of rank r in ascending order with the mask of their
  *   columns on r -- one move per (token, rank) pair.
  * Deterministic (no result depends on thread timing).  Enqueues one kernel: a single
- * block for N <= 128 (one tile), one thread-block cluster of one block per 128 tokens for
- * N <= 2048, else one cooperative kernel (three kernels where its grid cannot be
- * co-resident).
+ * block for N <= 128 (one tile); else one block per 128 tokens in thread-block clusters of
+ * up to 16 blocks, which combine their counts through distributed shared memory and, with
+ * more than one cluster, exchange the clusters' totals once through global memory (a
+ * cooperative launch); where those clusters cannot all be resident, one cooperative kernel
+ * with two grid barriers, or three kernels where even that grid cannot be co-resident.
+ * A device wait that runs out sets MOE_ERR_TIMEOUT, which stays in the error word until
+ * moe_plan_check reports it and rearms the plan.
  */
 MOE_API moe_status moe_plan(const int32_t *topk_idx, const float *topk_w, int32_t N, int32_t k,
                     int32_t E, int32_t R, void *stream, moe_plan_t *plan);
@@ -253,8 +278,10 @@ MOE_API moe_status moe_dispatch_combine(const void *x, moe_dtype dtype, const fl
  *   which = 0  the per-token ready-flag wait of moe_dispatch_combine, on a flag nothing sets;
  *   which = 1  the mbarrier wait of the bulk-copy pipelines, on a barrier that expects two
  *              arrivals and gets one (no copy in flight);
- *   which = 2  the grid barrier of the plan kernel, in a grid of two blocks of which only
- *              one arrives.
+ *   which = 2  the grid barrier of the cooperative plan kernel, in a grid of two blocks of
+ *              which only one arrives;
+ *   which = 3  the exchange wait of the group plan kernel, on two groups' arrival words of
+ *              which only the first is ever set.
  * Each wait gives up after about one second; *flags is then MOE_ERR_TIMEOUT and the CUDA
  * context stays usable.  Synchronous: allocates three device words, launches two 32-thread
  * blocks on `stream`, waits for them and frees the words.  MOE_EINVAL for another `which`
@@ -268,7 +295,8 @@ MOE_API moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *view);
 /*
  * moe_plan_check -- wait for `stream`, then copy the plan's error word to *flags
  * (MOE_ERR_* bits; 0 = the routing was valid and every wait finished).  After a reported
- * MOE_ERR_TIMEOUT it also rearms the plan's grid-barrier words.
+ * MOE_ERR_TIMEOUT it also rearms the plan: its grid-barrier and work words, its ready flags
+ * and its error word.
  */
 MOE_API moe_status moe_plan_check(moe_plan_t plan, void *stream, uint32_t *flags);
 
@@ -296,7 +324,8 @@ typedef enum {
     MOE_TUNE_COMBINE_SMEM_KB = 8,        /* bulk combine: shared-memory budget per CTA (KB) */
     MOE_TUNE_DISPATCH_UNITS_PER_WARP = 9, /* (token, chunk) units per dispatch warp */
     MOE_TUNE_COMBINE_TOKENS_PER_CTA = 10, /* tokens per bulk-combine CTA */
-    MOE_TUNE_PLAN_ENGINE = 11,           /* 0 or 1: one cooperative plan kernel, 2: three kernels */
+    MOE_TUNE_PLAN_ENGINE = 11,           /* 0 or 1: automatic, 2: three kernels, 3: no cluster
+                                            kernel (the cooperative one for N > 128) */
     MOE_TUNE_FUSED_CTAS_PER_SM = 12,     /* moe_dispatch_combine: resident CTAs per SM */
     MOE_TUNE_FUSED_DISPATCH_SHARE = 13,  /* moe_dispatch_combine: % of CTAs that start on dispatch */
     MOE_TUNE_FUSED_DISPATCH_RUN = 14,    /* moe_dispatch_combine: tokens per dispatch work item (1..32) */
@@ -305,8 +334,16 @@ typedef enum {
     MOE_TUNE_FUSED_MIN_KB = 17,          /* moe_dispatch_combine: least traffic (KB) for the
                                             one-launch kernel; smaller calls run the two
                                             kernels back to back (default 327680 = 320 MB) */
-    MOE_TUNE_COMBINE_MAX_CW = 18         /* bulk combine: most consumer warps per CTA (4 or 8;
+    MOE_TUNE_COMBINE_MAX_CW = 18,        /* bulk combine: most consumer warps per CTA (4 or 8;
                                             default 8: k <= 4 uses 8, wider k uses 4 or fewer) */
+    MOE_TUNE_PLAN_CLUSTER = 19,          /* plan: most 128-token tiles per thread-block cluster
+                                            (1..16; default 16) */
+    MOE_TUNE_PDL = 20,                   /* 0 or 1: kernels are programmatic dependent launches
+                                            (each may start while the previous kernel on the
+                                            stream finishes), 2: ordinary launches */
+    MOE_TUNE_PLAN_MATCH = 21             /* plan: how a token's ids are compared: 0 by k (match
+                                            instructions for k > 16), 1 shuffle compares,
+                                            2 warp match instructions */
 } moe_knob;
 
 MOE_API moe_status moe_tune(moe_knob knob, int32_t value);

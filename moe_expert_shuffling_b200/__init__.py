@@ -38,7 +38,9 @@ KNOBS = {
     "dispatch_units_per_warp": 9, "combine_tokens_per_cta": 10, "plan_engine": 11,
     "fused_ctas_per_sm": 12, "fused_dispatch_share": 13, "fused_dispatch_run": 14,
     "fused_combine_run": 15, "fused_smem_kb": 16, "fused_min_kb": 17, "combine_max_cw": 18,
+    "plan_cluster": 19, "pdl": 20, "plan_match": 21,
 }
+PLAN_KINDS = {0: "one_tile", 1: "groups", 2: "cooperative", 3: "three"}
 
 _i32 = ctypes.c_int32
 _vp = ctypes.c_void_p
@@ -50,7 +52,7 @@ class _PlanView(ctypes.Structure):
         ("capacity_tokens", _i32), ("cnt", _vp), ("expert_off", _vp), ("rcnt", _vp),
         ("rank_off", _vp), ("rtok_off", _vp), ("slot", _vp), ("src_tok", _vp), ("src_j", _vp),
         ("rtok", _vp), ("fanout", _vp), ("err", _vp), ("topk_w", _vp), ("plan_kernels", _i32),
-        ("align", _i32), ("recv_rows", _i32),
+        ("align", _i32), ("recv_rows", _i32), ("plan_kind", _i32), ("dedup_lists", _i32),
     ]
 
 
@@ -65,6 +67,9 @@ def _load():
     lib.moe_plan_create.argtypes = [_i32, _i32, _i32, _i32, ctypes.POINTER(_vp)]
     lib.moe_plan_create_aligned.restype = st
     lib.moe_plan_create_aligned.argtypes = [_i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp)]
+    lib.moe_plan_create_ex.restype = st
+    lib.moe_plan_create_ex.argtypes = [_i32, _i32, _i32, _i32, _i32, ctypes.c_uint32,
+                                       ctypes.POINTER(_vp)]
     lib.moe_plan.restype = st
     lib.moe_plan.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, ctypes.POINTER(_vp)]
     lib.moe_dispatch.restype = st
@@ -93,16 +98,26 @@ def _load():
     return lib
 
 
-class _Missing:
-    """Stands in for the library until it is built; every call fails loudly."""
+class _Library:
+    """The library, loaded on first use (so that the package, and its build module, import
+    before the library is built or while it is being rebuilt).  Without the built library
+    every call fails loudly: there is no fallback implementation."""
+
+    def __init__(self):
+        self._handle = None
 
     def __getattr__(self, name):
-        raise ImportError(
-            f"{_LIB_PATH} is missing: build it with `python -m moe_expert_shuffling_b200.build` "
-            "(there is no fallback implementation)")
+        if self._handle is None:
+            if not os.path.exists(_LIB_PATH):
+                raise ImportError(
+                    f"{_LIB_PATH} is missing: build it with "
+                    "`python -m moe_expert_shuffling_b200.build` (there is no fallback "
+                    "implementation)")
+            self._handle = _load()
+        return getattr(self._handle, name)
 
 
-_lib = _load() if os.path.exists(_LIB_PATH) else _Missing()
+_lib = _Library()
 
 
 class MoeError(RuntimeError):
@@ -200,8 +215,18 @@ class Plan:
 
     @property
     def plan_kernels(self) -> int:
-        """Kernels the last moe_plan call enqueued (1 cooperative kernel, or 3)."""
+        """Kernels the last moe_plan call enqueued (1, or 3)."""
         return self._view().plan_kernels
+
+    @property
+    def plan_kind(self) -> str:
+        """Planner kernel of the last moe_plan call: one_tile, groups, cooperative or three."""
+        return PLAN_KINDS[self._view().plan_kind]
+
+    @property
+    def dedup_lists(self) -> bool:
+        """Whether moe_plan writes the per-rank lists rtok / fanout."""
+        return bool(self._view().dedup_lists)
 
     def arrays(self) -> dict[str, torch.Tensor]:
         """Zero-copy int32 views of the plan's device arrays (fanout/err as bit patterns)."""
@@ -245,11 +270,17 @@ class Plan:
             pass
 
 
-def moe_plan_create(max_tokens: int, k: int, E: int, R: int, align: int = 1) -> Plan:
-    """Allocate a reusable plan; with align > 1 expert segments start on multiples of it."""
+PLAN_NO_DEDUP_LISTS = 1
+
+
+def moe_plan_create(max_tokens: int, k: int, E: int, R: int, align: int = 1,
+                    dedup_lists: bool = True) -> Plan:
+    """Allocate a reusable plan; with align > 1 expert segments start on multiples of it;
+    with dedup_lists=False moe_plan skips the per-rank lists rtok / fanout."""
     h = _vp(0)
-    _check(_lib.moe_plan_create_aligned(int(max_tokens), int(k), int(E), int(R), int(align),
-                                        ctypes.byref(h)))
+    flags = 0 if dedup_lists else PLAN_NO_DEDUP_LISTS
+    _check(_lib.moe_plan_create_ex(int(max_tokens), int(k), int(E), int(R), int(align), flags,
+                                   ctypes.byref(h)))
     return Plan(h.value)
 
 

@@ -126,6 +126,62 @@ int max_smem_optin(int device)
     return cache[device];
 }
 
+cudaError_t launch_ex(const void *kernel, void **args, dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t stream, bool cooperative, int device,
+                      const cudaLaunchAttribute *extra, int n_extra)
+{
+    // [device][cooperative]: 1 once a programmatic launch of that kind succeeded, -1 once
+    // the runtime refused the attribute for it
+    static int pdl_state[64][2] = {};
+    const int dv = device >= 0 && device < 64 ? device : 0;
+    const int kind = cooperative ? 1 : 0;
+    bool pdl = tuning().pdl != 2 && pdl_state[dv][kind] >= 0;
+    if (pdl && pdl_state[dv][kind] == 0) {
+        // the first launch of a kind is not tried inside a stream capture, where a refused
+        // launch would invalidate the capture
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+            (void)cudaGetLastError();
+            pdl = false;
+        } else if (cs != cudaStreamCaptureStatusNone) {
+            pdl = false;
+        }
+    }
+    cudaLaunchAttribute attr[4];
+    int n = 0;
+    for (int i = 0; i < n_extra && n < 2; ++i)
+        attr[n++] = extra[i];
+    if (cooperative) {
+        attr[n].id = cudaLaunchAttributeCooperative;
+        attr[n].val.cooperative = 1;
+        ++n;
+    }
+    const int without_pdl = n;
+    if (pdl) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = static_cast<unsigned>(n);
+    cudaError_t e = cudaLaunchKernelExC(&cfg, kernel, args);
+    if (pdl && e == cudaSuccess) {
+        pdl_state[dv][kind] = 1;
+    } else if (pdl && pdl_state[dv][kind] == 0) {
+        (void)cudaGetLastError();
+        cfg.numAttrs = static_cast<unsigned>(without_pdl);
+        e = cudaLaunchKernelExC(&cfg, kernel, args);
+        if (e == cudaSuccess)
+            pdl_state[dv][kind] = -1;
+    }
+    return e;
+}
+
 namespace {
 struct FitEntry {
     const void *kernel;
@@ -211,6 +267,9 @@ moe_status moe_tune(moe_knob knob, int32_t value)
     case MOE_TUNE_FUSED_SMEM_KB: t.fused_smem_kb = value; break;
     case MOE_TUNE_FUSED_MIN_KB: t.fused_min_kb = value; break;
     case MOE_TUNE_COMBINE_MAX_CW: t.combine_max_cw = value; break;
+    case MOE_TUNE_PLAN_CLUSTER: t.plan_cluster = value; break;
+    case MOE_TUNE_PDL: t.pdl = value; break;
+    case MOE_TUNE_PLAN_MATCH: t.plan_match = value; break;
     default: return fail(MOE_EINVAL, "unknown tuning knob %d", static_cast<int>(knob));
     }
     return ok();
@@ -224,6 +283,14 @@ moe_status moe_plan_create(int32_t max_tokens, int32_t k, int32_t E, int32_t R, 
 moe_status moe_plan_create_aligned(int32_t max_tokens, int32_t k, int32_t E, int32_t R,
                                    int32_t align, moe_plan_t *out)
 {
+    return moe_plan_create_ex(max_tokens, k, E, R, align, 0u, out);
+}
+
+moe_status moe_plan_create_ex(int32_t max_tokens, int32_t k, int32_t E, int32_t R, int32_t align,
+                              uint32_t flags, moe_plan_t *out)
+{
+    if (flags & ~static_cast<uint32_t>(MOE_PLAN_NO_DEDUP_LISTS))
+        return fail(MOE_EINVAL, "unknown plan flags 0x%x", flags);
     if (!out)
         return fail(MOE_EINVAL, "out must not be NULL");
     *out = nullptr;
@@ -251,6 +318,7 @@ moe_status moe_plan_create_aligned(int32_t max_tokens, int32_t k, int32_t E, int
     p->rtok_cap = static_cast<int64_t>(max_tokens) * (k < R ? k : R);
     p->align = align;
     p->rows_cap = moe::recv_rows(max_tokens, k, E, align);
+    p->dedup_lists = (flags & MOE_PLAN_NO_DEDUP_LISTS) == 0;
     const int64_t rows = static_cast<int64_t>(max_tokens) * k;
     const int64_t all_rows = p->rows_cap;
     const int64_t nt = p->nt_cap > 0 ? p->nt_cap : 1;
@@ -275,6 +343,7 @@ moe_status moe_plan_create_aligned(int32_t max_tokens, int32_t k, int32_t E, int
         {reinterpret_cast<void **>(&p->tile_cnt), sizeof(int32_t) * E * nt},
         {reinterpret_cast<void **>(&p->tile_rcnt), sizeof(int32_t) * R * nt},
         {reinterpret_cast<void **>(&p->tile_err), sizeof(uint32_t) * nt},
+        {reinterpret_cast<void **>(&p->group_flag), sizeof(uint32_t) * nt},
         {reinterpret_cast<void **>(&p->work), 4 * sizeof(uint32_t)},
         {reinterpret_cast<void **>(&p->ready), sizeof(uint32_t) * (max_tokens > 0 ? max_tokens : 1)},
     };
@@ -543,6 +612,8 @@ moe_status moe_plan_query(moe_plan_t plan, moe_plan_view *v)
     v->err = p->err;
     v->topk_w = p->topk_w;
     v->plan_kernels = p->plan_kernels;
+    v->plan_kind = p->plan_kind;
+    v->dedup_lists = p->dedup_lists ? 1 : 0;
     v->align = p->align;
     v->recv_rows = static_cast<int32_t>(moe::recv_rows(p->N, p->k, p->E, p->align));
     return ok();
@@ -559,8 +630,14 @@ moe_status moe_plan_check(moe_plan_t plan, void *stream, uint32_t *flags)
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaMemcpy(err)");
     if (*flags & MOE_ERR_TIMEOUT) {
-        // a grid barrier was abandoned: rearm its words for the next plan
+        // a grid barrier was abandoned: rearm its words (and clear the error word, which
+        // keeps a timeout until it has been reported here) for the next plan
         e = cudaMemset(plan->sync, 0, 2 * sizeof(uint32_t));
+        if (e == cudaSuccess)
+            e = cudaMemset(plan->err, 0, sizeof(uint32_t));
+        if (e == cudaSuccess)
+            e = cudaMemset(plan->group_flag, 0,
+                           sizeof(uint32_t) * (plan->nt_cap > 0 ? plan->nt_cap : 1));
         if (e != cudaSuccess)
             return cuda_fail(e, "cudaMemset(sync)");
         // and the fused kernel's work words, with its flags (the epoch starts again)
@@ -577,9 +654,10 @@ moe_status moe_wait_selftest(int32_t which, void *stream, uint32_t *flags)
 {
     if (!flags)
         return fail(MOE_EINVAL, "flags must not be NULL");
-    if (which < 0 || which > 2)
+    if (which < 0 || which > 3)
         return fail(MOE_EINVAL,
-                    "which must be 0 (flag wait), 1 (mbarrier wait) or 2 (grid barrier), got %d",
+                    "which must be 0 (flag wait), 1 (mbarrier wait), 2 (grid barrier) or 3 "
+                    "(group exchange), got %d",
                     which);
     cudaError_t e = moe::run_wait_selftest(which, static_cast<cudaStream_t>(stream), flags);
     if (e != cudaSuccess)

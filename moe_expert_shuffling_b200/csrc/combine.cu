@@ -41,6 +41,10 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, CW >= 8 ? 2 : 1)
     const int n_tok = b < static_cast<uint32_t>(p.N)
                           ? static_cast<int>(min(p.per_cta, static_cast<uint32_t>(p.N) - b))
                           : 0;
+    if (threadIdx.x == 0)
+        r.init<CW>();
+    pdl_trigger();
+    pdl_wait();  // the plan and the expert outputs are read from here on
     // the first token's slots (and, for the consumers, weights) are fetched before the
     // barrier so that their latency overlaps the set-up
     int32_t s_first = -1;
@@ -53,8 +57,6 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, CW >= 8 ? 2 : 1)
     if (RANKED)
         for (int q = threadIdx.x; q <= p.R; q += blockDim.x)
             r.roff_s[q] = __ldg(p.rank_off + q);
-    if (threadIdx.x == 0)
-        r.init<CW>();
     __syncthreads();
 
     int i = 0;
@@ -128,8 +130,8 @@ cudaError_t launch_bulk_shape(const CombineArgs &a, int device, cudaStream_t str
         per_cta = std::max<int64_t>(1, ceil_div(a.N, resident));
     p.per_cta = static_cast<uint32_t>(per_cta);
     const int64_t grid = std::max<int64_t>(1, ceil_div(a.N, per_cta));
-    kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream,
+                         false, device, p);
 }
 
 template <bool RANKED>

@@ -167,6 +167,20 @@ __device__ __forceinline__ uint4 lds_v4(const void *p)
     return v;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization
+// may begin while the kernel before it on the stream is still finishing.  pdl_wait() returns
+// once every earlier grid on the stream has completed and its memory operations are visible;
+// every thread calls it before its first access to global memory (which an earlier kernel
+// may still be writing, or still be reading).  pdl_trigger() lets the next kernel on the
+// stream begin launching; it still waits for this grid to complete before its own global
+// accesses.  Both do nothing in a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // gpu-scope acquire / release accesses for flags and counters shared between CTAs.
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *a)
 {
@@ -232,6 +246,39 @@ __device__ __forceinline__ bool grid_barrier(uint32_t *sync, uint32_t *err, uint
             }
         }
         *s_ok = ok;
+    }
+    __syncthreads();
+    return *s_ok != 0;
+}
+
+// Wait (warp 0 of the CTA) until words[0..n) all hold `want` -- the arrival words that the
+// leader CTA of each group of a grid releases (the group plan kernel).  All threads must
+// call.  False after kWaitLimitNs (MOE_ERR_TIMEOUT set).
+__device__ __forceinline__ bool wait_words(const uint32_t *words, uint32_t n, uint32_t want,
+                                           uint32_t *err, int *s_ok)
+{
+    if (threadIdx.x < 32) {
+        const uint32_t lane = threadIdx.x;
+        bool ok = true;
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t it = 0;; ++it) {
+            bool mine = true;
+            for (uint32_t q = lane; q < n; q += 32)
+                mine = mine && ld_acquire_gpu(words + q) == want;
+            if (__all_sync(0xffffffffu, mine))
+                break;
+            if ((it & 15u) == 15u) {
+                const bool late = global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30);
+                if (__shfl_sync(0xffffffffu, late, 0)) {
+                    if (lane == 0)
+                        atomicOr(err, MOE_ERR_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        if (lane == 0)
+            *s_ok = ok;
     }
     __syncthreads();
     return *s_ok != 0;

@@ -39,6 +39,8 @@ __global__ void __launch_bounds__(128) dispatch_bulk_kernel(const DispatchParams
             mbar_init(&bars[s], 1);
         mbar_init_fence();
     }
+    pdl_trigger();
+    pdl_wait();  // the plan's slots and the payload are read from here on
     __syncwarp();
     (void)dispatch_warp_run(p, bars, stage0, u0, n_my, 0u, true);
 }
@@ -48,6 +50,8 @@ __global__ void dispatch_scales_kernel(const float *__restrict__ xs, float *__re
                                        const int32_t *__restrict__ slot, int64_t entries,
                                        int32_t k, int32_t ncols, int32_t n_rows)
 {
+    pdl_trigger();
+    pdl_wait();
     const int64_t total = entries * ncols;
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -136,8 +140,8 @@ cudaError_t launch_dispatch(const DispatchArgs &a, int device, cudaStream_t stre
         per_warp = std::max<int64_t>(1, ceil_div(units, resident_warps));
     p.per_warp = static_cast<uint32_t>(per_warp);
     const int64_t grid = std::max<int64_t>(1, ceil_div(ceil_div(units, per_warp), wpc));
-    dispatch_bulk_kernel<<<static_cast<unsigned>(grid), wpc * 32, smem, stream>>>(p);
-    e = cudaGetLastError();
+    e = launch_kernel(dispatch_bulk_kernel, dim3(static_cast<unsigned>(grid)), dim3(wpc * 32),
+                      smem, stream, false, device, p);
     if (e != cudaSuccess)
         return e;
 
@@ -146,11 +150,11 @@ cudaError_t launch_dispatch(const DispatchArgs &a, int device, cudaStream_t stre
         const int64_t entries = static_cast<int64_t>(a.N) * a.k;
         const int64_t total = entries * ncols;
         const int64_t blocks = std::min<int64_t>(ceil_div(total, 256), sm_count(device) * 8);
-        dispatch_scales_kernel<<<static_cast<unsigned>(std::max<int64_t>(blocks, 1)), 256, 0,
-                                 stream>>>(reinterpret_cast<const float *>(a.xs),
-                                           reinterpret_cast<float *>(a.rs), a.slot, entries, a.k,
-                                           ncols, a.n_rows);
-        e = cudaGetLastError();
+        e = launch_kernel(dispatch_scales_kernel,
+                          dim3(static_cast<unsigned>(std::max<int64_t>(blocks, 1))), dim3(256), 0,
+                          stream, false, device, reinterpret_cast<const float *>(a.xs),
+                          reinterpret_cast<float *>(a.rs), a.slot, entries,
+                          static_cast<int32_t>(a.k), ncols, static_cast<int32_t>(a.n_rows));
     }
     return e;
 }

@@ -43,10 +43,17 @@ namespace {
 //  * 10% of the CTAs starting on dispatch (30% when the combine waits on flags: with fewer,
 //    most CTAs would wait for the few that dispatch).
 // With these the fused step takes 0.95-0.98x the time of the two separate kernels.
+// The wide combine shape for k <= 4 (eight consumer warps, 4 KB per row) was measured on the
+// Mixtral shape: 3 CTAs of 64 KB per SM, combine items of up to 4 tokens (also when they
+// wait on flags) and 30% of the CTAs starting on dispatch; these defaults gave 76-80 us per
+// step against 85-101 us for the narrower shape's defaults.
 constexpr int kDefaultCtasPerSm = 4;
 constexpr int kDefaultSmemKb = 48;
 constexpr int kDefaultDispatchSharePct = 10;
 constexpr int kDefaultDispatchSharePctFlags = 30;
+constexpr int kWideCtasPerSm = 3;
+constexpr int kWideSmemKb = 64;
+constexpr int kWideDispatchSharePct = 30;
 constexpr double kDispatchItemBytes = 256.0 * 1024;
 constexpr double kCombineItemBytes = 512.0 * 1024;
 constexpr uint32_t kMaxCombineRun = 4;
@@ -77,6 +84,8 @@ __global__ void __launch_bounds__(Shape<CW>::kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const DispatchParams &dp = fp.d;
     const CombineBulkParams &cp = fp.c;
+    pdl_trigger();
+    pdl_wait();  // every global access of the launch follows the previous kernel on the stream
 
     // Shared memory: combine mbarriers | combine ring + rank tables, overlaid by the
     // dispatch warps' rings | dispatch mbarriers.  A CTA switches roles only after all of
@@ -261,8 +270,11 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
     // Shared memory: as many 4-stage dispatch rings as the budget holds (at least one,
     // with fewer stages if even one does not fit), and a combine ring using the larger of
     // the budget and the dispatch rings' area.
+    constexpr bool kWide = CW >= 8;
     const size_t budget = static_cast<size_t>(
-        std::min((tu.fused_smem_kb > 0 ? tu.fused_smem_kb : kDefaultSmemKb * CW / 4) * 1024,
+        std::min((tu.fused_smem_kb > 0 ? tu.fused_smem_kb
+                                       : kWide ? kWideSmemKb : kDefaultSmemKb * CW / 4) *
+                     1024,
                  max_optin));
     int d_stages = kDispatchStages;
     while (d_stages > 2 && static_cast<size_t>(d_stages) * g.stage_bytes > budget)
@@ -297,7 +309,8 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
     if (per_sm < 1)
         return cudaErrorInvalidConfiguration;
     per_sm = std::min(per_sm, tu.fused_ctas_per_sm > 0 ? tu.fused_ctas_per_sm
-                                                       : kDefaultCtasPerSm * 4 / CW);
+                              : kWide                     ? kWideCtasPerSm
+                                                          : kDefaultCtasPerSm * 4 / CW);
 
     // work items
     const double d_token_bytes = static_cast<double>(a.d.row_bytes + a.d.srow_bytes) * (1 + a.d.k);
@@ -308,7 +321,7 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
     uint32_t c_run = static_cast<uint32_t>(tu.fused_combine_run);
     if (c_run == 0) {
         const double c_token_bytes = static_cast<double>(c.row_bytes) * (1 + a.c.k);
-        const double div = a.use_flags ? 2.0 : 1.0;
+        const double div = a.use_flags && !kWide ? 2.0 : 1.0;
         c_run = static_cast<uint32_t>(kCombineItemBytes / div / c_token_bytes + 0.5);
         c_run = std::min<uint32_t>(std::max<uint32_t>(c_run, 1),
                                    static_cast<uint32_t>(kMaxCombineRun / div));
@@ -334,6 +347,7 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
         d_first = grid;
     } else {
         const int share = tu.fused_dispatch_share > 0 ? std::min(tu.fused_dispatch_share, 100)
+                          : kWide       ? kWideDispatchSharePct
                           : a.use_flags ? kDefaultDispatchSharePctFlags
                                         : kDefaultDispatchSharePct;
         d_first = grid * share / 100;
@@ -343,20 +357,19 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
 
     // Only the ready-flag waits need every CTA resident at once (cooperative launch); with
     // no flags no CTA waits on another and an ordinary launch, cheaper to start, is enough.
-    if (!a.use_flags) {
-        kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(fp);
-        return cudaGetLastError();
-    }
-    void *args[] = {&fp};
-    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern),
-                                    dim3(static_cast<unsigned>(grid)), dim3(threads), args, smem,
-                                    stream);
-    return e;
+    return launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream,
+                         a.use_flags, device, fp);
 }
 
 template <bool RANKED>
 cudaError_t launch_fused_k(const FusedArgs &a, int device, cudaStream_t stream)
 {
+    // The combine side takes the separate combine kernel's chunk widths: for k <= 4, eight
+    // consumer warps and 4 KB of every row per stage, so that a stage is not a couple of
+    // 2 KB rows with a barrier round each.
+    const int max_cw = tuning().combine_max_cw > 0 ? tuning().combine_max_cw : 8;
+    if (a.c.k <= 4 && max_cw >= 8)
+        return launch_fused_shape<4, 8, RANKED>(a, device, stream);
     if (a.c.k <= 8)
         return launch_fused_shape<8, 4, RANKED>(a, device, stream);
     if (a.c.k <= 16)

@@ -12,6 +12,7 @@ struct moe_plan_s {
     int32_t cap = 0;        // largest N accepted
     int32_t N = 0, k = 0, E = 0, R = 0, epr = 0;
     int32_t align = 1;      // expert segments start on multiples of this many rows
+    bool dedup_lists = true;  // moe_plan writes rtok / fanout
     int32_t nt_cap = 0;     // tiles for `cap` tokens
     int64_t rtok_cap = 0;   // entries of rtok/fanout: cap * min(k, R)
     int64_t rows_cap = 0;   // receive rows for `cap` tokens: cap * k + E * (align - 1)
@@ -25,10 +26,13 @@ struct moe_plan_s {
     uint32_t *fanout = nullptr, *err = nullptr;
     uint32_t *sync = nullptr;  // [2] grid-barrier words of the fused plan kernel (zero at rest)
     // scratch: per-tile counts [E][nt] and [R][nt] (then their column prefixes), tile flags
+    // (the group kernel keeps its groups' totals and flags in the first rows of these)
     int32_t *tile_cnt = nullptr, *tile_rcnt = nullptr;
     uint32_t *tile_err = nullptr;
+    uint32_t *group_flag = nullptr;  // [nt] per-group arrival words of the group plan kernel
     const float *topk_w = nullptr;
     int32_t plan_kernels = 0;  // kernels the last launch_plan enqueued
+    int32_t plan_kind = 0;     // MOE_PLAN_KIND_* of the last launch_plan
     // moe_dispatch_combine: work words [next dispatch item, next combine item, CTAs done,
     // epoch of the last launch] (the launch's last CTA resets the counters and advances the
     // epoch) and per-token ready flags [cap] holding the epoch of the launch that last
@@ -62,7 +66,7 @@ struct Tuning {
     int combine_smem_kb = 0;
     int dispatch_units_per_warp = 0;
     int combine_tokens_per_cta = 0;
-    int plan_engine = 0;       // 0/1: one cooperative kernel when it fits, 2: three kernels
+    int plan_engine = 0;       // 0/1: automatic, 2: three kernels, 3: no cluster kernel
     int fused_ctas_per_sm = 0;
     int fused_dispatch_share = 0;  // percent of CTAs that start on dispatch work
     int fused_dispatch_run = 0;    // tokens per dispatch work item
@@ -70,10 +74,31 @@ struct Tuning {
     int fused_smem_kb = 0;
     int fused_min_kb = 0;          // least traffic for the one-launch kernel
     int combine_max_cw = 0;        // cap on consumer warps per combine CTA (4, 8 or 16)
+    int plan_cluster = 0;          // most tiles per cluster of the group plan kernel (1..16)
+    int pdl = 0;                   // 0/1: programmatic dependent launch, 2: ordinary launches
+    int plan_match = 0;            // 0: by k, 1: shuffle compares, 2: warp match instructions
 };
 Tuning &tuning();
 
 int sm_count(int device);
+
+// Launch `kernel` with cudaLaunchKernelEx, as a programmatic dependent launch (the kernel
+// may begin while the previous kernel on the stream finishes; the kernels wait with
+// pdl_wait before touching global memory) unless MOE_TUNE_PDL turns it off, and
+// cooperatively when asked.  If the runtime refuses the programmatic attribute for a kind
+// of launch on a device, that kind is launched without it from then on.
+cudaError_t launch_ex(const void *kernel, void **args, dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t stream, bool cooperative, int device,
+                      const cudaLaunchAttribute *extra = nullptr, int n_extra = 0);
+
+template <typename... KArgs>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, bool cooperative, int device, KArgs... args)
+{
+    void *ptrs[] = {static_cast<void *>(&args)..., nullptr};
+    return launch_ex(reinterpret_cast<const void *>(kernel), ptrs, grid, block, smem, stream,
+                     cooperative, device);
+}
 
 // Largest dynamic shared memory a CTA may opt into on `device` (cached).
 int max_smem_optin(int device);

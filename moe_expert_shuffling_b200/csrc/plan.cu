@@ -16,10 +16,11 @@
 // By default the phases run in one cooperative kernel (plan_fused_kernel) whose CTAs
 // meet at two sense-reversing grid barriers; a wait gives up after 1 s and reports
 // MOE_ERR_TIMEOUT.  A routing of at most one tile (N <= 128, e.g. a decode step) runs
-// all phases in one CTA (plan_one_tile_kernel), and one of 2..16 tiles on one thread-block
-// cluster with the tile counts shared through distributed shared memory
-// (plan_cluster_kernel).
-// When the grid cannot be co-resident the phases run as three kernels instead.
+// all phases in one CTA (plan_one_tile_kernel).  Larger routings run on thread-block
+// clusters of up to 16 tiles whose counts are combined through distributed shared memory,
+// with one grid-wide exchange of the groups' totals when there is more than one group
+// (plan_group_kernel); the cooperative kernel is the fallback when those clusters cannot
+// all be resident, and three kernels when its grid cannot be co-resident either.
 //
 // Inside a tile a warp looks at several tokens at once: lane = (token, column) with the
 // columns of one token in a segment of W = next power of two >= k lanes, so a token's
@@ -42,12 +43,15 @@ constexpr uint32_t kFull = 0xffffffffu;  // all lanes of a warp
 struct PlanK {
     const int32_t *topk_idx;
     int32_t N, k, E, R, epr, nt, n_rows, align;
+    int32_t match;  // classify with warp match instructions (1) or shuffle compares (0)
+    int32_t lists;  // write the per-rank dedup lists rtok / fanout (0: skip them)
     int64_t rtok_cap;
     int32_t *tile_cnt, *tile_rcnt;
     uint32_t *tile_err;
     int32_t *cnt, *expert_off, *rcnt, *rank_off, *rtok_off, *slot, *src_tok, *src_j, *rtok;
     uint32_t *fanout, *err;
     uint32_t *sync;  // [2] grid-barrier arrival count (zero at rest) and generation
+    uint32_t *group_flag;  // [groups] arrival words of the group kernel
 };
 
 // Classification of one entry, shared by the count and rank kernels so both see the
@@ -78,29 +82,39 @@ __device__ __forceinline__ LaneMap lane_map(int k)
 }
 
 // All 32 lanes must call.  `tl` is the token's index in the tile, `present` whether
-// this lane holds an entry (token in range and column < k).
+// this lane holds an entry (token in range and column < k); W >= k is the width of a token's
+// lane segment.  The W shuffles of each comparison are independent of one another (the
+// loops are unrolled), so they issue back to back instead of one round trip each; lanes
+// q >= k of a segment hold id -1 and rank -1, which match no valid entry.
+template <int W>
 __device__ __forceinline__ Entry classify(const int32_t *ids, const int32_t *rank_of, int tl,
-                                          int j, bool present, int k, int E, int width)
+                                          int j, bool present, int k, int E)
 {
     Entry c;
     const int32_t id = present ? ids[tl * k + j] : -1;
     const bool in_range = present && static_cast<uint32_t>(id) < static_cast<uint32_t>(E);
+    int32_t other[W];
+#pragma unroll
+    for (int q = 0; q < W; ++q)
+        other[q] = __shfl_sync(kFull, id, q, W);
     bool valid = in_range;
-    for (int q = 0; q < k; ++q) {
-        const int32_t iq = __shfl_sync(kFull, id, q, width);
-        if (q < j && iq == id)
+#pragma unroll
+    for (int q = 0; q < W; ++q)
+        if (q < j && other[q] == id)
             valid = false;
-    }
     // -1 marks an entry the router dropped: no row, no contribution, not an error
     c.flags = (present && !in_range && id != -1 ? MOE_ERR_ID_RANGE : 0u) |
               (in_range && !valid ? MOE_ERR_ID_DUP : 0u);
     c.e = valid ? id : -1;
     c.r = valid ? rank_of[id] : -1;
+#pragma unroll
+    for (int q = 0; q < W; ++q)
+        other[q] = __shfl_sync(kFull, c.r, q, W);
     uint32_t mask = 0;
     bool leader = valid;
-    for (int q = 0; q < k; ++q) {
-        const int32_t rq = __shfl_sync(kFull, c.r, q, width);
-        if (valid && rq == c.r) {
+#pragma unroll
+    for (int q = 0; q < W; ++q) {
+        if (valid && other[q] == c.r) {
             if (q < j)
                 leader = false;
             mask |= 1u << q;
@@ -170,8 +184,12 @@ __device__ void scan_into(const int32_t *src, int n, int32_t *dst, int32_t *warp
         dst[n] = carry;
 }
 
-// Shared-memory layout of every plan kernel (words).
+// Shared-memory layout of every plan kernel (words).  The ids come first so that they are
+// 16-byte aligned for vector loads (kPlanTile * k words is a multiple of 4).
 struct PlanSmem {
+    int32_t *ids;       // [kPlanTile * k] the tile's routing ids
+    int32_t *vid;       // [kPlanTile * k] valid id or -1
+    uint32_t *lead;     // [kPlanTile * k] leader masks
     int32_t *eoff;      // [E+1] segment starts of the experts
     int32_t *roff;      // [R+1] starts of the ranks' dedup lists
     int32_t *ebase;     // [E]   tile base per expert; the histogram while counting
@@ -179,9 +197,7 @@ struct PlanSmem {
     int32_t *rank_of;   // [E]   rank of each expert
     uint32_t *emask;    // [E][4] tokens of the tile on each expert
     uint32_t *rmask;    // [R][4] tokens of the tile on each rank
-    int32_t *ids;       // [kPlanTile * k] the tile's routing ids
-    int32_t *vid;       // [kPlanTile * k] valid id or -1
-    uint32_t *lead;     // [kPlanTile * k] leader masks
+    int32_t *end;       // first word after the layout
 };
 
 __host__ __device__ constexpr size_t plan_smem_words(int E, int R, int k)
@@ -193,16 +209,17 @@ __host__ __device__ constexpr size_t plan_smem_words(int E, int R, int k)
 __device__ PlanSmem carve(int32_t *w, int E, int R, int k)
 {
     PlanSmem m;
-    m.eoff = w;
+    m.ids = w;
+    m.vid = m.ids + kPlanTile * k;
+    m.lead = reinterpret_cast<uint32_t *>(m.vid + kPlanTile * k);
+    m.eoff = reinterpret_cast<int32_t *>(m.lead + kPlanTile * k);
     m.roff = m.eoff + E + 1;
     m.ebase = m.roff + R + 1;
     m.rbase = m.ebase + E;
     m.rank_of = m.rbase + R;
     m.emask = reinterpret_cast<uint32_t *>(m.rank_of + E);
     m.rmask = m.emask + 4 * E;
-    m.ids = reinterpret_cast<int32_t *>(m.rmask + 4 * R);
-    m.vid = m.ids + kPlanTile * k;
-    m.lead = reinterpret_cast<uint32_t *>(m.vid + kPlanTile * k);
+    m.end = reinterpret_cast<int32_t *>(m.rmask + 4 * R);
     return m;
 }
 
@@ -218,33 +235,118 @@ __device__ void init_rank_of(const PlanK &p, const PlanSmem &m)
         m.rank_of[e] = e / p.epr;
 }
 
+// The tile's ids into shared memory in one round trip: every thread issues all of its
+// loads (16-byte vectors when the tile's ids are 16-byte aligned) before storing any.
 __device__ void load_ids(const PlanK &p, const PlanSmem &m, int tile, int ntok)
 {
+    constexpr int kVecPerThread = kPlanTile * kMaxTopk / 4 / kPlanThreads;  // 4
     const int32_t *src = p.topk_idx + static_cast<int64_t>(tile) * kPlanTile * p.k;
-    for (int i = threadIdx.x; i < ntok * p.k; i += blockDim.x)
-        m.ids[i] = __ldg(src + i);
+    const int n = ntok * p.k;
+    int head = 0;
+    if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0 && (smem_addr(m.ids) & 15u) == 0) {
+        const int n4 = n >> 2;
+        const int4 *s4 = reinterpret_cast<const int4 *>(src);
+        int4 v[kVecPerThread];
+#pragma unroll
+        for (int q = 0; q < kVecPerThread; ++q) {
+            const int i = threadIdx.x + q * kPlanThreads;
+            if (i < n4)
+                v[q] = __ldg(s4 + i);
+        }
+#pragma unroll
+        for (int q = 0; q < kVecPerThread; ++q) {
+            const int i = threadIdx.x + q * kPlanThreads;
+            if (i < n4)
+                reinterpret_cast<int4 *>(m.ids)[i] = v[q];
+        }
+        head = 4 * n4;
+    }
+    constexpr int kPerThread = 4;
+    for (int base = head; base < n; base += kPerThread * kPlanThreads) {
+        int32_t v[kPerThread];
+#pragma unroll
+        for (int q = 0; q < kPerThread; ++q) {
+            const int i = base + threadIdx.x + q * kPlanThreads;
+            if (i < n)
+                v[q] = __ldg(src + i);
+        }
+#pragma unroll
+        for (int q = 0; q < kPerThread; ++q) {
+            const int i = base + threadIdx.x + q * kPlanThreads;
+            if (i < n)
+                m.ids[i] = v[q];
+        }
+    }
 }
+
+__device__ __forceinline__ void clear_tile_masks(const PlanK &p, const PlanSmem &m)
+{
+    for (int i = threadIdx.x; i < 4 * (p.E + p.R); i += blockDim.x)
+        m.emask[i] = 0u;  // emask and rmask are contiguous
+}
+
+__device__ uint32_t classify_loaded(const PlanK &p, const PlanSmem &m, int ntok);
 
 // Classify a tile's entries into shared memory: vid/lead per entry, and each token's bit
 // in its experts' and ranks' tile masks.  All threads must call; rank_of must be ready.
 // Returns this thread's MOE_ERR_* flags.
 __device__ uint32_t classify_tile(const PlanK &p, const PlanSmem &m, int tile, int ntok)
 {
+    clear_tile_masks(p, m);
+    load_ids(p, m, tile, ntok);
+    return classify_loaded(p, m, ntok);
+}
+
+// classify<W> with two warp match instructions instead of 2W shuffle compares: lanes whose
+// (token, id) keys match hold the same expert, and the lowest of them is the first column;
+// lanes whose (token, rank) keys match are the token's valid columns on one rank.  Lanes
+// without a valid key get one no other lane has.  Ids are below 2^20 (E <= 1024), token
+// segments below 32.
+template <int W>
+__device__ __forceinline__ Entry classify_match(const int32_t *ids, const int32_t *rank_of,
+                                                int tl, int j, bool present, int k, int E)
+{
+    Entry c;
+    const int lane = threadIdx.x & 31;
+    const uint32_t seg = static_cast<uint32_t>(lane / W);
+    const int32_t id = present ? ids[tl * k + j] : -1;
+    const bool in_range = present && static_cast<uint32_t>(id) < static_cast<uint32_t>(E);
+    const uint32_t key = in_range ? (seg << 20) | static_cast<uint32_t>(id)
+                                  : 0x80000000u | static_cast<uint32_t>(lane);
+    const uint32_t same = __match_any_sync(kFull, key);
+    const bool valid = in_range && __ffs(same) - 1 == lane;
+    c.flags = (present && !in_range && id != -1 ? MOE_ERR_ID_RANGE : 0u) |
+              (in_range && !valid ? MOE_ERR_ID_DUP : 0u);
+    c.e = valid ? id : -1;
+    c.r = valid ? rank_of[id] : -1;
+    const uint32_t rkey = valid ? (seg << 20) | static_cast<uint32_t>(c.r)
+                                : 0x80000000u | static_cast<uint32_t>(lane);
+    const uint32_t rsame = __match_any_sync(kFull, rkey);
+    const bool leader = valid && __ffs(rsame) - 1 == lane;
+    const uint32_t cols = W == 32 ? 0xffffffffu : (1u << W) - 1u;
+    c.lead = leader ? (rsame >> (seg * W)) & cols : 0u;
+    return c;
+}
+
+// The warp steps of classify_loaded for one lane-segment width W (a power of two >= k).
+template <int W>
+__device__ __forceinline__ uint32_t classify_steps(const PlanK &p, const PlanSmem &m, int ntok)
+{
+    constexpr int kWbits = W == 1 ? 0 : W == 2 ? 1 : W == 4 ? 2 : W == 8 ? 3 : W == 16 ? 4 : 5;
+    constexpr int kPerStep = 32 / W;  // tokens per warp step
+    constexpr int kSteps = (kPlanTokensPerWarp + kPerStep - 1) / kPerStep;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int k = p.k;
-    for (int i = threadIdx.x; i < 4 * (p.E + p.R); i += blockDim.x)
-        m.emask[i] = 0u;  // emask and rmask are contiguous
-    load_ids(p, m, tile, ntok);
-    __syncthreads();
-    const LaneMap lm = lane_map(k);
-    const int j = lane & ((1 << lm.wbits) - 1);
-    const int sub = lane >> lm.wbits;
+    const int j = lane & (W - 1);
+    const int sub = lane >> kWbits;
     uint32_t flags = 0;
-    for (int st = 0; st < lm.steps; ++st) {
-        const int tw = st * lm.per_step + sub;           // token within the warp's 16
+#pragma unroll 1
+    for (int st = 0; st < kSteps; ++st) {
+        const int tw = st * kPerStep + sub;           // token within the warp's 16
         const int tl = warp * kPlanTokensPerWarp + tw;
         const bool present = tw < kPlanTokensPerWarp && tl < ntok && j < k;
-        const Entry c = classify(m.ids, m.rank_of, tl, j, present, k, p.E, 1 << lm.wbits);
+        const Entry c = p.match ? classify_match<W>(m.ids, m.rank_of, tl, j, present, k, p.E)
+                                : classify<W>(m.ids, m.rank_of, tl, j, present, k, p.E);
         flags |= c.flags;
         if (present) {
             m.vid[tl * k + j] = c.e;
@@ -255,6 +357,22 @@ __device__ uint32_t classify_tile(const PlanK &p, const PlanSmem &m, int tile, i
             if (c.lead)
                 atomicOr(&m.rmask[4 * c.r + (tl >> 5)], bit);
         }
+    }
+    return flags;
+}
+
+// classify_tile once the masks are clear and the ids are being stored (synchronises first).
+__device__ uint32_t classify_loaded(const PlanK &p, const PlanSmem &m, int ntok)
+{
+    __syncthreads();
+    uint32_t flags;
+    switch (1 << lane_map(p.k).wbits) {  // block-uniform
+    case 1: flags = classify_steps<1>(p, m, ntok); break;
+    case 2: flags = classify_steps<2>(p, m, ntok); break;
+    case 4: flags = classify_steps<4>(p, m, ntok); break;
+    case 8: flags = classify_steps<8>(p, m, ntok); break;
+    case 16: flags = classify_steps<16>(p, m, ntok); break;
+    default: flags = classify_steps<32>(p, m, ntok); break;
     }
     __syncthreads();
     return flags;
@@ -286,12 +404,13 @@ __device__ void count_tile(const PlanK &p, const PlanSmem &m, int tile, uint32_t
     __syncthreads();
 }
 
-// Segment sizes are the counts rounded up to the alignment.  Also marks every receive
-// row that no entry maps to (segment padding and rows after the last segment) with -1
-// in src_tok/src_j, spread over all CTAs of the grid.
-// Segment offsets from m.ebase (segment sizes) and m.rbase (rank counts), which the caller
-// has filled; the rest as rank_prepare.
-__device__ void prepare_offsets(const PlanK &p, const PlanSmem &m, int32_t *warp_sums);
+// Segment offsets from m.ebase (segment sizes: the counts rounded up to the alignment) and
+// m.rbase (rank counts), which the caller has filled; `raw_cnt` holds the expert counts
+// (shared memory when `raw_shared`, else the global cnt array).  Block 0 writes the offset
+// arrays; every receive row that no entry maps to (segment padding and rows after the last
+// segment) is marked -1 in src_tok/src_j, spread over all CTAs of the grid.
+__device__ void prepare_offsets(const PlanK &p, const PlanSmem &m, int32_t *warp_sums,
+                                const int32_t *raw_cnt, bool raw_shared);
 
 __device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_sums)
 {
@@ -303,10 +422,11 @@ __device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_su
             m.rbase[i - p.E] = __ldcg(p.rcnt + (i - p.E));
         }
     }
-    prepare_offsets(p, m, warp_sums);
+    prepare_offsets(p, m, warp_sums, p.cnt, false);
 }
 
-__device__ void prepare_offsets(const PlanK &p, const PlanSmem &m, int32_t *warp_sums)
+__device__ void prepare_offsets(const PlanK &p, const PlanSmem &m, int32_t *warp_sums,
+                                const int32_t *raw_cnt, bool raw_shared)
 {
     __syncthreads();
     scan_into(m.ebase, p.E, m.eoff, warp_sums);
@@ -322,7 +442,7 @@ __device__ void prepare_offsets(const PlanK &p, const PlanSmem &m, int32_t *warp
     }
     if (p.align > 1) {
         for (int e = blockIdx.x; e < p.E; e += gridDim.x) {
-            const int32_t first = m.eoff[e] + __ldcg(p.cnt + e);
+            const int32_t first = m.eoff[e] + (raw_shared ? raw_cnt[e] : __ldcg(raw_cnt + e));
             for (int32_t r = first + threadIdx.x; r < m.eoff[e + 1]; r += blockDim.x) {
                 p.src_tok[r] = -1;
                 p.src_j[r] = -1;
@@ -387,7 +507,7 @@ __device__ void rank_entries(const PlanK &p, const PlanSmem &m, int tile, int nt
                 s = -1;
             }
             const uint32_t msk = m.lead[i];
-            if (msk) {
+            if (msk && p.lists) {
                 const int32_t r = m.rank_of[e];
                 const int32_t pos = m.rbase[r] + bits_below(&m.rmask[4 * r], tl);
                 if (pos >= 0 && pos < p.rtok_cap) {
@@ -408,17 +528,20 @@ __device__ void rank_entries(const PlanK &p, const PlanSmem &m, int tile, int nt
 // ------------------------------------------------------------- three-kernel path
 __global__ void __launch_bounds__(kPlanThreads) plan_count_kernel(const PlanK p)
 {
-    extern __shared__ int32_t smem[];
+    extern __shared__ __align__(16) int32_t smem[];
     __shared__ uint32_t s_err;
     const PlanSmem m = carve(smem, p.E, p.R, p.k);
     init_rank_of(p, m);
+    pdl_wait();
     count_tile(p, m, blockIdx.x, &s_err);
+    pdl_trigger();  // late, so that the next kernel's CTAs do not wait beside this one's work
 }
 
 __global__ void __launch_bounds__(kScanThreads) plan_scan_kernel(const PlanK p)
 {
     __shared__ int32_t warp_sums[kScanThreads / 32];
     __shared__ uint32_t s_err;
+    pdl_wait();
     const int row = blockIdx.x;
     int32_t *rp = row < p.E ? p.tile_cnt + static_cast<int64_t>(row) * p.nt
                             : p.tile_rcnt + static_cast<int64_t>(row - p.E) * p.nt;
@@ -451,15 +574,18 @@ __global__ void __launch_bounds__(kScanThreads) plan_scan_kernel(const PlanK p)
         if (threadIdx.x == 0)
             *p.err = s_err;
     }
+    pdl_trigger();
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_rank_kernel(const PlanK p)
 {
-    extern __shared__ int32_t smem[];
+    extern __shared__ __align__(16) int32_t smem[];
     __shared__ int32_t warp_sums[kPlanThreads / 32];
     const PlanSmem m = carve(smem, p.E, p.R, p.k);
     init_rank_of(p, m);
+    pdl_wait();
     rank_prepare(p, m, warp_sums);
+    pdl_trigger();
     rank_tile(p, m, blockIdx.x, false);
 }
 
@@ -468,13 +594,15 @@ __global__ void __launch_bounds__(kPlanThreads) plan_rank_kernel(const PlanK p)
 // scratch, no grid barrier and no cooperative launch is needed.
 __global__ void __launch_bounds__(kPlanThreads) plan_one_tile_kernel(const PlanK p)
 {
-    extern __shared__ int32_t smem[];
+    extern __shared__ __align__(16) int32_t smem[];
     __shared__ uint32_t s_err;
     __shared__ int32_t warp_sums[kPlanThreads / 32];
     const PlanSmem m = carve(smem, p.E, p.R, p.k);
     if (threadIdx.x == 0)
         s_err = 0;
+    pdl_trigger();
     init_rank_of(p, m);
+    pdl_wait();  // the routing and the plan's arrays are accessed from here on
     const int ntok = tile_tokens(p, 0);
     const uint32_t flags = classify_tile(p, m, 0, ntok);  // synchronises first
     if (flags)
@@ -494,7 +622,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_one_tile_kernel(const PlanK
     __syncthreads();
     if (threadIdx.x == 0)
         *p.err = s_err;  // before any MOE_ERR_BOUNDS of the rank step is or-ed in
-    prepare_offsets(p, m, warp_sums);
+    prepare_offsets(p, m, warp_sums, p.cnt, false);
     // the tile's bases are the segment starts themselves
     for (int e = threadIdx.x; e < p.E; e += blockDim.x)
         m.ebase[e] = m.eoff[e];
@@ -505,90 +633,287 @@ __global__ void __launch_bounds__(kPlanThreads) plan_one_tile_kernel(const PlanK
         rank_entries(p, m, 0, ntok);
 }
 
-// ------------------------------------------- a few tiles on one thread-block cluster
-// Routings of 2..kClusterTiles tiles: one CTA per tile in one cluster.  Each CTA counts its
-// tile; after the cluster barrier every CTA reads all tiles' counts from the other CTAs'
-// shared memory (distributed shared memory) to get its tile base and the totals.  The
-// cluster's hardware barrier replaces the grid barriers, and no global scratch is used.
-// Every CTA takes the same two barriers whatever its data.  Up to 16 tiles: clusters of
-// more than 8 CTAs are opted into (non-portable size, which sm_100 supports); the launch
-// falls back to the cooperative kernel when such a cluster cannot be resident.
-constexpr int kClusterTiles = 16;
+// ------------------------------------------- groups of tiles on thread-block clusters
+// One CTA per tile; the tiles are grouped C at a time (C <= 16) into thread-block clusters.
+// Inside a group the tile counts are combined through distributed shared memory: each CTA
+// scans the rows it owns (row % C == its rank) across the group's C tiles with warp
+// shuffles and writes every tile's prefix (its base within the group) back into that
+// tile's CTA.  With one group the totals are final and are written back the same way.
+// With several, each group stores its totals in global memory and its leader CTA releases
+// the group's arrival word; every CTA then reads all groups' totals and adds up those of
+// the earlier groups (its group's base) and of all groups (the segment sizes) by itself.
+// That one exchange replaces the two grid barriers and the scan phase of the cooperative
+// kernel.  Every CTA takes the same cluster barriers whatever its data; the exchange's
+// wait gives up after the wait limit.  The launch is cooperative with several groups
+// (they wait on each other), and the host checks that all of its clusters can be resident.
+//
+// Work that depends only on the CTA's own tile runs before the exchange: the tile-local
+// offsets of every expert and rank (scans of the tile counts), and a staging order of the
+// tile's entries by (expert, token) and of its leaders by (rank, token) in shared memory.
+// After the exchange the receive-row inverse maps and the dedup lists are then stored in
+// runs of consecutive addresses, one run per (tile, expert) and per (tile, rank), rather
+// than one scattered word per entry.
+constexpr int kMaxClusterTiles = 16;
 
-__host__ __device__ constexpr size_t plan_cluster_smem_words(int E, int R, int k)
+// Shared memory of the group kernel after the common layout (words).
+struct GroupSmem {
+    int32_t *tc;     // [E+R] this tile's counts (read by the group's other CTAs)
+    int32_t *tb;     // [E+R] this tile's base: earlier tiles of its group, then of all
+    int32_t *tot;    // [E+R] the routing's counts
+    int32_t *loff;   // [E+1] tile-local first entry of each expert in the staging order
+    int32_t *lroff;  // [R+1] tile-local first leader of each rank in the staging order
+    int32_t *qloc;   // [kPlanTile * k] each entry's rank among the tile's entries of its expert
+    int32_t *lstage; // [kPlanTile * min(k, R)] leaders by (rank, token): rank << 16 | entry
+};
+
+__host__ __device__ constexpr size_t plan_group_smem_words(int E, int R, int k)
 {
-    return plan_smem_words(E, R, k) + 2 * static_cast<size_t>(E + R);
+    return plan_smem_words(E, R, k) + 3 * static_cast<size_t>(E + R) + (E + 1) + (R + 1) +
+           static_cast<size_t>(kPlanTile) * k + static_cast<size_t>(kPlanTile) * (k < R ? k : R);
 }
 
-__global__ void __launch_bounds__(kPlanThreads) plan_cluster_kernel(const PlanK p)
+__device__ __forceinline__ GroupSmem carve_group(const PlanSmem &m, int E, int R, int k)
+{
+    GroupSmem q;
+    const int ER = E + R;
+    q.tc = m.end;
+    q.tb = q.tc + ER;
+    q.tot = q.tb + ER;
+    q.loff = q.tot + ER;
+    q.lroff = q.loff + E + 1;
+    q.qloc = q.lroff + R + 1;
+    q.lstage = q.qloc + kPlanTile * k;
+    return q;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_group_kernel(const PlanK p)
 {
     namespace cg = cooperative_groups;
-    extern __shared__ int32_t smem[];
+    extern __shared__ __align__(16) int32_t smem[];
     __shared__ uint32_t s_err;
     __shared__ int32_t warp_sums[kPlanThreads / 32];
+    __shared__ int s_ok;
+    __shared__ uint32_t s_gen;  // the exchange generation, read once and shared by the CTA
     cg::cluster_group cluster = cg::this_cluster();
     const PlanSmem m = carve(smem, p.E, p.R, p.k);
-    int32_t *tc = reinterpret_cast<int32_t *>(m.lead + kPlanTile * p.k);  // [E+R] tile counts
-    int32_t *tb = tc + (p.E + p.R);                                       // [E+R] tile bases
-    const int tile = static_cast<int>(cluster.block_rank());  // the grid is one cluster
+    const GroupSmem q = carve_group(m, p.E, p.R, p.k);
+    const int ER = p.E + p.R;
+    const int k = p.k;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int C = static_cast<int>(cluster.num_blocks());
+    const int c = static_cast<int>(cluster.block_rank());
+    const uint32_t G = gridDim.x / static_cast<uint32_t>(C);  // groups (clusters are 1-D)
+    const int g = static_cast<int>(blockIdx.x) / C;
+    const int tile = static_cast<int>(blockIdx.x);
     const int ntok = tile_tokens(p, tile);
-    if (threadIdx.x == 0)
-        s_err = 0;
+    const bool multi = G > 1;
+
+    // Shared-memory set-up overlaps the previous kernel on the stream; global memory is
+    // touched only after pdl_wait.
     init_rank_of(p, m);
-    const uint32_t flags = classify_tile(p, m, tile, ntok);  // synchronises first
+    clear_tile_masks(p, m);
+    if (threadIdx.x == 0)
+        s_err = 0u;
+    pdl_wait();
+    load_ids(p, m, tile, ntok);
+    if (threadIdx.x == 0) {
+        s_gen = multi ? __ldcg(&p.sync[1]) : 0u;
+        // Clear the error word before any CTA can or bits into it (all of that happens after
+        // the cluster barrier below, and after the exchange with several groups).  A timeout
+        // of an earlier call stays until moe_plan_check rearms the plan.
+        if (blockIdx.x == 0)
+            atomicAnd(p.err, MOE_ERR_TIMEOUT);
+    }
+    const uint32_t flags = classify_loaded(p, m, ntok);  // synchronises first and last
     if (flags)
         atomicOr(&s_err, flags);
+    for (int row = threadIdx.x; row < ER; row += blockDim.x) {
+        const uint32_t *mk = row < p.E ? &m.emask[4 * row] : &m.rmask[4 * (row - p.E)];
+        q.tc[row] = __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+    }
+    __syncthreads();
+    // Tile-local offsets and the staging orders (this tile's data only).
+    scan_into(q.tc, p.E, q.loff, warp_sums);
+    scan_into(q.tc + p.E, p.R, q.lroff, warp_sums);
+    __syncthreads();
+    {
+        const LaneMap lm = lane_map(k);
+        const int j = lane & ((1 << lm.wbits) - 1);
+        const int sub = lane >> lm.wbits;
+        int32_t *estage = m.ids;  // the ids are no longer needed: entries by (expert, token)
+        for (int st = 0; st < lm.steps; ++st) {
+            const int tw = st * lm.per_step + sub;
+            const int tl = warp * kPlanTokensPerWarp + tw;
+            if (!(tw < kPlanTokensPerWarp && tl < ntok && j < k))
+                continue;
+            const int i = tl * k + j;
+            const int32_t e = m.vid[i];
+            if (e < 0)
+                continue;
+            const int32_t r_e = bits_below(&m.emask[4 * e], tl);
+            q.qloc[i] = r_e;
+            estage[q.loff[e] + r_e] = (e << 16) | i;
+            if (m.lead[i] && p.lists) {
+                const int32_t r = m.rank_of[e];
+                q.lstage[q.lroff[r] + bits_below(&m.rmask[4 * r], tl)] = (r << 16) | i;
+            }
+        }
+    }
+    cluster.sync();  // (A) every tile's counts and flags are visible to its group
+
+    // The rows this CTA owns (row % C == c): lane qq of a segment of `width` lanes reads the
+    // count of the group's tile qq; a segmented inclusive scan gives each tile's base.
+    {
+        int width = 1;
+        while (width < C)
+            width <<= 1;
+        const int per_warp = 32 / width;
+        const int qq = lane & (width - 1);
+        const int slot_in_warp = lane / width;
+        const int n_own = c < ER ? (ER - c + C - 1) / C : 0;
+        for (int i0 = warp * per_warp; i0 < n_own; i0 += kPlanWarps * per_warp) {
+            const int i = i0 + slot_in_warp;
+            const int row = c + C * i;
+            const bool ok = i < n_own && qq < C;
+            const int32_t v = ok ? cluster.map_shared_rank(q.tc, qq)[row] : 0;
+            int32_t incl = v;
+            for (int o = 1; o < width; o <<= 1) {
+                const int32_t y = __shfl_up_sync(kFull, incl, o, width);
+                if (qq >= o)
+                    incl += y;
+            }
+            const int32_t total = __shfl_sync(kFull, incl, width - 1, width);
+            if (ok) {
+                cluster.map_shared_rank(q.tb, qq)[row] = incl - v;
+                if (!multi)
+                    cluster.map_shared_rank(q.tot, qq)[row] = total;
+                else if (qq == 0) {
+                    if (row < p.E)
+                        p.tile_cnt[static_cast<int64_t>(g) * p.E + row] = total;
+                    else
+                        p.tile_rcnt[static_cast<int64_t>(g) * p.R + (row - p.E)] = total;
+                }
+            }
+        }
+    }
+    if (c == 0 && threadIdx.x == 0) {
+        uint32_t f = 0u;
+        for (int qq = 0; qq < C; ++qq)
+            f |= *cluster.map_shared_rank(&s_err, qq);
+        if (multi)
+            p.tile_err[g] = f;
+        else if (f)
+            atomicOr(p.err, f);
+    }
+    if (multi)
+        __threadfence();  // the group's totals are visible GPU-wide before its leader arrives
+    cluster.sync();       // (B) bases and totals are in place; no DSMEM access after this
+
+    if (multi) {
+        uint32_t want = s_gen + 1u;  // s_gen was set before the barriers above
+        if (want == 0u)
+            want = 1u;  // arrival words start at 0: the generation never takes that value
+        if (c == 0 && threadIdx.x == 0)
+            st_release_gpu(&p.group_flag[g], want);
+        if (!wait_words(p.group_flag, G, want, p.err, &s_ok))
+            return;
+        if (blockIdx.x == 0 && threadIdx.x == 0)
+            p.sync[1] = want;  // every CTA read the old generation before its group arrived
+        for (int row = threadIdx.x; row < ER; row += blockDim.x) {
+            const int32_t *col = row < p.E ? p.tile_cnt + row : p.tile_rcnt + (row - p.E);
+            const int stride = row < p.E ? p.E : p.R;
+            int32_t before = 0, total = 0;
+#pragma unroll 8
+            for (uint32_t gg = 0; gg < G; ++gg) {
+                const int32_t v = __ldcg(col + static_cast<int64_t>(gg) * stride);
+                before += static_cast<int>(gg) < g ? v : 0;
+                total += v;
+            }
+            q.tb[row] += before;
+            q.tot[row] = total;
+        }
+        if (blockIdx.x == 0 && threadIdx.x < 32) {
+            uint32_t f = 0u;
+            for (uint32_t gg = threadIdx.x; gg < G; gg += 32)
+                f |= __ldcg(p.tile_err + gg);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                f |= __shfl_xor_sync(kFull, f, o);
+            if (threadIdx.x == 0 && f)
+                atomicOr(p.err, f);
+        }
+        __syncthreads();
+    }
+    // Only the output stores remain: let the next kernel on the stream start launching.
+    pdl_trigger();
+
+    // Segment sizes are the counts rounded up to the alignment; block 0 publishes the counts.
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
-        const uint32_t *mk = &m.emask[4 * e];
-        tc[e] = __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+        m.ebase[e] = (q.tot[e] + p.align - 1) / p.align * p.align;
+        if (blockIdx.x == 0)
+            p.cnt[e] = q.tot[e];
     }
     for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
-        const uint32_t *mk = &m.rmask[4 * r];
-        tc[p.E + r] = __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+        m.rbase[r] = q.tot[p.E + r];
+        if (blockIdx.x == 0)
+            p.rcnt[r] = q.tot[p.E + r];
     }
-    cluster.sync();  // every tile's counts and flags are visible to the cluster
-
-    // this tile's base (earlier tiles) and the total of every expert / rank row
-    for (int row = threadIdx.x; row < p.E + p.R; row += blockDim.x) {
-        int32_t before = 0, total = 0;
-        for (int c = 0; c < C; ++c) {
-            const int32_t v = cluster.map_shared_rank(tc, c)[row];
-            before += c < tile ? v : 0;
-            total += v;
-        }
-        tb[row] = before;
-        // every CTA writes the same totals, so each reads back its own writes below
-        if (row < p.E) {
-            p.cnt[row] = total;
-            m.ebase[row] = (total + p.align - 1) / p.align * p.align;
-        } else {
-            p.rcnt[row - p.E] = total;
-            m.rbase[row - p.E] = total;
-        }
-    }
-    if (tile == 0 && threadIdx.x == 0) {
-        uint32_t f = 0;
-        for (int c = 0; c < C; ++c)
-            f |= *cluster.map_shared_rank(&s_err, c);
-        *p.err = f;  // before any MOE_ERR_BOUNDS of the rank step is or-ed in
-    }
-    cluster.sync();  // no shared memory is read across the cluster after this point
-
-    prepare_offsets(p, m, warp_sums);
+    prepare_offsets(p, m, warp_sums, q.tot, true);  // synchronises first
     for (int e = threadIdx.x; e < p.E; e += blockDim.x)
-        m.ebase[e] = m.eoff[e] + tb[e];
+        m.ebase[e] = m.eoff[e] + q.tb[e];
     for (int r = threadIdx.x; r < p.R; r += blockDim.x)
-        m.rbase[r] = m.roff[r] + tb[p.E + r];
+        m.rbase[r] = m.roff[r] + q.tb[p.E + r];
     __syncthreads();
-    rank_entries(p, m, tile, ntok);
+
+    // The stores: slot in entry order, the inverse maps in (expert, token) order, the dedup
+    // lists in (rank, token) order -- consecutive threads write consecutive addresses.
+    const int64_t t0 = static_cast<int64_t>(tile) * kPlanTile;
+    const int n_ent = ntok * k;
+    uint32_t bad = 0u;
+    for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
+        const int32_t e = m.vid[i];
+        int32_t sv = -1;
+        if (e >= 0) {
+            sv = m.ebase[e] + q.qloc[i];
+            if (static_cast<uint32_t>(sv) >= static_cast<uint32_t>(p.n_rows)) {
+                bad |= MOE_ERR_BOUNDS;
+                sv = -1;
+            }
+        }
+        p.slot[t0 * k + i] = sv;
+    }
+    const int32_t n_valid = q.loff[p.E];
+    const int32_t *estage = m.ids;
+    for (int x = threadIdx.x; x < n_valid; x += blockDim.x) {
+        const int32_t v = estage[x];
+        const int32_t e = v >> 16, i = v & 0xffff;
+        const int32_t sv = m.ebase[e] + (x - q.loff[e]);
+        if (static_cast<uint32_t>(sv) < static_cast<uint32_t>(p.n_rows)) {
+            p.src_tok[sv] = static_cast<int32_t>(t0 + i / k);
+            p.src_j[sv] = i % k;
+        }
+    }
+    const int32_t n_lead = p.lists ? q.lroff[p.R] : 0;
+    for (int x = threadIdx.x; x < n_lead; x += blockDim.x) {
+        const int32_t v = q.lstage[x];
+        const int32_t r = v >> 16, i = v & 0xffff;
+        const int32_t pos = m.rbase[r] + (x - q.lroff[r]);
+        if (pos >= 0 && pos < p.rtok_cap) {
+            p.rtok[pos] = static_cast<int32_t>(t0 + i / k);
+            p.fanout[pos] = m.lead[i];
+        } else {
+            bad |= MOE_ERR_BOUNDS;
+        }
+    }
+    if (bad)
+        atomicOr(p.err, bad);
 }
 
 // ----------------------------------------------------------- fused (cooperative)
 
 __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
 {
-    extern __shared__ int32_t smem[];
+    extern __shared__ __align__(16) int32_t smem[];
     __shared__ uint32_t s_err;
     __shared__ int32_t warp_sums[kPlanThreads / 32];
     __shared__ int s_ok;
@@ -596,8 +921,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
     const uint32_t G = gridDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-    uint32_t gen = threadIdx.x == 0 ? ld_acquire_gpu(&p.sync[1]) : 0u;
     init_rank_of(p, m);
+    pdl_wait();  // the routing and the plan's arrays are accessed from here on
+    uint32_t gen = threadIdx.x == 0 ? ld_acquire_gpu(&p.sync[1]) : 0u;
     for (int tile = blockIdx.x; tile < p.nt; tile += G)
         count_tile(p, m, tile, &s_err);
     if (!grid_barrier(p.sync, p.err, gen, &s_ok))
@@ -655,6 +981,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
     }
     if (!grid_barrier(p.sync, p.err, gen, &s_ok))
         return;
+    pdl_trigger();  // only the rank phase remains: let the next kernel start launching
 
     rank_prepare(p, m, warp_sums);
     // With one tile per CTA the count phase left that tile's classification in smem.
@@ -677,6 +1004,13 @@ PlanK make_params(const int32_t *topk_idx, int32_t N, int32_t k, int32_t E, int3
     p.align = align;
     p.n_rows = static_cast<int32_t>(recv_rows(N, k, E, align));
     p.rtok_cap = rtok_cap;
+    // Match instructions for the widest rows of ids (k > 16); shuffle compares below that.
+    // Measured on B200 at 16384 tokens of 256 experts: k = 32 plans in 42 us with match
+    // instructions against 46 with shuffles; at k = 16 the shuffles are faster (26 against
+    // 27 us), at k <= 8 clearly so.
+    const int mode = tuning().plan_match;
+    p.match = mode == 2 ? 1 : mode == 1 ? 0 : (k > 16 ? 1 : 0);
+    p.lists = 1;
     return p;
 }
 
@@ -702,49 +1036,123 @@ bool ensure_attrs(int dev)
     return true;
 }
 
-cudaError_t launch_three(const PlanK &p, cudaStream_t stream)
+cudaError_t launch_three(const PlanK &p, int device, cudaStream_t stream)
 {
     const size_t smem = sizeof(int32_t) * plan_smem_words(p.E, p.R, p.k);
+    cudaError_t e = cudaSuccess;
     if (p.nt > 0)
-        plan_count_kernel<<<p.nt, kPlanThreads, smem, stream>>>(p);
-    plan_scan_kernel<<<p.E + p.R, kScanThreads, 0, stream>>>(p);
-    plan_rank_kernel<<<p.nt > 0 ? p.nt : 1, kPlanThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+        e = launch_kernel(plan_count_kernel, dim3(p.nt), dim3(kPlanThreads), smem, stream, false,
+                          device, p);
+    if (e == cudaSuccess)
+        e = launch_kernel(plan_scan_kernel, dim3(p.E + p.R), dim3(kScanThreads), 0, stream,
+                          false, device, p);
+    if (e == cudaSuccess)
+        e = launch_kernel(plan_rank_kernel, dim3(p.nt > 0 ? p.nt : 1), dim3(kPlanThreads), smem,
+                          stream, false, device, p);
+    return e;
 }
 
 }  // namespace
 
-// Whether a cluster of `nt` plan CTAs with `smem` bytes each can be resident (cached: the
-// answer depends only on these and the device).
-bool cluster_fits(int nt, size_t smem, int device, const cudaLaunchConfig_t *cfg, int *clusters)
+namespace {
+
+// How many clusters of the group kernel, `C` CTAs with `smem` bytes each, can be resident at
+// once on `device` (cached: the answer depends only on these).  -1 when the query fails.
+int group_clusters_resident(int C, size_t smem, int device, const cudaLaunchConfig_t *cfg)
 {
     struct Fit {
-        int nt, device;
+        int C, device;
         size_t smem;
         int clusters;
     };
     static Fit cache[64];
     static int n_cache = 0;
     for (int i = 0; i < n_cache; ++i)
-        if (cache[i].nt == nt && cache[i].device == device && cache[i].smem == smem) {
-            *clusters = cache[i].clusters;
-            return true;
-        }
+        if (cache[i].C == C && cache[i].device == device && cache[i].smem == smem)
+            return cache[i].clusters;
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, reinterpret_cast<const void *>(plan_cluster_kernel),
-                                       cfg) != cudaSuccess)
-        return false;
+    if (cudaOccupancyMaxActiveClusters(&c, reinterpret_cast<const void *>(plan_group_kernel),
+                                       cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        c = -1;
+    }
     if (n_cache < 64)
-        cache[n_cache++] = {nt, device, smem, c};
-    *clusters = c;
+        cache[n_cache++] = {C, device, smem, c};
+    return c;
+}
+
+// The group kernel on `nt` >= 2 tiles, if its clusters can all be resident; false (nothing
+// enqueued) otherwise.  Clusters of more than 8 CTAs use the non-portable size that sm_100
+// allows.  With several groups the launch is cooperative; if the runtime refuses a
+// cooperative cluster launch, the group kernel is not used again on that device.
+bool launch_groups(const PlanK &p, int device, cudaStream_t stream, cudaError_t *err)
+{
+    static int non_portable[64] = {0};  // 1: allowed, -1: refused
+    static int coop_clusters[64] = {0}; // -1: a cooperative cluster launch was refused
+    const int dv = device >= 0 && device < 64 ? device : 0;
+    if (coop_clusters[dv] < 0)
+        return false;
+    const size_t smem = sizeof(int32_t) * plan_group_smem_words(p.E, p.R, p.k);
+    if (smem > static_cast<size_t>(max_smem_optin(device)))
+        return false;
+    int per_sm = 0;
+    if (kernel_fit(reinterpret_cast<const void *>(plan_group_kernel), device, kPlanThreads, smem,
+                   &per_sm) != cudaSuccess ||
+        per_sm < 1) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    int cmax = tuning().plan_cluster > 0 ? std::min(tuning().plan_cluster, kMaxClusterTiles)
+                                         : kMaxClusterTiles;
+    if (cmax > 8) {
+        if (non_portable[dv] == 0)
+            non_portable[dv] = cudaFuncSetAttribute(plan_group_kernel,
+                                                    cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                                    1) == cudaSuccess ? 1 : -1;
+        if (non_portable[dv] < 0) {
+            (void)cudaGetLastError();
+            cmax = 8;
+        }
+    }
+    const int C = std::min(cmax, p.nt);
+    const int G = static_cast<int>(ceil_div(p.nt, C));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(G * C));
+    cfg.blockDim = dim3(kPlanThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (group_clusters_resident(C, smem, device, &cfg) < G)
+        return false;
+    PlanK arg = p;
+    void *args[] = {&arg};
+    const cudaError_t e = launch_ex(reinterpret_cast<const void *>(plan_group_kernel), args,
+                                    cfg.gridDim, cfg.blockDim, smem, stream, G > 1, device, attr,
+                                    1);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        if (G > 1)
+            coop_clusters[dv] = -1;
+        return false;
+    }
+    *err = cudaSuccess;
     return true;
 }
+
+}  // namespace
 
 cudaError_t launch_plan(moe_plan_s *pl, const int32_t *topk_idx, cudaStream_t stream)
 {
     if (!ensure_attrs(pl->device))
         return cudaGetLastError() != cudaSuccess ? cudaGetLastError() : cudaErrorUnknown;
     PlanK p = make_params(topk_idx, pl->N, pl->k, pl->E, pl->R, pl->align, pl->rtok_cap);
+    p.lists = pl->dedup_lists ? 1 : 0;
     p.tile_cnt = pl->tile_cnt;
     p.tile_rcnt = pl->tile_rcnt;
     p.tile_err = pl->tile_err;
@@ -760,50 +1168,27 @@ cudaError_t launch_plan(moe_plan_s *pl, const int32_t *topk_idx, cudaStream_t st
     p.fanout = pl->fanout;
     p.err = pl->err;
     p.sync = pl->sync;
+    p.group_flag = pl->group_flag;
 
-    if (tuning().plan_engine != 2 && p.nt <= 1) {
+    const int engine = tuning().plan_engine;
+    if (engine != 2 && p.nt <= 1) {
         // A single tile: one ordinary launch of one CTA.
         const size_t smem = sizeof(int32_t) * plan_smem_words(p.E, p.R, p.k);
         pl->plan_kernels = 1;
-        plan_one_tile_kernel<<<1, kPlanThreads, smem, stream>>>(p);
-        return cudaGetLastError();
+        pl->plan_kind = MOE_PLAN_KIND_ONE_TILE;
+        return launch_kernel(plan_one_tile_kernel, dim3(1), dim3(kPlanThreads), smem, stream,
+                             false, pl->device, p);
     }
-    if (tuning().plan_engine != 2 && p.nt <= kClusterTiles) {
-        // A few tiles: one cluster of one CTA per tile, when such a cluster can be resident.
-        const size_t smem = sizeof(int32_t) * plan_cluster_smem_words(p.E, p.R, p.k);
-        int per_sm = 0;
-        static int non_portable[64] = {0};
-        const int dv = pl->device >= 0 && pl->device < 64 ? pl->device : 0;
-        if (non_portable[dv] == 0)
-            non_portable[dv] = cudaFuncSetAttribute(plan_cluster_kernel,
-                                                    cudaFuncAttributeNonPortableClusterSizeAllowed,
-                                                    1) == cudaSuccess ? 1 : -1;
-        if ((p.nt <= 8 || non_portable[dv] > 0) &&
-            smem <= static_cast<size_t>(max_smem_optin(pl->device)) &&
-            kernel_fit(reinterpret_cast<const void *>(plan_cluster_kernel), pl->device,
-                       kPlanThreads, smem, &per_sm) == cudaSuccess &&
-            per_sm > 0) {
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(static_cast<unsigned>(p.nt));
-            cfg.blockDim = dim3(kPlanThreads);
-            cfg.dynamicSmemBytes = smem;
-            cfg.stream = stream;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = static_cast<unsigned>(p.nt);
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            int clusters = 0;
-            if (cluster_fits(p.nt, smem, pl->device, &cfg, &clusters) && clusters > 0) {
-                pl->plan_kernels = 1;
-                return cudaLaunchKernelEx(&cfg, plan_cluster_kernel, p);
-            }
+    if (engine != 2 && engine != 3) {
+        // Groups of up to 16 tiles on thread-block clusters, when they can all be resident.
+        cudaError_t e = cudaSuccess;
+        if (launch_groups(p, pl->device, stream, &e)) {
+            pl->plan_kernels = 1;
+            pl->plan_kind = MOE_PLAN_KIND_GROUPS;
+            return e;
         }
-        (void)cudaGetLastError();
     }
-    if (tuning().plan_engine != 2) {
+    if (engine != 2) {
         // One cooperative launch when the grid fits on the device at once.
         static int coop[64] = {0};
         const int dev = pl->device >= 0 && pl->device < 64 ? pl->device : 0;
@@ -824,15 +1209,16 @@ cudaError_t launch_plan(moe_plan_s *pl, const int32_t *topk_idx, cudaStream_t st
             const int64_t fit = static_cast<int64_t>(sm_count(pl->device)) * per_sm;
             const int64_t want = std::max<int64_t>(p.nt, ceil_div(p.E + p.R, kPlanWarps));
             const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, fit)));
-            void *args[] = {&p};
             pl->plan_kernels = 1;
-            return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(plan_fused_kernel),
-                                               dim3(grid), dim3(kPlanThreads), args, smem, stream);
+            pl->plan_kind = MOE_PLAN_KIND_COOPERATIVE;
+            return launch_kernel(plan_fused_kernel, dim3(grid), dim3(kPlanThreads), smem, stream,
+                                 true, pl->device, p);
         }
         (void)cudaGetLastError();
     }
     pl->plan_kernels = 3;
-    return launch_three(p, stream);
+    pl->plan_kind = MOE_PLAN_KIND_THREE;
+    return launch_three(p, pl->device, stream);
 }
 
 cudaError_t launch_plan_arrays(const PlanArrays &a, cudaStream_t stream)
@@ -859,7 +1245,7 @@ cudaError_t launch_plan_arrays(const PlanArrays &a, cudaStream_t stream)
     p.fanout = a.fanout;
     p.err = a.err;
     p.sync = nullptr;
-    return launch_three(p, stream);
+    return launch_three(p, dev, stream);
 }
 
 }  // namespace moe

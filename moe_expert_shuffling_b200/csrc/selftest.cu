@@ -14,6 +14,8 @@ namespace {
 // which = 1: the mbarrier wait of the copy pipelines, on a barrier that expects two
 //            arrivals and gets one (no copy is in flight).
 // which = 2: the plan's grid barrier, in a grid of two CTAs of which only CTA 0 arrives.
+// which = 3: the group plan's exchange wait, on two arrival words of which nothing sets
+//            the second.
 __global__ void wait_selftest_kernel(uint32_t *words, uint32_t *err, int which)
 {
     __shared__ uint64_t bar;
@@ -22,6 +24,14 @@ __global__ void wait_selftest_kernel(uint32_t *words, uint32_t *err, int which)
     if (which == 2) {
         if (blockIdx.x == 0)
             (void)grid_barrier(words, err, 0u, &s_ok);  // words[0..1]: count, generation
+        return;
+    }
+    if (which == 3) {
+        if (blockIdx.x == 0) {
+            if (threadIdx.x == 0)
+                st_release_gpu(&words[0], 1u);  // the first group arrives, the second never
+            (void)wait_words(words, 2u, 1u, err, &s_ok);
+        }
         return;
     }
     if (blockIdx.x != 0)

@@ -157,3 +157,10 @@ def test_noalloc_rejects_more_tokens_than_its_scratch_holds(lib, N, k, E, R):
     st = lib.moe_plan_noalloc(None, N, k, E, R, *([None] * 11), None)
     assert st == 1
     assert b"scratch" in lib.moe_last_error()
+
+
+def test_plan_create_ex_rejects_unknown_flags(lib):
+    h = ctypes.c_void_p(0)
+    assert lib.moe_plan_create_ex(4, 2, 8, 4, 1, ctypes.c_uint32(2), ctypes.byref(h)) == 1
+    assert b"flags" in lib.moe_last_error()
+    assert not h.value

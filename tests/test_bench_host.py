@@ -93,3 +93,27 @@ def test_measured_peak_falls_back(tmp_path, monkeypatch):
     assert bench.measured_hbm_peak() == (bench.FALLBACK_HBM_GBS, "fallback")
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6000.5}))
     assert bench.measured_hbm_peak() == (6000.5, "measured")
+
+
+def test_step_traffic_lookup(tmp_path, monkeypatch):
+    """The whole-step DRAM figure comes from a step capture of the same shape and variant,
+    against the step's algorithmic bytes; variants that change the traffic get none."""
+    src = tmp_path / "k.cu"
+    src.write_text("int f() { return 1; }\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    shape = {"H": 7168, "k": 8, "payload": "bf16"}
+    rec = {key: {"bytes_per_unit": v, "unit": "token", "shape": shape, "sources": ["k.cu"],
+                 "sources_code_sha256": bench.code_digest(["k.cu"])}
+           for key, v in (("step_dsv3", 260000.0), ("step_dsv3_fused", 258000.0))}
+    (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps(rec))
+    cfg = CONFIGS["dsv3"]
+    alg = bench.dispatch_bytes(cfg) + bench.combine_bytes(cfg) + bench.plan_bytes(cfg)
+    t = bench.step_traffic(cfg, False, alg)
+    assert t["dram_bytes"] == round(260000.0 * cfg.N) and t["algorithmic_bytes"] == alg
+    assert t["ratio"] == round(260000.0 * cfg.N / alg, 4)
+    assert bench.step_traffic(cfg, True, alg)["dram_bytes"] == round(258000.0 * cfg.N)
+    assert bench.step_traffic(cfg, False, alg, dropped=True) is None
+    assert bench.step_traffic(cfg, False, alg, aligned=True) is None
+    assert bench.step_traffic(cfg, False, alg, ranked=True) is None
+    assert bench.step_traffic(CONFIGS["skew"], False, alg) is None   # not captured

@@ -91,6 +91,9 @@ CASES = [
     CONFIGS["tiny"].replace(N=70, H=20000),             # rows of two dispatch chunks
     CONFIGS["long"].replace(N=300, H=512),              # 16-byte scale rows
     CONFIGS["tiny"].replace(k=1, N=777),
+    CONFIGS["mixtral"].replace(N=2000, k=4),            # k <= 4: eight consumer warps
+    CONFIGS["long"].replace(N=1000, H=512, k=4, E=16, R=16),
+    CONFIGS["tiny"].replace(k=3, N=333),
 ]
 
 
@@ -247,3 +250,25 @@ def test_small_calls_run_the_two_kernels_with_the_same_results(identity):
     ms.moe_tune("fused_min_kb", 0)  # the default threshold: this call is below it
     fused_case(CONFIGS["mixtral"].with_tokens(300), 19, identity=identity, ranked=False)
     fused_case(CONFIGS["dsv3"].with_tokens(200), 20, identity=identity, ranked=True)
+
+
+@pytest.mark.parametrize("knobs", [{}, {"combine_max_cw": 4}, {"fused_combine_run": 8},
+                                   {"fused_smem_kb": 64, "fused_ctas_per_sm": 3}],
+                         ids=["default", "4-warps", "8-token-runs", "64KB-3-per-SM"])
+@pytest.mark.parametrize("cfg", [CONFIGS["mixtral"].with_tokens(4000),
+                                 CONFIGS["mixtral"].replace(N=3000, k=4),
+                                 CONFIGS["mixtral"].replace(N=3000, k=3, H=1024)],
+                         ids=lambda c: f"mixtral-N{c.N}-k{c.k}-H{c.H}")
+@pytest.mark.parametrize("identity", [False, True], ids=["y", "recv"])
+def test_fused_small_k_shapes(cfg, knobs, identity):
+    """Mixtral-shaped k = 2, 3, 4: the fused kernel's wide combine shape (and the narrower one
+    it replaced) match the oracle bit for bit, in both orders."""
+    import moe_expert_shuffling_b200 as ms
+    try:
+        for k, v in knobs.items():
+            ms.moe_tune(k, v)
+        fused_case(cfg, 30, identity=identity, ranked=False)
+        fused_case(cfg, 31, identity=identity, ranked=True)
+    finally:
+        for k in knobs:
+            ms.moe_tune(k, 0)

@@ -15,7 +15,7 @@ from tests.shuffle_cases import (
     plan_to_host,
 )
 from tests.test_oracle_plan import drop_some
-from workloads import CONFIGS
+from workloads import CONFIGS, make_routing
 
 pytestmark = pytest.mark.gpu
 
@@ -181,19 +181,26 @@ def test_plan_reuse_and_capacity():
         gpu_plan(idx[:10, :4].copy(), w[:10, :4].copy(), cfg.E, cfg.R, plan=p)
 
 
-def test_invalid_routing_is_flagged_and_contained():
+@pytest.mark.parametrize("cfg", [CONFIGS["tiny"].with_tokens(300),
+                                 CONFIGS["dsv3_k32"].replace(N=300, H=64)],
+                         ids=["tiny", "k32"])
+@pytest.mark.parametrize("match", [1, 2], ids=["shuffles", "match"])
+def test_invalid_routing_is_flagged_and_contained(cfg, match):
     """Out-of-range and repeated ids set error bits, get slot -1 and are skipped: plan,
     dispatch and combine equal, bit for bit, the oracle's on the routing with those entries
-    marked dropped (-1)."""
+    marked dropped (-1).  Both ways of comparing a token's ids give the same."""
     import moe_expert_shuffling_b200 as ms
-    cfg = CONFIGS["tiny"].with_tokens(300)
     idx, w, x, _, y = make_inputs(cfg, 0)
     bad = idx.copy()
     bad[3, 0] = cfg.E            # out of range
     bad[10, 1] = -5              # negative
     bad[20, 1] = bad[20, 0]      # repeated in one token (the first occurrence stays valid)
     bad[299, 0] = 2 ** 31 - 1
-    p, ti, tw = gpu_plan(bad, w, cfg.E, cfg.R)
+    ms.moe_tune("plan_match", match)
+    try:
+        p, ti, tw = gpu_plan(bad, w, cfg.E, cfg.R)
+    finally:
+        ms.moe_tune("plan_match", 0)
     recv = torch.zeros((cfg.N * cfg.k, cfg.H), dtype=torch.bfloat16, device="cuda")
     ms.moe_dispatch(x, p, recv=recv)
     out = ms.moe_combine(y, p)
@@ -319,51 +326,106 @@ def test_drops_alone_raise_no_error():
     assert np.all(a["slot"] == -1) and np.all(a["src_tok"] == -1) and a["cnt"].sum() == 0
 
 
-@pytest.mark.parametrize("cfg,frac,align", [
-    (CONFIGS["dsv3"].with_tokens(128), 0.0, 1),
-    (CONFIGS["dsv3"].with_tokens(16), 0.25, 64),
-    (CONFIGS["dsv3"].replace(N=100, H=64, E=1024, k=8, R=1024), 0.0, 1),
-    (CONFIGS["dsv3"].replace(N=50, H=64, E=64, k=32, R=8), 0.1, 8),
-    (CONFIGS["mixtral"].with_tokens(1), 0.0, 1),
+@pytest.mark.parametrize("cfg,frac,align,kind", [
+    (CONFIGS["dsv3"].with_tokens(128), 0.0, 1, "one_tile"),
+    (CONFIGS["dsv3"].with_tokens(16), 0.25, 64, "one_tile"),
+    (CONFIGS["dsv3"].replace(N=100, H=64, E=1024, k=8, R=1024), 0.0, 1, "one_tile"),
+    (CONFIGS["dsv3"].replace(N=50, H=64, E=64, k=32, R=8), 0.1, 8, "one_tile"),
+    (CONFIGS["mixtral"].with_tokens(1), 0.0, 1, "one_tile"),
     # 2..16 tiles: one thread-block cluster, tile counts through distributed shared memory
-    (CONFIGS["dsv3"].with_tokens(2048), 0.1, 8),
-    (CONFIGS["dsv3"].with_tokens(1100), 0.0, 1),
-    (CONFIGS["dsv3"].with_tokens(129), 0.0, 1),
-    (CONFIGS["dsv3"].with_tokens(1024), 0.0, 1),
-    (CONFIGS["dsv3"].with_tokens(700), 0.2, 16),
-    (CONFIGS["dsv3"].replace(N=1000, H=64, E=1024, k=8, R=1024), 0.05, 1),
-    (CONFIGS["dsv3"].replace(N=256, H=64, E=64, k=32, R=8), 0.1, 4),
-    (CONFIGS["mixtral"].with_tokens(1024), 0.0, 1),
-    (CONFIGS["tiny"].replace(k=1, N=1000), 0.0, 1),
+    (CONFIGS["dsv3"].with_tokens(2048), 0.1, 8, "groups"),
+    (CONFIGS["dsv3"].with_tokens(1100), 0.0, 1, "groups"),
+    (CONFIGS["dsv3"].with_tokens(129), 0.0, 1, "groups"),
+    (CONFIGS["dsv3"].with_tokens(1024), 0.0, 1, "groups"),
+    (CONFIGS["dsv3"].with_tokens(700), 0.2, 16, "groups"),
+    (CONFIGS["dsv3"].replace(N=1000, H=64, E=1024, k=8, R=1024), 0.05, 1, "groups"),
+    (CONFIGS["dsv3"].replace(N=256, H=64, E=64, k=32, R=8), 0.1, 4, "groups"),
+    (CONFIGS["mixtral"].with_tokens(1024), 0.0, 1, "groups"),
+    (CONFIGS["tiny"].replace(k=1, N=1000), 0.0, 1, "groups"),
+    # several clusters and one exchange of their totals
+    (CONFIGS["dsv3"].with_tokens(2049), 0.0, 1, "groups"),
+    (CONFIGS["dsv3"].with_tokens(4096), 0.1, 8, "groups"),
+    (CONFIGS["dsv3"].with_tokens(16384).replace(H=256), 0.0, 1, "groups"),
+    (CONFIGS["skew"].with_tokens(16384).replace(H=256), 0.05, 128, "groups"),
+    (CONFIGS["mixtral"].replace(H=256), 0.0, 1, "groups"),
+    (CONFIGS["long"].replace(H=128), 0.0, 1, "groups"),
+    (CONFIGS["dsv3"].replace(N=5000, H=64, E=1024, k=8, R=1024), 0.05, 1, "groups"),
+    (CONFIGS["dsv3"].replace(N=3333, H=64, E=64, k=32, R=8), 0.1, 4, "groups"),
 ], ids=lambda v: f"{v.name}-N{v.N}-E{v.E}-k{v.k}" if hasattr(v, "name") else str(v))
-def test_single_tile_plans(cfg, frac, align):
-    """Routings of at most one tile (N <= 128) take the one-CTA plan kernel, and those of
-    2..16 tiles the one-cluster kernel; their plan, dispatch and combine match the oracle bit
-    for bit."""
+def test_plan_kernels(cfg, frac, align, kind):
+    """Routings of at most one tile (N <= 128) take the one-CTA plan kernel and larger ones
+    the group kernel (clusters of up to 16 tiles, one exchange between clusters); their plan,
+    dispatch and combine match the oracle bit for bit."""
     import moe_expert_shuffling_b200 as ms
-    idx, w, x, _, _ = make_inputs(cfg, 17, y=False)
+    idx, w, x, xs, _ = make_inputs(cfg, 17, y=False)
     if frac > 0:
         idx = drop_some(idx, frac, 3)
     ref = oracle.plan(idx, cfg.E, cfg.R, align=align)
     p = ms.moe_plan_create(cfg.N, cfg.k, cfg.E, cfg.R, align=align)
     p, ti, tw = gpu_plan(idx, w, cfg.E, cfg.R, plan=p)
     assert p.plan_kernels == 1
+    assert p.plan_kind == kind
     got = plan_to_host(p)
     for name in ("cnt", "expert_off", "rcnt", "rank_off", "rtok_off", "slot", "src_tok",
                  "src_j", "rtok"):
         assert np.array_equal(got[name], getattr(ref, name)), name
     assert np.array_equal(got["fanout"], ref.fanout)
     assert int(got["err"][0]) == 0
+    used = ref.src_tok >= 0
+    if cfg.payload == "fp8":
+        recv, rs = ms.moe_dispatch(x, p, x_scale=xs)
+        want_recv, _ = oracle.dispatch(x.cpu().numpy(), ref.slot, xs.cpu().numpy(), rows=ref.rows)
+        got_recv = recv.cpu().numpy()
+        assert p.check() == 0
+        assert np.array_equal(got_recv[used], want_recv[used])
+        return
     recv = ms.moe_dispatch(x, p)
     out = ms.moe_combine(recv, p)
     assert p.check() == 0
-    used = ref.src_tok >= 0
     want_recv = oracle.dispatch(bits16(x).view(np.uint8).reshape(cfg.N, -1), ref.slot, rows=ref.rows)
     got_recv = bits16(recv).view(np.uint8).reshape(ref.rows, -1)
     assert np.array_equal(got_recv[used], want_recv[used])
     y_bits = want_recv.view(np.uint16).reshape(ref.rows, cfg.H).copy()
     y_bits[~used] = 0
     assert np.array_equal(bits16(out), oracle.combine(y_bits, ref.slot, w))
+
+
+@pytest.mark.parametrize("knobs,kind", [
+    ({"plan_cluster": 1}, "groups"), ({"plan_cluster": 2}, "groups"),
+    ({"plan_cluster": 3}, "groups"), ({"plan_cluster": 8}, "groups"),
+    ({"plan_cluster": 16}, "groups"), ({"plan_engine": 3}, "cooperative"),
+    ({"plan_engine": 2}, "three"), ({"plan_match": 1}, "groups"), ({"plan_match": 2}, "groups"),
+    ({"plan_match": 2, "plan_engine": 3}, "cooperative"),
+], ids=lambda v: str(v))
+@pytest.mark.parametrize("name,N,frac,align", [("dsv3", 3000, 0.1, 1), ("dsv3", 16384, 0.0, 8),
+                                               ("mixtral", 8192, 0.0, 1), ("long", 9000, 0.2, 4),
+                                               ("dsv3_k32", 2500, 0.1, 1), ("dsv3_k16", 1100, 0.0, 2)])
+def test_plan_engines_agree_with_the_oracle(knobs, kind, name, N, frac, align):
+    """Every planner kernel and cluster size gives the oracle's plan bit for bit, including
+    repeated calls on one plan (the exchange words are reused) and drops and alignment."""
+    import moe_expert_shuffling_b200 as ms
+    cfg = CONFIGS[name].with_tokens(N)
+    p = ms.moe_plan_create(N, cfg.k, cfg.E, cfg.R, align=align)
+    try:
+        for k, v in knobs.items():
+            ms.moe_tune(k, v)
+        for seed in (5, 6):
+            idx, w = make_routing(cfg, seed)
+            if frac > 0:
+                idx = drop_some(idx, frac, seed)
+            p, ti, tw = gpu_plan(idx, w, cfg.E, cfg.R, plan=p)
+            assert p.plan_kind == kind
+            got = plan_to_host(p)
+            ref = oracle.plan(idx, cfg.E, cfg.R, align=align)
+            for f in ("cnt", "expert_off", "rcnt", "rank_off", "rtok_off", "slot", "src_tok",
+                      "src_j", "rtok"):
+                assert np.array_equal(got[f], getattr(ref, f)), f
+            assert np.array_equal(got["fanout"], ref.fanout)
+            assert p.check() == 0
+    finally:
+        for k in knobs:
+            ms.moe_tune(k, 0)
+        p.close()
 
 
 @pytest.mark.parametrize("knobs", [{"combine_max_cw": 4}, {"combine_max_cw": 8},
@@ -392,3 +454,54 @@ def test_small_k_combine_shapes(cfg, knobs):
     yb = bits16(y)
     assert np.array_equal(bits16(out), oracle.combine(yb, ref.slot, w))
     assert np.array_equal(bits16(out_r), oracle.combine_ranked(yb, ref.slot, w, idx, cfg.E, cfg.R))
+
+
+def test_one_plan_reused_across_sizes():
+    """One plan object planned again and again with different token counts, so that the
+    planner kernel, the number of cluster groups and the exchange generation change from
+    call to call (stale arrival words of a larger earlier call stay in memory); every call
+    matches the oracle bit for bit."""
+    import moe_expert_shuffling_b200 as ms
+    cfg = CONFIGS["dsv3"].replace(H=64)
+    p = ms.moe_plan_create(16384, cfg.k, cfg.E, cfg.R)
+    try:
+        for i, N in enumerate((16384, 3000, 129, 16384, 2049, 100, 8192, 16384, 4097)):
+            c = cfg.with_tokens(N)
+            idx, w = make_routing(c, 40 + i)
+            if i % 3 == 1:
+                idx = drop_some(idx, 0.1, i)
+            p, ti, tw = gpu_plan(idx, w, c.E, c.R, plan=p)
+            got = plan_to_host(p)
+            ref = oracle.plan(idx, c.E, c.R)
+            for f in ("cnt", "expert_off", "rcnt", "rank_off", "rtok_off", "slot", "src_tok",
+                      "src_j", "rtok"):
+                assert np.array_equal(got[f], getattr(ref, f)), (N, f)
+            assert np.array_equal(got["fanout"], ref.fanout)
+            assert p.check() == 0
+    finally:
+        p.close()
+
+
+@pytest.mark.parametrize("name,N", [("dsv3", 16384), ("dsv3", 3000), ("dsv3", 100),
+                                    ("dsv3_k32", 2000), ("mixtral", 4000)])
+@pytest.mark.parametrize("engine", [0, 3, 2], ids=["auto", "cooperative", "three"])
+def test_plan_without_dedup_lists(name, N, engine):
+    """A plan created without the per-rank lists writes everything else bit for bit as the
+    oracle does (rcnt and rtok_off included) and leaves the list arrays untouched."""
+    import moe_expert_shuffling_b200 as ms
+    cfg = CONFIGS[name].with_tokens(N)
+    idx, w = make_routing(cfg, 77)
+    p = ms.moe_plan_create(N, cfg.k, cfg.E, cfg.R, dedup_lists=False)
+    assert not p.dedup_lists
+    ms.moe_tune("plan_engine", engine)
+    try:
+        p, ti, tw = gpu_plan(idx, w, cfg.E, cfg.R, plan=p)   # the lists stay as created: 0
+        got = plan_to_host(p)
+    finally:
+        ms.moe_tune("plan_engine", 0)
+    ref = oracle.plan(idx, cfg.E, cfg.R)
+    for f in ("cnt", "expert_off", "rcnt", "rank_off", "rtok_off", "slot", "src_tok", "src_j"):
+        assert np.array_equal(got[f], getattr(ref, f)), f
+    assert not got["rtok"].any() and not got["fanout"].any()
+    assert p.check() == 0
+    p.close()

@@ -16,7 +16,8 @@ from workloads import CONFIGS
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("which", [0, 1, 2], ids=["ready_flag", "mbarrier", "grid_barrier"])
+@pytest.mark.parametrize("which", [0, 1, 2, 3],
+                         ids=["ready_flag", "mbarrier", "grid_barrier", "group_exchange"])
 def test_wait_gives_up_and_reports_timeout(which):
     import moe_expert_shuffling_b200 as ms
     torch.cuda.synchronize()
@@ -26,18 +27,20 @@ def test_wait_gives_up_and_reports_timeout(which):
     assert flags == ms.ERR_TIMEOUT
     assert 0.5 < elapsed < 30.0
 
-    # the context still works: a small step matches the oracle
-    cfg = CONFIGS["tiny"]
-    idx, w, x, _, y = make_inputs(cfg, 2)
-    p, ti, tw = gpu_plan(idx, w, cfg.E, cfg.R)
-    recv = ms.moe_dispatch(x, p)
-    out = ms.moe_combine(y, p)
-    torch.cuda.synchronize()
-    assert p.check() == 0
-    ref = oracle.plan(idx, cfg.E, cfg.R)
-    assert np.array_equal(bits16(out), oracle.combine(bits16(y), ref.slot, w))
-    assert np.array_equal(bits16(recv).view(np.uint8).reshape(cfg.N * cfg.k, -1),
-                          oracle.dispatch(bits16(x).view(np.uint8).reshape(cfg.N, -1), ref.slot))
+    # the context still works: small steps (one tile, and several groups of tiles) match the
+    # oracle
+    for cfg in (CONFIGS["tiny"], CONFIGS["dsv3"].with_tokens(3000).replace(H=256)):
+        idx, w, x, _, y = make_inputs(cfg, 2)
+        p, ti, tw = gpu_plan(idx, w, cfg.E, cfg.R)
+        recv = ms.moe_dispatch(x, p)
+        out = ms.moe_combine(y, p)
+        torch.cuda.synchronize()
+        assert p.check() == 0
+        ref = oracle.plan(idx, cfg.E, cfg.R)
+        assert np.array_equal(bits16(out), oracle.combine(bits16(y), ref.slot, w))
+        assert np.array_equal(bits16(recv).view(np.uint8).reshape(cfg.N * cfg.k, -1),
+                              oracle.dispatch(bits16(x).view(np.uint8).reshape(cfg.N, -1),
+                                              ref.slot))
 
 
 def test_selftest_rejects_unknown_wait():
