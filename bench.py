@@ -721,14 +721,19 @@ def run_latency(args):
     dev = torch.device("cuda", 0)
     s = torch.cuda.Stream(device=dev)
 
-    def replay_us(fn, iters):
+    def replay_us(fn, iters, reps=1):
+        """µs per call: a graph holding `reps` calls back to back, replayed `iters` times.
+        With reps = 1 every call is its own graph launch, so small calls measure how fast
+        graphs are launched; with reps = 20 the calls follow one another on the device, as
+        in a decode step captured with the rest of a model."""
         with torch.cuda.stream(s):
             for _ in range(args.warmup):
                 fn()
         s.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=s):
-            fn()
+            for _ in range(reps):
+                fn()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(s):
             g.replay()
@@ -737,7 +742,8 @@ def run_latency(args):
                 g.replay()
             b.record(s)
         b.synchronize()
-        return round(1e3 * a.elapsed_time(b) / iters, 2)
+        del g
+        return round(1e3 * a.elapsed_time(b) / (iters * reps), 2)
 
     for N in (int(v) for v in args.latency.split(",")):
         cfg = CONFIGS[args.config].with_tokens(N)
@@ -768,10 +774,15 @@ def run_latency(args):
         def dc():
             ms.moe_dispatch_combine(x, plan, recv, y, plan, out=out, stream=s, **kw)
 
+        it = max(1, args.steps // 20)
         res = {"workload": workload_name(cfg), "tokens": N, "unit": "us",
-               "plan": replay_us(pl, args.steps), "dispatch": replay_us(dp, args.steps),
-               "combine": replay_us(cb, args.steps), "dispatch_combine": replay_us(dc, args.steps),
-               "step": replay_us(lambda: (pl(), dp(), cb()), args.steps),
+               "note": "per call, graphs of 20 calls back to back; single_launch: one call per "
+                       "graph launch",
+               "plan": replay_us(pl, it, 20), "dispatch": replay_us(dp, it, 20),
+               "combine": replay_us(cb, it, 20), "dispatch_combine": replay_us(dc, it, 20),
+               "step": replay_us(lambda: (pl(), dp(), cb()), it, 20),
+               "single_launch": {"plan": replay_us(pl, args.steps),
+                                 "step": replay_us(lambda: (pl(), dp(), cb()), args.steps)},
                "plan_kernels": plan.plan_kernels, "plan_kind": plan.plan_kind}
         if plan.check(s) != 0:
             raise SystemExit("device reported invalid routing or a timeout")

@@ -242,7 +242,7 @@ extern "C" {
 
 const char *moe_last_error(void) { return g_last_error.c_str(); }
 
-const char *moe_version(void) { return "moeshuffle 0.1.0 (sm_100a)"; }
+const char *moe_version(void) { return "moeshuffle 0.2.0 (sm_100a)"; }
 
 moe_status moe_tune(moe_knob knob, int32_t value)
 {
@@ -343,7 +343,7 @@ moe_status moe_plan_create_ex(int32_t max_tokens, int32_t k, int32_t E, int32_t 
         {reinterpret_cast<void **>(&p->tile_cnt), sizeof(int32_t) * E * nt},
         {reinterpret_cast<void **>(&p->tile_rcnt), sizeof(int32_t) * R * nt},
         {reinterpret_cast<void **>(&p->tile_err), sizeof(uint32_t) * nt},
-        {reinterpret_cast<void **>(&p->group_flag), sizeof(uint32_t) * nt},
+        {reinterpret_cast<void **>(&p->group_flag), sizeof(uint32_t) * (nt + 16)},
         {reinterpret_cast<void **>(&p->work), 4 * sizeof(uint32_t)},
         {reinterpret_cast<void **>(&p->ready), sizeof(uint32_t) * (max_tokens > 0 ? max_tokens : 1)},
     };
@@ -637,7 +637,7 @@ moe_status moe_plan_check(moe_plan_t plan, void *stream, uint32_t *flags)
             e = cudaMemset(plan->err, 0, sizeof(uint32_t));
         if (e == cudaSuccess)
             e = cudaMemset(plan->group_flag, 0,
-                           sizeof(uint32_t) * (plan->nt_cap > 0 ? plan->nt_cap : 1));
+                           sizeof(uint32_t) * ((plan->nt_cap > 0 ? plan->nt_cap : 1) + 16));
         if (e != cudaSuccess)
             return cuda_fail(e, "cudaMemset(sync)");
         // and the fused kernel's work words, with its flags (the epoch starts again)

@@ -262,9 +262,10 @@ __device__ __forceinline__ bool wait_words(const uint32_t *words, uint32_t n, ui
         bool ok = true;
         const uint64_t t0 = global_timer_ns();
         for (uint32_t it = 0;; ++it) {
+            // relaxed loads, all in flight at once; the fence below makes the wait an acquire
             bool mine = true;
             for (uint32_t q = lane; q < n; q += 32)
-                mine = mine && ld_acquire_gpu(words + q) == want;
+                mine &= ld_relaxed_gpu(words + q) == want;
             if (__all_sync(0xffffffffu, mine))
                 break;
             if ((it & 15u) == 15u) {
@@ -277,6 +278,7 @@ __device__ __forceinline__ bool wait_words(const uint32_t *words, uint32_t n, ui
                 }
             }
         }
+        __threadfence();  // what each arrival released is visible to this CTA from here on
         if (lane == 0)
             *s_ok = ok;
     }

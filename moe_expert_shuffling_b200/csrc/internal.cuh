@@ -29,7 +29,7 @@ struct moe_plan_s {
     // (the group kernel keeps its groups' totals and flags in the first rows of these)
     int32_t *tile_cnt = nullptr, *tile_rcnt = nullptr;
     uint32_t *tile_err = nullptr;
-    uint32_t *group_flag = nullptr;  // [nt] per-group arrival words of the group plan kernel
+    uint32_t *group_flag = nullptr;  // [nt + 16] arrival words of the group plan kernel's CTAs
     const float *topk_w = nullptr;
     int32_t plan_kernels = 0;  // kernels the last launch_plan enqueued
     int32_t plan_kind = 0;     // MOE_PLAN_KIND_* of the last launch_plan

@@ -167,21 +167,34 @@ __device__ int32_t block_exclusive_scan(int32_t v, int32_t *total, int32_t *warp
     return before + x - v;
 }
 
-// dst[0..n] = exclusive scan of src[0..n) followed by the total.  All threads must call.
-__device__ void scan_into(const int32_t *src, int n, int32_t *dst, int32_t *warp_sums)
+// dst[0..n] = exclusive scan of src[0..n) followed by the total, by one warp (n <= 1024):
+// each lane sums a run of consecutive values, a warp scan offsets the runs.  No block
+// barrier is taken, so two warps can scan two arrays at once.
+__device__ void warp_scan_into(const int32_t *src, int n, int32_t *dst)
 {
-    int32_t carry = 0;
-    for (int base = 0; base < n; base += blockDim.x) {
-        const int i = base + threadIdx.x;
-        const int32_t v = i < n ? src[i] : 0;
-        int32_t tot;
-        const int32_t ex = block_exclusive_scan(v, &tot, warp_sums);
-        if (i < n)
-            dst[i] = carry + ex;
-        carry += tot;
+    const int lane = threadIdx.x & 31;
+    const int per = (n + 31) / 32;
+    const int b = lane * per;
+    int32_t sum = 0;
+    for (int i = 0; i < per; ++i)
+        if (b + i < n)
+            sum += src[b + i];
+    int32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o)
+            incl += y;
     }
-    if (threadIdx.x == 0)
-        dst[n] = carry;
+    int32_t run = incl - sum;
+    for (int i = 0; i < per; ++i)
+        if (b + i < n) {
+            const int32_t v = src[b + i];
+            dst[b + i] = run;
+            run += v;
+        }
+    if (lane == 31)
+        dst[n] = incl;
 }
 
 // Shared-memory layout of every plan kernel (words).  The ids come first so that they are
@@ -361,6 +374,30 @@ __device__ __forceinline__ uint32_t classify_steps(const PlanK &p, const PlanSme
     return flags;
 }
 
+// classify_loaded for the lane-segment widths up to WMAX only (kernels instantiated per range
+// of k carry only the widths they need).
+template <int WMAX>
+__device__ uint32_t classify_loaded_w(const PlanK &p, const PlanSmem &m, int ntok)
+{
+    __syncthreads();
+    uint32_t flags;
+    const int w = 1 << lane_map(p.k).wbits;  // block-uniform
+    if (WMAX > 16 && w > 16)
+        flags = classify_steps<32>(p, m, ntok);
+    else if (w > 8)
+        flags = classify_steps<16>(p, m, ntok);
+    else if (w > 4)
+        flags = classify_steps<8>(p, m, ntok);
+    else if (w > 2)
+        flags = classify_steps<4>(p, m, ntok);
+    else if (w > 1)
+        flags = classify_steps<2>(p, m, ntok);
+    else
+        flags = classify_steps<1>(p, m, ntok);
+    __syncthreads();
+    return flags;
+}
+
 // classify_tile once the masks are clear and the ids are being stored (synchronises first).
 __device__ uint32_t classify_loaded(const PlanK &p, const PlanSmem &m, int ntok)
 {
@@ -409,10 +446,10 @@ __device__ void count_tile(const PlanK &p, const PlanSmem &m, int tile, uint32_t
 // (shared memory when `raw_shared`, else the global cnt array).  Block 0 writes the offset
 // arrays; every receive row that no entry maps to (segment padding and rows after the last
 // segment) is marked -1 in src_tok/src_j, spread over all CTAs of the grid.
-__device__ void prepare_offsets(const PlanK &p, const PlanSmem &m, int32_t *warp_sums,
-                                const int32_t *raw_cnt, bool raw_shared);
+__device__ void prepare_offsets(const PlanK &p, const PlanSmem &m, const int32_t *raw_cnt,
+                                bool raw_shared);
 
-__device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_sums)
+__device__ void rank_prepare(const PlanK &p, const PlanSmem &m)
 {
     for (int i = threadIdx.x; i < p.E + p.R; i += blockDim.x) {
         if (i < p.E) {
@@ -422,15 +459,17 @@ __device__ void rank_prepare(const PlanK &p, const PlanSmem &m, int32_t *warp_su
             m.rbase[i - p.E] = __ldcg(p.rcnt + (i - p.E));
         }
     }
-    prepare_offsets(p, m, warp_sums, p.cnt, false);
+    prepare_offsets(p, m, p.cnt, false);
 }
 
-__device__ void prepare_offsets(const PlanK &p, const PlanSmem &m, int32_t *warp_sums,
-                                const int32_t *raw_cnt, bool raw_shared)
+__device__ void prepare_offsets(const PlanK &p, const PlanSmem &m, const int32_t *raw_cnt,
+                                bool raw_shared)
 {
     __syncthreads();
-    scan_into(m.ebase, p.E, m.eoff, warp_sums);
-    scan_into(m.rbase, p.R, m.roff, warp_sums);
+    if (threadIdx.x < 32)
+        warp_scan_into(m.ebase, p.E, m.eoff);
+    else if (threadIdx.x < 64)
+        warp_scan_into(m.rbase, p.R, m.roff);
     __syncthreads();
     if (blockIdx.x == 0) {
         for (int i = threadIdx.x; i <= p.E; i += blockDim.x)
@@ -580,11 +619,10 @@ __global__ void __launch_bounds__(kScanThreads) plan_scan_kernel(const PlanK p)
 __global__ void __launch_bounds__(kPlanThreads) plan_rank_kernel(const PlanK p)
 {
     extern __shared__ __align__(16) int32_t smem[];
-    __shared__ int32_t warp_sums[kPlanThreads / 32];
     const PlanSmem m = carve(smem, p.E, p.R, p.k);
     init_rank_of(p, m);
     pdl_wait();
-    rank_prepare(p, m, warp_sums);
+    rank_prepare(p, m);
     pdl_trigger();
     rank_tile(p, m, blockIdx.x, false);
 }
@@ -596,7 +634,6 @@ __global__ void __launch_bounds__(kPlanThreads) plan_one_tile_kernel(const PlanK
 {
     extern __shared__ __align__(16) int32_t smem[];
     __shared__ uint32_t s_err;
-    __shared__ int32_t warp_sums[kPlanThreads / 32];
     const PlanSmem m = carve(smem, p.E, p.R, p.k);
     if (threadIdx.x == 0)
         s_err = 0;
@@ -622,7 +659,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_one_tile_kernel(const PlanK
     __syncthreads();
     if (threadIdx.x == 0)
         *p.err = s_err;  // before any MOE_ERR_BOUNDS of the rank step is or-ed in
-    prepare_offsets(p, m, warp_sums, p.cnt, false);
+    prepare_offsets(p, m, p.cnt, false);
     // the tile's bases are the segment starts themselves
     for (int e = threadIdx.x; e < p.E; e += blockDim.x)
         m.ebase[e] = m.eoff[e];
@@ -634,32 +671,33 @@ __global__ void __launch_bounds__(kPlanThreads) plan_one_tile_kernel(const PlanK
 }
 
 // ------------------------------------------- groups of tiles on thread-block clusters
-// One CTA per tile; the tiles are grouped C at a time (C <= 16) into thread-block clusters.
-// Inside a group the tile counts are combined through distributed shared memory: each CTA
-// scans the rows it owns (row % C == its rank) across the group's C tiles with warp
-// shuffles and writes every tile's prefix (its base within the group) back into that
-// tile's CTA.  With one group the totals are final and are written back the same way.
-// With several, each group stores its totals in global memory and its leader CTA releases
-// the group's arrival word; every CTA then reads all groups' totals and adds up those of
-// the earlier groups (its group's base) and of all groups (the segment sizes) by itself.
-// That one exchange replaces the two grid barriers and the scan phase of the cooperative
-// kernel.  Every CTA takes the same cluster barriers whatever its data; the exchange's
-// wait gives up after the wait limit.  The launch is cooperative with several groups
-// (they wait on each other), and the host checks that all of its clusters can be resident.
-//
-// Work that depends only on the CTA's own tile runs before the exchange: the tile-local
-// offsets of every expert and rank (scans of the tile counts), and a staging order of the
-// tile's entries by (expert, token) and of its leaders by (rank, token) in shared memory.
-// After the exchange the receive-row inverse maps and the dedup lists are then stored in
-// runs of consecutive addresses, one run per (tile, expert) and per (tile, rank), rather
-// than one scattered word per entry.
+// One CTA per tile; the CTAs are grouped C at a time (C <= 16) into thread-block clusters.
+//  1. Each CTA counts its tile, stores the counts column-wise (row * tiles + tile) and
+//     releases its arrival word.  (A grid of one cluster skips the global exchange: after a
+//     cluster barrier its CTAs read the counts straight from each other's shared memory.)
+//  2. While the other tiles arrive, it prepares everything that depends only on its own
+//     tile: the tile-local offset of every expert and rank (scans of the tile counts) and a
+//     staging order of the tile's entries by (expert, token) and of its leaders by (rank,
+//     token) in shared memory.
+//  3. Once every CTA has arrived, each CTA of a cluster scans its share of the rows (1/C of
+//     them) across all tiles with coalesced loads, and writes through distributed shared
+//     memory, into each CTA of its cluster, that tile's prefix of the row (its base) and
+//     the row's total.
+//  4. After one cluster barrier every CTA has its bases and the totals: segment offsets,
+//     then the stores -- slot in entry order, the inverse maps and the dedup lists in runs of
+//     consecutive addresses (one run per (tile, expert) and per (tile, rank)).
+// One grid-wide exchange and one cluster barrier replace the cooperative kernel's two grid
+// barriers and its scan phase.  The launch is cooperative (every CTA waits for all others),
+// and the host checks that all of its clusters can be resident at once.  The exchange's wait
+// gives up after the wait limit; a CTA that gave up still takes every cluster barrier, so no
+// barrier of its cluster can hang.
 constexpr int kMaxClusterTiles = 16;
 
 // Shared memory of the group kernel after the common layout (words).
 struct GroupSmem {
-    int32_t *tc;     // [E+R] this tile's counts (read by the group's other CTAs)
-    int32_t *tb;     // [E+R] this tile's base: earlier tiles of its group, then of all
-    int32_t *tot;    // [E+R] the routing's counts
+    int32_t *tc;     // [E+R] this tile's counts, then the expert counts of the routing
+    int32_t *tb;     // [E+R] this tile's base (earlier tiles), written by the row's owner CTA
+    int32_t *tot;    // [E+R] the routing's counts, written by the row's owner CTA
     int32_t *loff;   // [E+1] tile-local first entry of each expert in the staging order
     int32_t *lroff;  // [R+1] tile-local first leader of each rank in the staging order
     int32_t *qloc;   // [kPlanTile * k] each entry's rank among the tile's entries of its expert
@@ -686,12 +724,24 @@ __device__ __forceinline__ GroupSmem carve_group(const PlanSmem &m, int E, int R
     return q;
 }
 
-__global__ void __launch_bounds__(kPlanThreads) plan_group_kernel(const PlanK p)
+// Split cluster barrier: every thread of every CTA arrives, and later waits for the phase.
+__device__ __forceinline__ void cluster_arrive_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait()
+{
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// kWide: rows of more than 16 ids (k > 16); the other instantiation takes k <= 16.
+template <bool kWide>
+__global__ void __launch_bounds__(kPlanThreads, 4) plan_group_kernel(const PlanK p)
 {
     namespace cg = cooperative_groups;
     extern __shared__ __align__(16) int32_t smem[];
     __shared__ uint32_t s_err;
-    __shared__ int32_t warp_sums[kPlanThreads / 32];
     __shared__ int s_ok;
     __shared__ uint32_t s_gen;  // the exchange generation, read once and shared by the CTA
     cg::cluster_group cluster = cg::this_cluster();
@@ -702,12 +752,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_group_kernel(const PlanK p)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int C = static_cast<int>(cluster.num_blocks());
     const int c = static_cast<int>(cluster.block_rank());
-    const uint32_t G = gridDim.x / static_cast<uint32_t>(C);  // groups (clusters are 1-D)
-    const int g = static_cast<int>(blockIdx.x) / C;
+    const int t_first = static_cast<int>(blockIdx.x) - c;  // the cluster's first tile
     const int tile = static_cast<int>(blockIdx.x);
-    const int ntok = tile_tokens(p, tile);
-    const bool multi = G > 1;
+    const int ntok = tile_tokens(p, tile);  // 0 for the CTAs past the last tile
 
+    // Arrive at once on the cluster barrier that is waited on before the first access to
+    // another CTA's shared memory (every CTA of the cluster has started by then).
+    cluster_arrive_relaxed();
     // Shared-memory set-up overlaps the previous kernel on the stream; global memory is
     // touched only after pdl_wait.
     init_rank_of(p, m);
@@ -717,24 +768,45 @@ __global__ void __launch_bounds__(kPlanThreads) plan_group_kernel(const PlanK p)
     pdl_wait();
     load_ids(p, m, tile, ntok);
     if (threadIdx.x == 0) {
-        s_gen = multi ? __ldcg(&p.sync[1]) : 0u;
+        s_gen = __ldcg(&p.sync[1]);
         // Clear the error word before any CTA can or bits into it (all of that happens after
-        // the cluster barrier below, and after the exchange with several groups).  A timeout
-        // of an earlier call stays until moe_plan_check rearms the plan.
+        // the exchange).  A timeout of an earlier call stays until moe_plan_check rearms the
+        // plan.
         if (blockIdx.x == 0)
             atomicAnd(p.err, MOE_ERR_TIMEOUT);
     }
-    const uint32_t flags = classify_loaded(p, m, ntok);  // synchronises first and last
+    const uint32_t flags = classify_loaded_w<kWide ? 32 : 16>(p, m, ntok);  // syncs first and last
     if (flags)
         atomicOr(&s_err, flags);
+    const bool one_cluster = static_cast<int>(gridDim.x) == C;
     for (int row = threadIdx.x; row < ER; row += blockDim.x) {
         const uint32_t *mk = row < p.E ? &m.emask[4 * row] : &m.rmask[4 * (row - p.E)];
-        q.tc[row] = __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+        const int32_t v = __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
+        q.tc[row] = v;
+        if (!one_cluster && tile < p.nt) {
+            if (row < p.E)
+                p.tile_cnt[static_cast<int64_t>(row) * p.nt + tile] = v;
+            else
+                p.tile_rcnt[static_cast<int64_t>(row - p.E) * p.nt + tile] = v;
+        }
     }
-    __syncthreads();
-    // Tile-local offsets and the staging orders (this tile's data only).
-    scan_into(q.tc, p.E, q.loff, warp_sums);
-    scan_into(q.tc + p.E, p.R, q.lroff, warp_sums);
+    uint32_t want = s_gen + 1u;  // s_gen was set before classify_loaded's barriers
+    if (want == 0u)
+        want = 1u;  // arrival words start at 0: the generation never takes that value
+    __syncthreads();  // the tile's counts are stored and s_err is final
+    if (threadIdx.x == 0 && !one_cluster) {
+        if (tile < p.nt)
+            p.tile_err[tile] = s_err;
+        __threadfence();  // the CTA's stores (ordered before by the barrier) first
+        st_release_gpu(&p.group_flag[tile], want);  // every CTA arrives, the last ones too
+    }
+
+    // Tile-local offsets and the staging orders (this tile's data only), while the other
+    // tiles arrive.
+    if (threadIdx.x < 32)
+        warp_scan_into(q.tc, p.E, q.loff);
+    else if (threadIdx.x < 64)
+        warp_scan_into(q.tc + p.E, p.R, q.lroff);
     __syncthreads();
     {
         const LaneMap lm = lane_map(k);
@@ -759,11 +831,17 @@ __global__ void __launch_bounds__(kPlanThreads) plan_group_kernel(const PlanK p)
             }
         }
     }
-    cluster.sync();  // (A) every tile's counts and flags are visible to its group
 
-    // The rows this CTA owns (row % C == c): lane qq of a segment of `width` lanes reads the
-    // count of the group's tile qq; a segmented inclusive scan gives each tile's base.
-    {
+    // The exchange: every CTA's arrival word holds this launch's generation.  A grid of one
+    // cluster needs none: its counts are read from the other CTAs' shared memory.
+    const bool ok = one_cluster || wait_words(p.group_flag, gridDim.x, want, p.err, &s_ok);
+    if (ok && !one_cluster && blockIdx.x == 0 && threadIdx.x == 0)
+        p.sync[1] = want;  // every CTA read the old generation before it arrived
+    cluster_wait();        // every CTA of the cluster has started (DSMEM is usable)
+    if (one_cluster) {
+        cluster.sync();  // every tile's counts and flags are in its CTA's shared memory
+        // The rows this CTA owns (row % C == c): lane qq of a segment of `width` lanes reads
+        // the count of tile qq; a segmented scan gives each tile's base and the total.
         int width = 1;
         while (width < C)
             width <<= 1;
@@ -774,8 +852,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_group_kernel(const PlanK p)
         for (int i0 = warp * per_warp; i0 < n_own; i0 += kPlanWarps * per_warp) {
             const int i = i0 + slot_in_warp;
             const int row = c + C * i;
-            const bool ok = i < n_own && qq < C;
-            const int32_t v = ok ? cluster.map_shared_rank(q.tc, qq)[row] : 0;
+            const bool own = i < n_own && qq < C;
+            const int32_t v = own ? cluster.map_shared_rank(q.tc, qq)[row] : 0;
             int32_t incl = v;
             for (int o = 1; o < width; o <<= 1) {
                 const int32_t y = __shfl_up_sync(kFull, incl, o, width);
@@ -783,67 +861,86 @@ __global__ void __launch_bounds__(kPlanThreads) plan_group_kernel(const PlanK p)
                     incl += y;
             }
             const int32_t total = __shfl_sync(kFull, incl, width - 1, width);
-            if (ok) {
+            if (own) {
                 cluster.map_shared_rank(q.tb, qq)[row] = incl - v;
-                if (!multi)
-                    cluster.map_shared_rank(q.tot, qq)[row] = total;
-                else if (qq == 0) {
-                    if (row < p.E)
-                        p.tile_cnt[static_cast<int64_t>(g) * p.E + row] = total;
-                    else
-                        p.tile_rcnt[static_cast<int64_t>(g) * p.R + (row - p.E)] = total;
+                cluster.map_shared_rank(q.tot, qq)[row] = total;
+            }
+        }
+        if (c == 0 && threadIdx.x == 0) {
+            uint32_t f = 0u;
+            for (int x = 0; x < C; ++x)
+                f |= *cluster.map_shared_rank(&s_err, x);
+            if (f)
+                atomicOr(p.err, f);
+        }
+    } else if (ok) {
+        // This CTA's rows, one warp per row: a scan over all tiles (coalesced loads of up to
+        // kRounds * 32 tiles at a time); each tile of the cluster gets its prefix, and every
+        // CTA of the cluster the row's total.
+        // A warp takes kRows rows at a time and loads kRounds * 32 tiles of each of them before
+        // scanning any, so that its loads are in flight together.
+        constexpr int kRows = 3, kRounds = 4;
+        const int rpc = (ER + C - 1) / C;
+        const int r_lo = c * rpc, r_hi = min(ER, r_lo + rpc);
+        for (int rb = r_lo + warp * kRows; rb < r_hi; rb += kPlanWarps * kRows) {
+            int32_t carry[kRows];
+#pragma unroll
+            for (int a = 0; a < kRows; ++a)
+                carry[a] = 0;
+            for (int t0 = 0; t0 < p.nt; t0 += 32 * kRounds) {
+                int32_t v[kRows][kRounds];
+#pragma unroll
+                for (int a = 0; a < kRows; ++a) {
+                    const int row = rb + a;
+                    const int32_t *col =
+                        row >= r_hi ? nullptr
+                        : row < p.E ? p.tile_cnt + static_cast<int64_t>(row) * p.nt
+                                    : p.tile_rcnt + static_cast<int64_t>(row - p.E) * p.nt;
+#pragma unroll
+                    for (int rr = 0; rr < kRounds; ++rr) {
+                        const int t = t0 + rr * 32 + lane;
+                        v[a][rr] = col != nullptr && t < p.nt ? __ldcg(col + t) : 0;
+                    }
+                }
+#pragma unroll
+                for (int a = 0; a < kRows; ++a) {
+                    const int row = rb + a;
+#pragma unroll
+                    for (int rr = 0; rr < kRounds; ++rr) {
+                        const int t = t0 + rr * 32 + lane;
+                        int32_t incl = v[a][rr];
+#pragma unroll
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const int32_t y = __shfl_up_sync(kFull, incl, o);
+                            if (lane >= o)
+                                incl += y;
+                        }
+                        if (row < r_hi && t >= t_first && t < t_first + C && t < p.nt)
+                            cluster.map_shared_rank(q.tb, t - t_first)[row] =
+                                carry[a] + incl - v[a][rr];
+                        carry[a] += __shfl_sync(kFull, incl, 31);
+                    }
                 }
             }
+#pragma unroll
+            for (int a = 0; a < kRows; ++a)
+                if (rb + a < r_hi && lane < C)
+                    cluster.map_shared_rank(q.tot, lane)[rb + a] = carry[a];
         }
-    }
-    if (c == 0 && threadIdx.x == 0) {
-        uint32_t f = 0u;
-        for (int qq = 0; qq < C; ++qq)
-            f |= *cluster.map_shared_rank(&s_err, qq);
-        if (multi)
-            p.tile_err[g] = f;
-        else if (f)
-            atomicOr(p.err, f);
-    }
-    if (multi)
-        __threadfence();  // the group's totals are visible GPU-wide before its leader arrives
-    cluster.sync();       // (B) bases and totals are in place; no DSMEM access after this
-
-    if (multi) {
-        uint32_t want = s_gen + 1u;  // s_gen was set before the barriers above
-        if (want == 0u)
-            want = 1u;  // arrival words start at 0: the generation never takes that value
-        if (c == 0 && threadIdx.x == 0)
-            st_release_gpu(&p.group_flag[g], want);
-        if (!wait_words(p.group_flag, G, want, p.err, &s_ok))
-            return;
-        if (blockIdx.x == 0 && threadIdx.x == 0)
-            p.sync[1] = want;  // every CTA read the old generation before its group arrived
-        for (int row = threadIdx.x; row < ER; row += blockDim.x) {
-            const int32_t *col = row < p.E ? p.tile_cnt + row : p.tile_rcnt + (row - p.E);
-            const int stride = row < p.E ? p.E : p.R;
-            int32_t before = 0, total = 0;
-#pragma unroll 8
-            for (uint32_t gg = 0; gg < G; ++gg) {
-                const int32_t v = __ldcg(col + static_cast<int64_t>(gg) * stride);
-                before += static_cast<int>(gg) < g ? v : 0;
-                total += v;
-            }
-            q.tb[row] += before;
-            q.tot[row] = total;
-        }
-        if (blockIdx.x == 0 && threadIdx.x < 32) {
+        if (blockIdx.x == 0 && warp == kPlanWarps - 1) {
             uint32_t f = 0u;
-            for (uint32_t gg = threadIdx.x; gg < G; gg += 32)
-                f |= __ldcg(p.tile_err + gg);
+            for (int t = lane; t < p.nt; t += 32)
+                f |= __ldcg(p.tile_err + t);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
                 f |= __shfl_xor_sync(kFull, f, o);
-            if (threadIdx.x == 0 && f)
+            if (lane == 0 && f)
                 atomicOr(p.err, f);
         }
-        __syncthreads();
     }
+    cluster.sync();  // bases and totals are in place; no DSMEM access after this point
+    if (!ok)
+        return;
     // Only the output stores remain: let the next kernel on the stream start launching.
     pdl_trigger();
 
@@ -858,7 +955,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_group_kernel(const PlanK p)
         if (blockIdx.x == 0)
             p.rcnt[r] = q.tot[p.E + r];
     }
-    prepare_offsets(p, m, warp_sums, q.tot, true);  // synchronises first
+    prepare_offsets(p, m, q.tot, true);  // synchronises first
+    if (ntok == 0)
+        return;  // block-uniform: a CTA past the last tile has nothing to store
     for (int e = threadIdx.x; e < p.E; e += blockDim.x)
         m.ebase[e] = m.eoff[e] + q.tb[e];
     for (int r = threadIdx.x; r < p.R; r += blockDim.x)
@@ -915,7 +1014,6 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
 {
     extern __shared__ __align__(16) int32_t smem[];
     __shared__ uint32_t s_err;
-    __shared__ int32_t warp_sums[kPlanThreads / 32];
     __shared__ int s_ok;
     const PlanSmem m = carve(smem, p.E, p.R, p.k);
     const uint32_t G = gridDim.x;
@@ -983,7 +1081,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_fused_kernel(const PlanK p)
         return;
     pdl_trigger();  // only the rank phase remains: let the next kernel start launching
 
-    rank_prepare(p, m, warp_sums);
+    rank_prepare(p, m);
     // With one tile per CTA the count phase left that tile's classification in smem.
     const bool one_tile = static_cast<int>(G) >= p.nt;
     for (int tile = blockIdx.x; tile < p.nt; tile += G)
@@ -1058,9 +1156,11 @@ namespace {
 
 // How many clusters of the group kernel, `C` CTAs with `smem` bytes each, can be resident at
 // once on `device` (cached: the answer depends only on these).  -1 when the query fails.
-int group_clusters_resident(int C, size_t smem, int device, const cudaLaunchConfig_t *cfg)
+int group_clusters_resident(const void *kernel, int C, size_t smem, int device,
+                            const cudaLaunchConfig_t *cfg)
 {
     struct Fit {
+        const void *kernel;
         int C, device;
         size_t smem;
         int clusters;
@@ -1068,16 +1168,16 @@ int group_clusters_resident(int C, size_t smem, int device, const cudaLaunchConf
     static Fit cache[64];
     static int n_cache = 0;
     for (int i = 0; i < n_cache; ++i)
-        if (cache[i].C == C && cache[i].device == device && cache[i].smem == smem)
+        if (cache[i].kernel == kernel && cache[i].C == C && cache[i].device == device &&
+            cache[i].smem == smem)
             return cache[i].clusters;
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, reinterpret_cast<const void *>(plan_group_kernel),
-                                       cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&c, kernel, cfg) != cudaSuccess) {
         (void)cudaGetLastError();
         c = -1;
     }
     if (n_cache < 64)
-        cache[n_cache++] = {C, device, smem, c};
+        cache[n_cache++] = {kernel, C, device, smem, c};
     return c;
 }
 
@@ -1087,17 +1187,19 @@ int group_clusters_resident(int C, size_t smem, int device, const cudaLaunchConf
 // cooperative cluster launch, the group kernel is not used again on that device.
 bool launch_groups(const PlanK &p, int device, cudaStream_t stream, cudaError_t *err)
 {
-    static int non_portable[64] = {0};  // 1: allowed, -1: refused
-    static int coop_clusters[64] = {0}; // -1: a cooperative cluster launch was refused
+    static int non_portable[64][2] = {};  // 1: allowed, -1: refused
+    static int coop_clusters[64] = {0};   // -1: a cooperative cluster launch was refused
     const int dv = device >= 0 && device < 64 ? device : 0;
     if (coop_clusters[dv] < 0)
         return false;
+    const int wide = p.k > 16 ? 1 : 0;
+    const void *kernel = wide ? reinterpret_cast<const void *>(plan_group_kernel<true>)
+                              : reinterpret_cast<const void *>(plan_group_kernel<false>);
     const size_t smem = sizeof(int32_t) * plan_group_smem_words(p.E, p.R, p.k);
     if (smem > static_cast<size_t>(max_smem_optin(device)))
         return false;
     int per_sm = 0;
-    if (kernel_fit(reinterpret_cast<const void *>(plan_group_kernel), device, kPlanThreads, smem,
-                   &per_sm) != cudaSuccess ||
+    if (kernel_fit(kernel, device, kPlanThreads, smem, &per_sm) != cudaSuccess ||
         per_sm < 1) {
         (void)cudaGetLastError();
         return false;
@@ -1105,36 +1207,46 @@ bool launch_groups(const PlanK &p, int device, cudaStream_t stream, cudaError_t 
     int cmax = tuning().plan_cluster > 0 ? std::min(tuning().plan_cluster, kMaxClusterTiles)
                                          : kMaxClusterTiles;
     if (cmax > 8) {
-        if (non_portable[dv] == 0)
-            non_portable[dv] = cudaFuncSetAttribute(plan_group_kernel,
-                                                    cudaFuncAttributeNonPortableClusterSizeAllowed,
-                                                    1) == cudaSuccess ? 1 : -1;
-        if (non_portable[dv] < 0) {
+        if (non_portable[dv][wide] == 0)
+            non_portable[dv][wide] =
+                cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                        cudaSuccess
+                    ? 1
+                    : -1;
+        if (non_portable[dv][wide] < 0) {
             (void)cudaGetLastError();
             cmax = 8;
         }
     }
-    const int C = std::min(cmax, p.nt);
-    const int G = static_cast<int>(ceil_div(p.nt, C));
+    // The largest cluster size whose clusters can all be resident at once (16 CTAs of a
+    // cluster share one GPC, so a grid of many large clusters may not fit where smaller
+    // clusters do).
+    int C = 0, G = 0;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(G * C));
-    cfg.blockDim = dim3(kPlanThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(C);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (group_clusters_resident(C, smem, device, &cfg) < G)
+    for (int c = std::min(cmax, p.nt); c >= 1 && C == 0; c = c > 8 ? 8 : 0) {
+        const int g = static_cast<int>(ceil_div(p.nt, c));
+        cfg.gridDim = dim3(static_cast<unsigned>(g * c));
+        cfg.blockDim = dim3(kPlanThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(c);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (group_clusters_resident(kernel, c, smem, device, &cfg) >= g) {
+            C = c;
+            G = g;
+        }
+    }
+    if (C == 0)
         return false;
     PlanK arg = p;
     void *args[] = {&arg};
-    const cudaError_t e = launch_ex(reinterpret_cast<const void *>(plan_group_kernel), args,
-                                    cfg.gridDim, cfg.blockDim, smem, stream, G > 1, device, attr,
-                                    1);
+    const cudaError_t e = launch_ex(kernel, args, cfg.gridDim, cfg.blockDim, smem, stream, G > 1,
+                                    device, attr, 1);
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
         if (G > 1)
