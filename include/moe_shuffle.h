@@ -341,9 +341,14 @@ typedef enum {
     MOE_TUNE_PDL = 20,                   /* 0 or 1: kernels are programmatic dependent launches
                                             (each may start while the previous kernel on the
                                             stream finishes), 2: ordinary launches */
-    MOE_TUNE_PLAN_MATCH = 21             /* plan: how a token's ids are compared: 0 by k (match
+    MOE_TUNE_PLAN_MATCH = 21,            /* plan: how a token's ids are compared: 0 by k (match
                                             instructions for k > 16), 1 shuffle compares,
                                             2 warp match instructions */
+    MOE_TUNE_DISPATCH_SPLIT_UNITS = 22,  /* dispatch: below this many (token, chunk) units rows
+                                            are cut into chunks of >= 2 KB (0: 4 per SM;
+                                            1: never) */
+    MOE_TUNE_COMBINE_SPLIT = 23          /* combine: CTAs that share a run of tokens when the
+                                            tokens are few (0: automatic; 1: never) */
 } moe_knob;
 
 MOE_API moe_status moe_tune(moe_knob knob, int32_t value);

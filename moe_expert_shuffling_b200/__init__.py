@@ -38,7 +38,8 @@ KNOBS = {
     "dispatch_units_per_warp": 9, "combine_tokens_per_cta": 10, "plan_engine": 11,
     "fused_ctas_per_sm": 12, "fused_dispatch_share": 13, "fused_dispatch_run": 14,
     "fused_combine_run": 15, "fused_smem_kb": 16, "fused_min_kb": 17, "combine_max_cw": 18,
-    "plan_cluster": 19, "pdl": 20, "plan_match": 21,
+    "plan_cluster": 19, "pdl": 20, "plan_match": 21, "dispatch_split_units": 22,
+    "combine_split": 23,
 }
 PLAN_KINDS = {0: "one_tile", 1: "groups", 2: "cooperative", 3: "three"}
 

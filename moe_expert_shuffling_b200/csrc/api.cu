@@ -270,6 +270,8 @@ moe_status moe_tune(moe_knob knob, int32_t value)
     case MOE_TUNE_PLAN_CLUSTER: t.plan_cluster = value; break;
     case MOE_TUNE_PDL: t.pdl = value; break;
     case MOE_TUNE_PLAN_MATCH: t.plan_match = value; break;
+    case MOE_TUNE_DISPATCH_SPLIT_UNITS: t.dispatch_split_units = value; break;
+    case MOE_TUNE_COMBINE_SPLIT: t.combine_split = value; break;
     default: return fail(MOE_EINVAL, "unknown tuning knob %d", static_cast<int>(knob));
     }
     return ok();

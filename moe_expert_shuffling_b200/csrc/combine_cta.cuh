@@ -69,6 +69,7 @@ struct CombineBulkParams {
     const int32_t *rank_off;  // [R+1] first receive row of each rank (rank-grouped order)
     int32_t R;
     uint32_t ring_bytes;    // bytes of the stage ring (the rank tables follow it)
+    uint32_t csplit;        // CTAs sharing one run of tokens, each taking a range of chunks
 };
 
 // Shared-memory layout of one combine CTA: 2S mbarriers, the ring, then (rank-grouped
@@ -150,15 +151,17 @@ __device__ __forceinline__ bool wait_flag(const uint32_t *flag, uint32_t epoch, 
     return false;
 }
 
-// Producer warp over tokens [b, b + n_tok).  `i` is the ring position (chunks issued so
-// far), carried across runs.  `s_cur` holds lane j's slot of token b (j < k) or -1.  With
+// Producer warp over tokens [b, b + n_tok), chunks [c_lo, c_hi) of each.  `i` is the ring
+// position (chunks issued so far), carried across runs.  `s_cur` holds lane j's slot of token b (j < k) or -1.  With
 // `ready`, token t's rows are read only once ready[t] == epoch (they are being written by
 // the same launch).  Returns false after a timeout (MOE_ERR_TIMEOUT set).
 template <int KMAX, int CW, bool RANKED>
 __device__ __forceinline__ bool combine_produce(const CombineBulkParams &p, const CombineRing &r,
                                                 uint32_t b, int n_tok, int32_t s_cur, int &i,
-                                                const uint32_t *ready, uint32_t epoch)
+                                                const uint32_t *ready, uint32_t epoch,
+                                                uint32_t c_lo = 0u, uint32_t c_hi = ~0u)
 {
+    c_hi = min(c_hi, p.nchunks);
     constexpr uint32_t kChunk_ = Shape<CW>::kChunk;
     const int lane = threadIdx.x & 31;
     const int k = p.k;
@@ -190,7 +193,7 @@ __device__ __forceinline__ bool combine_produce(const CombineBulkParams &p, cons
                 fence_proxy_async_global();
             }
         }
-        for (uint32_t c = 0; c < p.nchunks; ++c, ++i) {
+        for (uint32_t c = c_lo; c < c_hi; ++c, ++i) {
             const int st = i % S;
             const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
             if (!__all_sync(0xffffffffu, mbar_wait_bounded(&r.empty[st], ph ^ 1u))) {
@@ -219,16 +222,18 @@ __device__ __forceinline__ bool combine_produce(const CombineBulkParams &p, cons
     return ok;
 }
 
-// Consumer warps over tokens [b, b + n_tok): thread v owns bytes [16v, 16v + 16) of every
-// chunk.  A token's valid columns (bitmask) and weights are broadcast once per token and
+// Consumer warps over tokens [b, b + n_tok), chunks [c_lo, c_hi) of each: thread v owns bytes
+// [16v, 16v + 16) of every chunk.  A token's valid columns (bitmask) and weights are broadcast once per token and
 // kept in registers; each chunk then costs k shared loads, 8k fmas and one 16-byte store.
 // `s_nxt` / `w_nxt` hold lane j's slot and weight of token b.  Returns false after a
 // timeout (MOE_ERR_TIMEOUT set).
 template <int KMAX, int CW, bool RANKED>
 __device__ __forceinline__ bool combine_consume(const CombineBulkParams &p, const CombineRing &r,
                                                 uint32_t b, int n_tok, int32_t s_nxt,
-                                                float w_nxt, int &i)
+                                                float w_nxt, int &i, uint32_t c_lo = 0u,
+                                                uint32_t c_hi = ~0u)
 {
+    c_hi = min(c_hi, p.nchunks);
     constexpr uint32_t kChunk_ = Shape<CW>::kChunk;
     constexpr int kJ = KMAX < 8 ? KMAX : 8;  // rows held in registers at once
     const int lane = threadIdx.x & 31;
@@ -270,7 +275,7 @@ __device__ __forceinline__ bool combine_consume(const CombineBulkParams &p, cons
             s_nxt = __ldg(p.slot + static_cast<int64_t>(t + 1) * k + lane);
             w_nxt = __ldg(p.w + static_cast<int64_t>(t + 1) * k + lane);
         }
-        for (uint32_t c = 0; c < p.nchunks; ++c, ++i) {
+        for (uint32_t c = c_lo; c < c_hi; ++c, ++i) {
             const int st = i % S;
             const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
             if (!__all_sync(0xffffffffu, mbar_wait_bounded(&r.full[st], ph))) {

@@ -21,6 +21,7 @@ namespace {
 // covers all units beat persistent warps by ~12% (the block scheduler evens out the
 // tail); 4 stages with 2 store groups in flight per warp.
 constexpr int kDefaultUnitsPerWarp = 2;
+constexpr int64_t kSplitUnitsPerSm = 4;
 
 __global__ void __launch_bounds__(128) dispatch_bulk_kernel(const DispatchParams p)
 {
@@ -77,7 +78,18 @@ cudaError_t launch_dispatch(const DispatchArgs &a, int device, cudaStream_t stre
     int wpc = tu.dispatch_warps_per_cta > 0 ? tu.dispatch_warps_per_cta : 1;
     wpc = std::min(std::max(wpc, 1), 4);
 
-    const DispatchGeometry g = dispatch_geometry(a.row_bytes, a.srow_bytes);
+    // Few tokens (a decode-sized batch): cut the rows into more chunks, so that there are
+    // about kSplitUnitsPerSm (token, chunk) units per SM rather than a handful of warps each
+    // moving whole rows.
+    DispatchGeometry g = dispatch_geometry(a.row_bytes, a.srow_bytes);
+    const int64_t split_units = tu.dispatch_split_units == 1 ? 0
+                                : tu.dispatch_split_units > 1
+                                    ? tu.dispatch_split_units
+                                    : static_cast<int64_t>(sm_count(device)) * kSplitUnitsPerSm;
+    if (static_cast<int64_t>(a.N) * g.nchunks < split_units)
+        g = dispatch_geometry(a.row_bytes, a.srow_bytes,
+                              static_cast<uint32_t>(std::min<int64_t>(
+                                  ceil_div(split_units, a.N), 1 << 16)));
     const uint32_t nchunks = g.nchunks, chunk = g.chunk, scale_off = g.scale_off,
                    stage_bytes = g.stage_bytes;
     const bool bulk_scales = g.bulk_scales;

@@ -9,6 +9,8 @@
 // refilled only after the stores that read it have drained (wait_group.read).
 #pragma once
 
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -22,11 +24,21 @@ struct DispatchGeometry {
     bool bulk_scales;  // the scale row rides in the stage (its size is a multiple of 16 B)
 };
 
-inline DispatchGeometry dispatch_geometry(uint32_t row_bytes, uint32_t srow_bytes)
+// `min_chunks` asks for at least that many chunks per row (a decode-sized batch spreads its
+// rows over more warps); chunks stay at least kDispatchMinChunkBytes.
+constexpr uint32_t kDispatchMinChunkBytes = 2048;
+
+inline DispatchGeometry dispatch_geometry(uint32_t row_bytes, uint32_t srow_bytes,
+                                          uint32_t min_chunks = 1)
 {
     DispatchGeometry g;
-    g.nchunks = static_cast<uint32_t>(ceil_div(row_bytes, kDispatchMaxChunkBytes));
-    g.chunk = static_cast<uint32_t>(round_up(ceil_div(row_bytes, g.nchunks), 16));
+    uint32_t n = static_cast<uint32_t>(ceil_div(row_bytes, kDispatchMaxChunkBytes));
+    const uint32_t most = static_cast<uint32_t>(
+        std::max<int64_t>(1, row_bytes / kDispatchMinChunkBytes));
+    if (min_chunks > n)
+        n = std::min(min_chunks, std::max(n, most));
+    g.chunk = static_cast<uint32_t>(round_up(ceil_div(row_bytes, n), 16));
+    g.nchunks = static_cast<uint32_t>(ceil_div(row_bytes, g.chunk));
     g.bulk_scales = srow_bytes > 0 && srow_bytes % 16 == 0;
     g.scale_off = static_cast<uint32_t>(round_up(g.chunk, 128));
     g.stage_bytes =

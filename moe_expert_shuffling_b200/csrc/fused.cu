@@ -264,6 +264,7 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
     c.nchunks = static_cast<uint32_t>(ceil_div(c.row_bytes, chunk));
     c.stage_bytes = static_cast<uint32_t>(a.c.k) * chunk;
     c.per_cta = 0;
+    c.csplit = 1;
     c.rank_off = a.c.rank_off;
     c.R = a.c.R;
 

@@ -77,6 +77,8 @@ struct Tuning {
     int plan_cluster = 0;          // most tiles per cluster of the group plan kernel (1..16)
     int pdl = 0;                   // 0/1: programmatic dependent launch, 2: ordinary launches
     int plan_match = 0;            // 0: by k, 1: shuffle compares, 2: warp match instructions
+    int dispatch_split_units = 0;  // 0: automatic, 1: never cut rows finer, n: below n units
+    int combine_split = 0;         // 0: automatic, 1: never split a token's chunks, n: at most n
 };
 Tuning &tuning();
 

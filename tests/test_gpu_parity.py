@@ -505,3 +505,45 @@ def test_plan_without_dedup_lists(name, N, engine):
     assert not got["rtok"].any() and not got["fanout"].any()
     assert p.check() == 0
     p.close()
+
+
+@pytest.mark.parametrize("knobs", [{}, {"dispatch_split_units": 1, "combine_split": 1},
+                                   {"dispatch_split_units": 100000, "combine_split": 7},
+                                   {"combine_split": 2}],
+                         ids=["auto", "off", "finest", "two"])
+@pytest.mark.parametrize("cfg", [CONFIGS["dsv3"].with_tokens(16), CONFIGS["dsv3"].with_tokens(128),
+                                 CONFIGS["dsv3"].with_tokens(300),
+                                 CONFIGS["long"].with_tokens(100),
+                                 CONFIGS["mixtral"].with_tokens(64),
+                                 CONFIGS["dsv3_k32"].with_tokens(50)],
+                         ids=lambda c: f"{c.name}-N{c.N}")
+def test_small_batch_splits(cfg, knobs):
+    """Decode-sized batches cut rows into smaller dispatch chunks and share a token's column
+    chunks among several combine CTAs; every split gives the oracle's bytes and bits."""
+    import moe_expert_shuffling_b200 as ms
+    idx, w, x, xs, y = make_inputs(cfg, 51)
+    try:
+        for k, v in knobs.items():
+            ms.moe_tune(k, v)
+        p, ti, tw = gpu_plan(idx, w, cfg.E, cfg.R)
+        if cfg.payload == "fp8":
+            recv, rs = ms.moe_dispatch(x, p, x_scale=xs)
+        else:
+            recv, rs = ms.moe_dispatch(x, p), None
+        out = ms.moe_combine(y, p)
+        out_r = ms.moe_combine(y, p, ranked=True)
+        assert p.check() == 0
+    finally:
+        for k in knobs:
+            ms.moe_tune(k, 0)
+    ref = oracle.plan(idx, cfg.E, cfg.R)
+    if cfg.payload == "fp8":
+        want, want_rs = oracle.dispatch(x.cpu().numpy(), ref.slot, xs.cpu().numpy())
+        assert np.array_equal(recv.cpu().numpy(), want)
+        assert np.array_equal(rs.cpu().numpy().view(np.uint8), want_rs)
+    else:
+        want = oracle.dispatch(bits16(x).view(np.uint8).reshape(cfg.N, -1), ref.slot)
+        assert np.array_equal(bits16(recv).view(np.uint8).reshape(cfg.N * cfg.k, -1), want)
+    yb = bits16(y)
+    assert np.array_equal(bits16(out), oracle.combine(yb, ref.slot, w))
+    assert np.array_equal(bits16(out_r), oracle.combine_ranked(yb, ref.slot, w, idx, cfg.E, cfg.R))
