@@ -251,35 +251,44 @@ __device__ __forceinline__ bool grid_barrier(uint32_t *sync, uint32_t *err, uint
     return *s_ok != 0;
 }
 
-// Wait (warp 0 of the CTA) until words[0..n) all hold `want` -- the arrival words that the
-// leader CTA of each group of a grid releases (the group plan kernel).  All threads must
-// call.  False after kWaitLimitNs (MOE_ERR_TIMEOUT set).
+// Wait (one whole warp) until words[0..n) all hold `want` -- the arrival words that the CTAs
+// or groups of a grid release (the group plan kernel).  Relaxed loads, all in flight at once,
+// then one acquire fence.  Returns the same value in every lane; false after kWaitLimitNs
+// (MOE_ERR_TIMEOUT set).
+__device__ __forceinline__ bool wait_words_warp(const uint32_t *words, uint32_t n, uint32_t want,
+                                                uint32_t *err)
+{
+    const uint32_t lane = threadIdx.x & 31u;
+    bool ok = true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        bool mine = true;
+        for (uint32_t q = lane; q < n; q += 32)
+            mine &= ld_relaxed_gpu(words + q) == want;
+        if (__all_sync(0xffffffffu, mine))
+            break;
+        if ((it & 15u) == 15u) {
+            const bool late = global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30);
+            if (__shfl_sync(0xffffffffu, late, 0)) {
+                if (lane == 0)
+                    atomicOr(err, MOE_ERR_TIMEOUT);
+                ok = false;
+                break;
+            }
+        }
+    }
+    // what each arrival released is visible to this CTA from here on
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    return ok;
+}
+
+// wait_words_warp run by warp 0, the result shared with the CTA.  All threads must call.
 __device__ __forceinline__ bool wait_words(const uint32_t *words, uint32_t n, uint32_t want,
                                            uint32_t *err, int *s_ok)
 {
     if (threadIdx.x < 32) {
-        const uint32_t lane = threadIdx.x;
-        bool ok = true;
-        const uint64_t t0 = global_timer_ns();
-        for (uint32_t it = 0;; ++it) {
-            // relaxed loads, all in flight at once; the fence below makes the wait an acquire
-            bool mine = true;
-            for (uint32_t q = lane; q < n; q += 32)
-                mine &= ld_relaxed_gpu(words + q) == want;
-            if (__all_sync(0xffffffffu, mine))
-                break;
-            if ((it & 15u) == 15u) {
-                const bool late = global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30);
-                if (__shfl_sync(0xffffffffu, late, 0)) {
-                    if (lane == 0)
-                        atomicOr(err, MOE_ERR_TIMEOUT);
-                    ok = false;
-                    break;
-                }
-            }
-        }
-        __threadfence();  // what each arrival released is visible to this CTA from here on
-        if (lane == 0)
+        const bool ok = wait_words_warp(words, n, want, err);
+        if (threadIdx.x == 0)
             *s_ok = ok;
     }
     __syncthreads();

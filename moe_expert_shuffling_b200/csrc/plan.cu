@@ -735,8 +735,14 @@ __device__ __forceinline__ void cluster_wait()
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 }
 
-// kWide: rows of more than 16 ids (k > 16); the other instantiation takes k <= 16.
-template <bool kWide>
+// Grids of several clusters and up to this many CTAs wait for the exchange while they stage
+// their tiles (the kEarlyPoll instantiation); larger ones stage first.
+constexpr int kEarlyPollCtas = 256;
+
+// kWide: rows of more than 16 ids (k > 16); the other instantiations take k <= 16.
+// kEarlyPoll: warp 0 waits for the exchange while warps 1..7 stage the tile (grids of several
+// clusters only; a grid of one cluster has no exchange and ignores it).
+template <bool kWide, bool kEarlyPoll>
 __global__ void __launch_bounds__(kPlanThreads, 4) plan_group_kernel(const PlanK p)
 {
     namespace cg = cooperative_groups;
@@ -756,6 +762,8 @@ __global__ void __launch_bounds__(kPlanThreads, 4) plan_group_kernel(const PlanK
     const int tile = static_cast<int>(blockIdx.x);
     const int ntok = tile_tokens(p, tile);  // 0 for the CTAs past the last tile
 
+    const bool one_cluster = static_cast<int>(gridDim.x) == C;
+    const bool early_poll = kEarlyPoll && !one_cluster;
     // Arrive at once on the cluster barrier that is waited on before the first access to
     // another CTA's shared memory (every CTA of the cluster has started by then).
     cluster_arrive_relaxed();
@@ -778,7 +786,6 @@ __global__ void __launch_bounds__(kPlanThreads, 4) plan_group_kernel(const PlanK
     const uint32_t flags = classify_loaded_w<kWide ? 32 : 16>(p, m, ntok);  // syncs first and last
     if (flags)
         atomicOr(&s_err, flags);
-    const bool one_cluster = static_cast<int>(gridDim.x) == C;
     for (int row = threadIdx.x; row < ER; row += blockDim.x) {
         const uint32_t *mk = row < p.E ? &m.emask[4 * row] : &m.rmask[4 * (row - p.E)];
         const int32_t v = __popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3]);
@@ -801,27 +808,34 @@ __global__ void __launch_bounds__(kPlanThreads, 4) plan_group_kernel(const PlanK
         st_release_gpu(&p.group_flag[tile], want);  // every CTA arrives, the last ones too
     }
 
-    // Tile-local offsets and the staging orders (this tile's data only), while the other
-    // tiles arrive.
-    if (threadIdx.x < 32)
-        warp_scan_into(q.tc, p.E, q.loff);
-    else if (threadIdx.x < 64)
-        warp_scan_into(q.tc + p.E, p.R, q.lroff);
-    __syncthreads();
-    {
+    // Tile-local offsets and the staging orders (this tile's data only).  With an early poll,
+    // warp 0 waits for the arrival words meanwhile and warps 1..7 prepare the tile between
+    // themselves (a named barrier joins them).
+    const int w0 = early_poll ? 1 : 0;  // first staging warp
+    const int n_stage = kPlanWarps - w0;
+    if (warp >= w0) {
+        if (warp == w0)
+            warp_scan_into(q.tc, p.E, q.loff);
+        else if (warp == w0 + 1)
+            warp_scan_into(q.tc + p.E, p.R, q.lroff);
+        if (early_poll)
+            asm volatile("bar.sync 1, %0;" ::"r"(n_stage * 32) : "memory");
+        else
+            __syncthreads();
         const LaneMap lm = lane_map(k);
         const int j = lane & ((1 << lm.wbits) - 1);
         const int sub = lane >> lm.wbits;
         int32_t *estage = m.ids;  // the ids are no longer needed: entries by (expert, token)
-        for (int st = 0; st < lm.steps; ++st) {
+        // One (token run, step) pair of the tile.
+        auto stage = [&](int vw, int st) {
             const int tw = st * lm.per_step + sub;
-            const int tl = warp * kPlanTokensPerWarp + tw;
+            const int tl = vw * kPlanTokensPerWarp + tw;
             if (!(tw < kPlanTokensPerWarp && tl < ntok && j < k))
-                continue;
+                return;
             const int i = tl * k + j;
             const int32_t e = m.vid[i];
             if (e < 0)
-                continue;
+                return;
             const int32_t r_e = bits_below(&m.emask[4 * e], tl);
             q.qloc[i] = r_e;
             estage[q.loff[e] + r_e] = (e << 16) | i;
@@ -829,12 +843,32 @@ __global__ void __launch_bounds__(kPlanThreads, 4) plan_group_kernel(const PlanK
                 const int32_t r = m.rank_of[e];
                 q.lstage[q.lroff[r] + bits_below(&m.rmask[4 * r], tl)] = (r << 16) | i;
             }
+        };
+        if (!kEarlyPoll) {
+            for (int st = 0; st < lm.steps; ++st)  // warp w takes token run w
+                stage(warp, st);
+        } else {
+            // the pairs dealt out round robin to the staging warps
+            for (int it = warp - w0; it < kPlanWarps * lm.steps; it += n_stage) {
+                const int vw = it / lm.steps;
+                stage(vw, it - vw * lm.steps);
+            }
         }
+    } else {
+        // warp 0 of an early poll
+        const bool arrived = wait_words_warp(p.group_flag, gridDim.x, want, p.err);
+        if (lane == 0)
+            s_ok = arrived;
     }
-
     // The exchange: every CTA's arrival word holds this launch's generation.  A grid of one
     // cluster needs none: its counts are read from the other CTAs' shared memory.
-    const bool ok = one_cluster || wait_words(p.group_flag, gridDim.x, want, p.err, &s_ok);
+    bool ok = true;
+    if (early_poll) {
+        __syncthreads();  // warp 0's result
+        ok = s_ok != 0;
+    } else if (!one_cluster) {
+        ok = wait_words(p.group_flag, gridDim.x, want, p.err, &s_ok);
+    }
     if (ok && !one_cluster && blockIdx.x == 0 && threadIdx.x == 0)
         p.sync[1] = want;  // every CTA read the old generation before it arrived
     cluster_wait();        // every CTA of the cluster has started (DSMEM is usable)
@@ -1187,37 +1221,48 @@ int group_clusters_resident(const void *kernel, int C, size_t smem, int device,
 // cooperative cluster launch, the group kernel is not used again on that device.
 bool launch_groups(const PlanK &p, int device, cudaStream_t stream, cudaError_t *err)
 {
-    static int non_portable[64][2] = {};  // 1: allowed, -1: refused
+    static int non_portable[64][4] = {};  // per kernel: 1 allowed, -1 refused
     static int coop_clusters[64] = {0};   // -1: a cooperative cluster launch was refused
     const int dv = device >= 0 && device < 64 ? device : 0;
     if (coop_clusters[dv] < 0)
         return false;
     const int wide = p.k > 16 ? 1 : 0;
-    const void *kernel = wide ? reinterpret_cast<const void *>(plan_group_kernel<true>)
-                              : reinterpret_cast<const void *>(plan_group_kernel<false>);
+    const void *const kernels[4] = {reinterpret_cast<const void *>(plan_group_kernel<false, false>),
+                                    reinterpret_cast<const void *>(plan_group_kernel<true, false>),
+                                    reinterpret_cast<const void *>(plan_group_kernel<false, true>),
+                                    reinterpret_cast<const void *>(plan_group_kernel<true, true>)};
     const size_t smem = sizeof(int32_t) * plan_group_smem_words(p.E, p.R, p.k);
     if (smem > static_cast<size_t>(max_smem_optin(device)))
         return false;
-    int per_sm = 0;
-    if (kernel_fit(kernel, device, kPlanThreads, smem, &per_sm) != cudaSuccess ||
-        per_sm < 1) {
-        (void)cudaGetLastError();
-        return false;
-    }
-    int cmax = tuning().plan_cluster > 0 ? std::min(tuning().plan_cluster, kMaxClusterTiles)
-                                         : kMaxClusterTiles;
-    if (cmax > 8) {
-        if (non_portable[dv][wide] == 0)
-            non_portable[dv][wide] =
-                cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-                        cudaSuccess
+    // The kernel's shared-memory limit raised, and its clusters of more than 8 CTAs allowed
+    // (false if it cannot run at all; *big false if clusters stay at 8 CTAs at most).
+    auto prepare = [&](int which, bool *big) {
+        int per_sm = 0;
+        if (kernel_fit(kernels[which], device, kPlanThreads, smem, &per_sm) != cudaSuccess ||
+            per_sm < 1) {
+            (void)cudaGetLastError();
+            return false;
+        }
+        if (non_portable[dv][which] == 0)
+            non_portable[dv][which] =
+                cudaFuncSetAttribute(kernels[which],
+                                     cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                     1) == cudaSuccess
                     ? 1
                     : -1;
-        if (non_portable[dv][wide] < 0) {
+        if (non_portable[dv][which] < 0)
             (void)cudaGetLastError();
-            cmax = 8;
-        }
-    }
+        *big = non_portable[dv][which] > 0;
+        return true;
+    };
+    bool big = false;
+    if (!prepare(wide, &big))
+        return false;
+    const void *kernel = kernels[wide];
+    int cmax = tuning().plan_cluster > 0 ? std::min(tuning().plan_cluster, kMaxClusterTiles)
+                                         : kMaxClusterTiles;
+    if (cmax > 8 && !big)
+        cmax = 8;
     // The largest cluster size whose clusters can all be resident at once (16 CTAs of a
     // cluster share one GPC, so a grid of many large clusters may not fit where smaller
     // clusters do).
@@ -1243,6 +1288,13 @@ bool launch_groups(const PlanK &p, int device, cudaStream_t stream, cudaError_t 
     }
     if (C == 0)
         return false;
+    if (G > 1 && G * C <= kEarlyPollCtas) {
+        // the early-poll instantiation, where it fits the same clusters
+        bool big_e = false;
+        if (prepare(2 + wide, &big_e) && (C <= 8 || big_e) &&
+            group_clusters_resident(kernels[2 + wide], C, smem, device, &cfg) >= G)
+            kernel = kernels[2 + wide];
+    }
     PlanK arg = p;
     void *args[] = {&arg};
     const cudaError_t e = launch_ex(kernel, args, cfg.gridDim, cfg.blockDim, smem, stream, G > 1,
