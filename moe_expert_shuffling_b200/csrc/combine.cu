@@ -21,12 +21,24 @@ namespace moe {
 namespace {
 
 // Measured on B200 (dsv3 and long shapes): a ring of 32-36 KB per CTA, 3 CTAs per SM and
-// short runs of 4 tokens per CTA (the block scheduler evens out the tail) are fastest;
-// deeper rings, more CTAs per SM and persistent CTAs are slower.  The wide shape for
-// k <= 4 (Mixtral) is fastest with runs of 8 tokens.
+// short runs of tokens per CTA (the block scheduler evens out the tail) are fastest;
+// deeper rings, more CTAs per SM and persistent CTAs are slower.  A run moves about 256 KB
+// of rows: graph-replayed steps of the DeepSeek-V3 shape (129 KB per token) took 651 us with
+// runs of 2 tokens against 659 us with 4; top-16 (244 KB per token) 1211 against 1226 us and
+// top-32 (473 KB) 2381 against 2422 us with runs of 1 token against 4; long context (57 KB)
+// is the same from 2 to 4 tokens.  The wide shape for k <= 4 (Mixtral, 24 KB per token)
+// starts from runs of 8 tokens.
 constexpr int kDefaultSmemBudget = 36 * 1024 + 128;
 constexpr int kDefaultCtasPerSm = 3;
 constexpr int kDefaultTokensPerCta = 4;
+constexpr int64_t kRunTargetBytes = 256 * 1024;
+// Below this many waves of resident CTAs the runs change length to fill whole waves, up to
+// kMaxRunBytes of rows read and written per run.  Measured on B200 at the Mixtral shape
+// (k = 2, 24 KB per token; graph-replayed steps): 8192 tokens 75.0 -> 71.8 us, 4096 tokens
+// 40.8 -> 39.0 us, 2048 tokens 27.7 -> 22.3 us.  At the DeepSeek-V3 shape a run of 4 tokens
+// already moves 516 KB, and longer runs were slower (4096 tokens: 186.6 against 189.0 us).
+constexpr int64_t kWholeWavesBelow = 3;
+constexpr int64_t kMaxRunBytes = 512 * 1024;
 
 template <int KMAX, int CW, bool RANKED>
 __global__ void __launch_bounds__(Shape<CW>::kThreads, CW >= 8 ? 2 : 1)
@@ -124,16 +136,36 @@ cudaError_t launch_bulk_shape(const CombineArgs &a, int device, cudaStream_t str
         return e;
     if (per_sm < 1)
         return cudaErrorInvalidConfiguration;
+    // CTAs the device holds at once (what the block scheduler runs as one wave)
+    const int64_t wave = static_cast<int64_t>(sm_count(device)) * per_sm;
     // the default keeps about 12 consumer warps per SM whatever the chunk width
     per_sm = std::min(per_sm, tu.combine_ctas_per_sm > 0 ? tu.combine_ctas_per_sm
                                                           : std::max(1, kDefaultCtasPerSm * 4 / CW));
     // Contiguous runs of tokens per CTA; the grid covers all tokens so that CTAs that
     // finish early are replaced by the block scheduler.
     const int64_t resident = static_cast<int64_t>(sm_count(device)) * per_sm;
-    int64_t per_cta = tu.combine_tokens_per_cta > 0 ? tu.combine_tokens_per_cta
-                                                    : (CW >= 8 ? 2 : 1) * kDefaultTokensPerCta;
-    if (ceil_div(a.N, per_cta) < resident)
+    // A run moves about kRunTargetBytes (at most kDefaultTokensPerCta tokens) in the shapes
+    // for k > 4, and 2 * kDefaultTokensPerCta tokens in the wide shape for k <= 4.
+    const int64_t token_bytes = 2LL * a.H * (a.k + 1);
+    int64_t per_cta = 2 * kDefaultTokensPerCta;
+    if (tu.combine_tokens_per_cta > 0)
+        per_cta = tu.combine_tokens_per_cta;
+    else if (CW < 8)
+        per_cta = std::min<int64_t>(kDefaultTokensPerCta,
+                                    std::max<int64_t>(1, (kRunTargetBytes + token_bytes / 2) /
+                                                             token_bytes));
+    if (ceil_div(a.N, per_cta) < resident) {
         per_cta = std::max<int64_t>(1, ceil_div(a.N, resident));
+    } else if (tu.combine_tokens_per_cta == 0 && ceil_div(a.N, per_cta) < kWholeWavesBelow * wave) {
+        // Fewer than three waves: a last wave that is partly empty costs a large share of the
+        // kernel, so the runs change length until the grid fills whole waves (the count of
+        // waves rounded down; less than one wave is shortened to fill one), as long as a run
+        // moves at most kMaxRunBytes.
+        const int64_t waves = std::max<int64_t>(1, ceil_div(a.N, per_cta) / wave);
+        const int64_t t = ceil_div(a.N, waves * wave);
+        if (t * token_bytes <= kMaxRunBytes)
+            per_cta = t;
+    }
     p.per_cta = static_cast<uint32_t>(per_cta);
     int64_t grid = std::max<int64_t>(1, ceil_div(a.N, per_cta));
     // Few tokens (a decode-sized batch): several CTAs share each run of tokens, each taking a
