@@ -37,7 +37,9 @@ namespace {
 // (independent expert outputs), and dsv3 and Mixtral with y = recv:
 //  * 4 CTAs of 48 KB per SM for CW = 4 consumer warps; narrower chunks (CW = 2, 1) get
 //    proportionally more, smaller CTAs, as the combine kernel does;
-//  * dispatch items of about 256 KB of traffic (2 tokens of the dsv3 shape, 8 of Mixtral);
+//  * dispatch items of about 64 KB of traffic, at least one token (1 token of the dsv3 shape,
+//    2 of long context, 3 of Mixtral), or about 144 KB when the combine waits on flags (6
+//    tokens of Mixtral: smaller items raise the flag traffic);
 //  * combine items of about 512 KB of traffic, at most 4 tokens (half of both when they
 //    wait on flags);
 //  * 10% of the CTAs starting on dispatch (30% when the combine waits on flags: with fewer,
@@ -54,7 +56,11 @@ constexpr int kDefaultDispatchSharePctFlags = 30;
 constexpr int kWideCtasPerSm = 3;
 constexpr int kWideSmemKb = 64;
 constexpr int kWideDispatchSharePct = 30;
-constexpr double kDispatchItemBytes = 256.0 * 1024;
+// Graph-replayed steps with 256 KB dispatch items against the current sizes: long context
+// 857.6 -> 837.5 us, dsv3 639.5 -> 638.6, Mixtral 79.2 -> 75.6 (independent expert outputs)
+// and 78.2 -> 74.1 us (y = recv, flags); top-32 unchanged (one token is already 473 KB).
+constexpr double kDispatchItemBytes = 64.0 * 1024;
+constexpr double kDispatchItemBytesFlags = 144.0 * 1024;
 constexpr double kCombineItemBytes = 512.0 * 1024;
 constexpr uint32_t kMaxCombineRun = 4;
 constexpr int kDispatchStages = 4;
@@ -317,7 +323,10 @@ cudaError_t launch_fused_shape(const FusedArgs &a, int device, cudaStream_t stre
     const double d_token_bytes = static_cast<double>(a.d.row_bytes + a.d.srow_bytes) * (1 + a.d.k);
     uint32_t d_run = tu.fused_dispatch_run > 0
                          ? static_cast<uint32_t>(tu.fused_dispatch_run)
-                         : static_cast<uint32_t>(kDispatchItemBytes / d_token_bytes + 0.5);
+                         : static_cast<uint32_t>((a.use_flags ? kDispatchItemBytesFlags
+                                                              : kDispatchItemBytes) /
+                                                     d_token_bytes +
+                                                 0.5);
     d_run = std::min<uint32_t>(std::max<uint32_t>(d_run, 1), 32);  // one flag per lane
     uint32_t c_run = static_cast<uint32_t>(tu.fused_combine_run);
     if (c_run == 0) {
