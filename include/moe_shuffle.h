@@ -323,12 +323,17 @@ typedef enum {
                                          /* 7: retired */
     MOE_TUNE_COMBINE_SMEM_KB = 8,        /* bulk combine: shared-memory budget per CTA (KB) */
     MOE_TUNE_DISPATCH_UNITS_PER_WARP = 9, /* (token, chunk) units per dispatch warp */
-    MOE_TUNE_COMBINE_TOKENS_PER_CTA = 10, /* tokens per bulk-combine CTA */
+    MOE_TUNE_COMBINE_TOKENS_PER_CTA = 10, /* tokens per bulk-combine CTA (0: runs of about
+                                            256 KB of rows for k > 4, 8 tokens for k <= 4,
+                                            resized to fill whole waves of resident CTAs
+                                            when there are fewer than three) */
     MOE_TUNE_PLAN_ENGINE = 11,           /* 0 or 1: automatic, 2: three kernels, 3: no cluster
                                             kernel (the cooperative one for N > 128) */
     MOE_TUNE_FUSED_CTAS_PER_SM = 12,     /* moe_dispatch_combine: resident CTAs per SM */
     MOE_TUNE_FUSED_DISPATCH_SHARE = 13,  /* moe_dispatch_combine: % of CTAs that start on dispatch */
-    MOE_TUNE_FUSED_DISPATCH_RUN = 14,    /* moe_dispatch_combine: tokens per dispatch work item (1..32) */
+    MOE_TUNE_FUSED_DISPATCH_RUN = 14,    /* moe_dispatch_combine: tokens per dispatch work item
+                                            (1..32; 0: about 64 KB of traffic, 144 KB when
+                                            the combine waits on ready flags) */
     MOE_TUNE_FUSED_COMBINE_RUN = 15,     /* moe_dispatch_combine: tokens per combine work item */
     MOE_TUNE_FUSED_SMEM_KB = 16,         /* moe_dispatch_combine: shared memory per CTA (KB) */
     MOE_TUNE_FUSED_MIN_KB = 17,          /* moe_dispatch_combine: least traffic (KB) for the
