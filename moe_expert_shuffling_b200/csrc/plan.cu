@@ -738,6 +738,11 @@ __device__ __forceinline__ void cluster_wait()
 // Grids of several clusters and up to this many CTAs wait for the exchange while they stage
 // their tiles (the kEarlyPoll instantiation); larger ones stage first.
 constexpr int kEarlyPollCtas = 256;
+// Grids of several clusters with at most kPlanWarps * kLocalRowsPerWarp rows (E + R) and
+// 32 * kLocalRounds tiles scan the tile counts in every CTA rather than spreading the rows
+// over a cluster and exchanging the results through distributed shared memory.
+constexpr int kLocalRowsPerWarp = 4;
+constexpr int kLocalRounds = 4;
 
 // kWide: rows of more than 16 ids (k > 16); the other instantiations take k <= 16.
 // kEarlyPoll: warp 0 waits for the exchange while warps 1..7 stage the tile (grids of several
@@ -764,6 +769,9 @@ __global__ void __launch_bounds__(kPlanThreads, 4) plan_group_kernel(const PlanK
 
     const bool one_cluster = static_cast<int>(gridDim.x) == C;
     const bool early_poll = kEarlyPoll && !one_cluster;
+    // Several clusters but few rows and tiles: every CTA scans the whole table of tile counts.
+    const bool local_rows = !one_cluster && ER <= kPlanWarps * kLocalRowsPerWarp &&
+                            p.nt <= 32 * kLocalRounds;
     // Arrive at once on the cluster barrier that is waited on before the first access to
     // another CTA's shared memory (every CTA of the cluster has started by then).
     cluster_arrive_relaxed();
@@ -907,6 +915,52 @@ __global__ void __launch_bounds__(kPlanThreads, 4) plan_group_kernel(const PlanK
             if (f)
                 atomicOr(p.err, f);
         }
+    } else if (ok && local_rows) {
+        // Few rows and tiles: every CTA reads all of them and takes its own bases and every
+        // total itself, with no distributed shared memory and no closing cluster barrier.
+        // Warp w takes rows w, w + 8, ...; all of its loads are in flight together.
+        int32_t v[kLocalRowsPerWarp][kLocalRounds];
+#pragma unroll
+        for (int a = 0; a < kLocalRowsPerWarp; ++a) {
+            const int row = warp + kPlanWarps * a;
+            const int32_t *col = row >= ER    ? nullptr
+                                 : row < p.E ? p.tile_cnt + static_cast<int64_t>(row) * p.nt
+                                             : p.tile_rcnt + static_cast<int64_t>(row - p.E) * p.nt;
+#pragma unroll
+            for (int rr = 0; rr < kLocalRounds; ++rr) {
+                const int t = rr * 32 + lane;
+                v[a][rr] = col != nullptr && t < p.nt ? __ldcg(col + t) : 0;
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < kLocalRowsPerWarp; ++a) {
+            const int row = warp + kPlanWarps * a;
+            int32_t below = 0, total = 0;
+#pragma unroll
+            for (int rr = 0; rr < kLocalRounds; ++rr) {
+                total += v[a][rr];
+                below += rr * 32 + lane < tile ? v[a][rr] : 0;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                total += __shfl_xor_sync(kFull, total, o);
+                below += __shfl_xor_sync(kFull, below, o);
+            }
+            if (row < ER && lane == 0) {
+                q.tb[row] = below;
+                q.tot[row] = total;
+            }
+        }
+        if (blockIdx.x == 0 && warp == kPlanWarps - 1) {
+            uint32_t f = 0u;
+            for (int t = lane; t < p.nt; t += 32)
+                f |= __ldcg(p.tile_err + t);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                f |= __shfl_xor_sync(kFull, f, o);
+            if (lane == 0 && f)
+                atomicOr(p.err, f);
+        }
     } else if (ok) {
         // This CTA's rows, one warp per row: a scan over all tiles (coalesced loads of up to
         // kRounds * 32 tiles at a time); each tile of the cluster gets its prefix, and every
@@ -972,7 +1026,10 @@ __global__ void __launch_bounds__(kPlanThreads, 4) plan_group_kernel(const PlanK
                 atomicOr(p.err, f);
         }
     }
-    cluster.sync();  // bases and totals are in place; no DSMEM access after this point
+    if (local_rows)
+        __syncthreads();  // this CTA's bases and totals; no other CTA touches its shared memory
+    else
+        cluster.sync();  // bases and totals are in place; no DSMEM access after this point
     if (!ok)
         return;
     // Only the output stores remain: let the next kernel on the stream start launching.
