@@ -34,15 +34,32 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
+    """Compile the library if a source is newer than it (or always, with force).  Processes
+    that start together (one per GPU) take a file lock, so one of them compiles and the
+    others find the library fresh; the output goes to a file of its own and is renamed into
+    place in one step."""
     if not force and not _stale():
         return LIB
-    nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + ".tmp"
-    cmd = [nvcc, *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, *sources(), "-o", tmp]
-    if verbose:
-        print(" ".join(cmd), flush=True)
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    import fcntl
+
+    with open(LIB + ".lock", "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        try:
+            if not force and not _stale():
+                return LIB
+            nvcc = os.environ.get("NVCC", "nvcc")
+            tmp = f"{LIB}.tmp{os.getpid()}"
+            cmd = [nvcc, *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, *sources(), "-o", tmp]
+            if verbose:
+                print(" ".join(cmd), flush=True)
+            try:
+                subprocess.run(cmd, check=True)
+                os.replace(tmp, LIB)
+            finally:
+                if os.path.exists(tmp):
+                    os.remove(tmp)
+        finally:
+            fcntl.flock(lock, fcntl.LOCK_UN)
     return LIB
 
 
