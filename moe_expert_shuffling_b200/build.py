@@ -25,42 +25,44 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    """Compile the library if a source is newer than it (or always, with force).  Processes
-    that start together (one per GPU) take a file lock, so one of them compiles and the
-    others find the library fresh; the output goes to a file of its own and is renamed into
-    place in one step."""
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          out: str | None = None) -> str:
+    """Compile the library (to `out`, default the package's libmoeshuffle.so) if a source is
+    newer than it, or always with force.  Processes that start together (one per GPU) take a
+    file lock, so one of them compiles and the others find the library fresh; the compiler
+    writes a file of its own, which is renamed into place in one step."""
+    lib = out or LIB
+    if not force and not _stale(lib):
+        return lib
     import fcntl
 
-    with open(LIB + ".lock", "w") as lock:
+    with open(lib + ".lock", "w") as lock:
         fcntl.flock(lock, fcntl.LOCK_EX)
         try:
-            if not force and not _stale():
-                return LIB
+            if not force and not _stale(lib):
+                return lib
             nvcc = os.environ.get("NVCC", "nvcc")
-            tmp = f"{LIB}.tmp{os.getpid()}"
+            tmp = f"{lib}.tmp{os.getpid()}"
             cmd = [nvcc, *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, *sources(), "-o", tmp]
             if verbose:
                 print(" ".join(cmd), flush=True)
             try:
                 subprocess.run(cmd, check=True)
-                os.replace(tmp, LIB)
+                os.replace(tmp, lib)
             finally:
                 if os.path.exists(tmp):
                     os.remove(tmp)
         finally:
             fcntl.flock(lock, fcntl.LOCK_UN)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":

@@ -164,3 +164,28 @@ def test_plan_create_ex_rejects_unknown_flags(lib):
     assert lib.moe_plan_create_ex(4, 2, 8, 4, 1, ctypes.c_uint32(2), ctypes.byref(h)) == 1
     assert b"flags" in lib.moe_last_error()
     assert not h.value
+
+
+def test_ranks_started_together_build_the_library_once(tmp_path):
+    """Two processes that need the library at once (two ranks of one node) compile it once:
+    the second waits on the build lock and then finds the first one's library fresh.  The
+    compiler is a stand-in script, so this runs without nvcc or a GPU."""
+    count = tmp_path / "compiles"
+    fake = tmp_path / "fake_nvcc"
+    fake.write_text(
+        "#!/bin/bash\n"
+        f"echo run >> {count}\n"
+        "sleep 1\n"
+        "out=''\n"
+        "while [ $# -gt 0 ]; do if [ \"$1\" = -o ]; then out=$2; fi; shift; done\n"
+        "echo library > \"$out\"\n")
+    fake.chmod(0o755)
+    out = tmp_path / "libtest.so"
+    code = ("import sys; sys.path.insert(0, %r); from moe_expert_shuffling_b200 import build; "
+            "build.build(out=%r)" % (ROOT, str(out)))
+    env = dict(os.environ, NVCC=str(fake))
+    procs = [subprocess.Popen(["python", "-c", code], env=env) for _ in range(2)]
+    assert all(p.wait(timeout=120) == 0 for p in procs)
+    assert count.read_text().splitlines() == ["run"]
+    assert out.read_text() == "library\n"
+    assert not list(tmp_path.glob("libtest.so.tmp*"))
